@@ -1,0 +1,320 @@
+"""Pins of the oracle's router, permutation, GEMM, SwiGLU, combine and bias
+update (CPU only).
+
+Each pin computes the same quantity another way: brute-force enumeration of
+expert and group subsets, exact rational arithmetic, per-element Python loops,
+or a closed form / invariant from "DeepSeek_V3_Report：Annotation"
+(eqs. (12)-(16), "Auxiliary-Loss-Free Load Balancing", "Node-Limited
+Routing", "No Token-Dropping").
+"""
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+
+
+# ---------------------------------------------------------------- routing --
+def _bruteforce_select(beta_row, G, M, K):
+    """Best group subset by enumeration, then best expert subset by enumeration.
+    Scores are exact (fp64 sums of dyadic grid values).  Ties: the subset whose
+    sorted index tuple is lexicographically smallest wins."""
+    E = len(beta_row)
+    gs = E // G
+    if M < G:
+        n = K // M
+        gscore = []
+        for g in range(G):
+            vals = beta_row[g * gs:(g + 1) * gs]
+            gscore.append(max(sum(c) for c in itertools.combinations(vals, n)))
+        best = None
+        for sub in itertools.combinations(range(G), M):
+            sc = sum(gscore[g] for g in sub)
+            if best is None or sc > best[0]:
+                best = (sc, sub)
+        allowed = [e for g in best[1] for e in range(g * gs, (g + 1) * gs)]
+    else:
+        allowed = list(range(E))
+    best = None
+    for sub in itertools.combinations(sorted(allowed), K):
+        sc = sum(beta_row[e] for e in sub)
+        if best is None or sc > best[0]:
+            best = (sc, sub)
+    chosen = list(best[1])
+    chosen.sort(key=lambda e: (-beta_row[e], e))
+    return chosen
+
+
+def _grid_logits(rng, T, E, ties=False):
+    """Logits whose sigmoid+bias lands on a dyadic grid (exact sums): pick the
+    biased score beta on a 1/64 grid and solve for (z, b) with b = 0."""
+    beta = rng.integers(4, 60, (T, E)) / 64.0
+    if ties:
+        beta[:, 1::3] = beta[:, 0::3][:, : beta[:, 1::3].shape[1]]
+    z = np.log(beta / (1.0 - beta))
+    return z, beta
+
+
+@pytest.mark.parametrize("G,M,K", [(4, 2, 4), (4, 4, 4), (8, 4, 8), (2, 1, 2), (1, 1, 3)])
+def test_route_select_matches_bruteforce(G, M, K):
+    rng = np.random.default_rng(10 + G * 7 + M + K)
+    E = 16
+    for ties in (False, True):
+        z, _ = _grid_logits(rng, 60, E, ties)
+        bias = np.zeros(E)
+        idx, gate, info = O.route_select(z, bias, G, M, K)
+        beta = info["beta"]
+        for t in range(z.shape[0]):
+            want = _bruteforce_select(list(beta[t]), G, M, K)
+            assert list(idx[t]) == want, (t, list(idx[t]), want)
+
+
+def test_no_group_limit_is_plain_topk():
+    rng = np.random.default_rng(5)
+    T, E, K = 200, 64, 6
+    z = rng.normal(0, 1, (T, E))
+    b = rng.uniform(-0.05, 0.05, E)
+    idx, _, _ = O.route_select(z, b, 1, 1, K)
+    s = 1.0 / (1.0 + np.exp(-z))
+    for t in range(T):
+        beta = [s[t, e] + b[e] for e in range(E)]
+        want = sorted(range(E), key=lambda e: (-beta[e], e))[:K]
+        assert list(idx[t]) == want
+    # M == G behaves like no limit
+    idx2, _, _ = O.route_select(z, b, 8, 8, K)
+    assert np.array_equal(idx, idx2)
+
+
+def test_sigmoid_against_math_exp():
+    z = np.array([-30.0, -2.5, -1e-3, 0.0, 0.7, 12.0])
+    want = np.array([1.0 / (1.0 + math.exp(-v)) for v in z])
+    assert np.allclose(O.sigmoid(z), want, rtol=1e-15, atol=0)
+
+
+def test_gates_normalised_and_bias_only_selects():
+    rng = np.random.default_rng(6)
+    T, E, G, M, K = 300, 32, 4, 2, 4
+    z = rng.normal(0, 1, (T, E))
+    b0 = np.zeros(E)
+    b1 = rng.uniform(-0.1, 0.1, E)
+    i0, g0, _ = O.route_select(z, b0, G, M, K)
+    i1, g1, info = O.route_select(z, b1, G, M, K)
+    assert np.allclose(g1.sum(axis=1), 1.0, atol=1e-12, rtol=0)
+    s = info["s"]
+    # eq. (13): gates are the raw affinities of the chosen experts, normalised
+    for t in range(T):
+        raw = [s[t, e] for e in i1[t]]
+        assert np.allclose(g1[t], np.array(raw) / sum(raw), rtol=1e-14, atol=0)
+    # eq. (16): the bias changes which experts are chosen, never the gate of a
+    # given chosen set
+    same = [t for t in range(T) if set(i0[t]) == set(i1[t])]
+    assert 0 < len(same) < T
+    for t in same:
+        m0 = dict(zip(i0[t], g0[t]))
+        m1 = dict(zip(i1[t], g1[t]))
+        for e in m0:   # same set, possibly summed in another order
+            assert math.isclose(m0[e], m1[e], rel_tol=2e-15, abs_tol=0)
+
+
+def test_route_with_group_limit_uses_at_most_m_groups():
+    rng = np.random.default_rng(7)
+    T, E, G, M, K = 500, 64, 8, 3, 6
+    z = rng.normal(0, 1, (T, E))
+    idx, _, _ = O.route_select(z, rng.uniform(-0.05, 0.05, E), G, M, K)
+    for t in range(T):
+        assert len(set(idx[t] // (E // G))) <= M
+        assert len(set(idx[t])) == K
+
+
+# ----------------------------------------------------------- permutation --
+def test_permute_bruteforce():
+    rng = np.random.default_rng(8)
+    T, E, K = 97, 12, 3
+    idx = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
+    counts, offsets, src_row, dst_of = O.permute(idx, E)
+    assert counts.sum() == T * K                               # no token dropped
+    slot = 0
+    for e in range(E):
+        toks = [t for t in range(T) if e in idx[t]]            # ascending tokens
+        assert counts[e] == len(toks) and offsets[e] == slot
+        for t in toks:
+            assert src_row[slot] == t
+            k = list(idx[t]).index(e)
+            assert dst_of[t, k] == slot
+            slot += 1
+    assert offsets[E] == T * K
+
+
+def test_mtile_table_bruteforce():
+    offs = np.array([0, 0, 5, 133, 261, 262, 600], np.int64)
+    grp, start = O.mtile_table(offs)
+    want = []
+    for g in range(len(offs) - 1):
+        n = offs[g + 1] - offs[g]
+        want += [g] * math.ceil(n / 128)
+    assert list(grp) == want
+    assert list(start) == [0, 0, 1, 2, 3, 4, 7]
+
+
+# -------------------------------------------------------------------- GEMM --
+def _exact_block_gemm(aq, sa, bq, sb):
+    """D[m][n] = sum_kb sa[m,kb] sb[n/128,kb] sum_k deq(a) deq(b), exactly."""
+    dec = {c: Fraction(float(O.e4m3_decode(np.uint8(c)))) for c in range(256) if c not in (0x7F, 0xFF)}
+    M, K = aq.shape
+    N = bq.shape[0]
+    out = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            tot = Fraction(0)
+            for kb in range(K // 128):
+                part = sum(dec[int(aq[m, k])] * dec[int(bq[n, k])] for k in range(kb * 128, kb * 128 + 128))
+                tot += Fraction(float(sa[m, kb])) * Fraction(float(sb[n // 128, kb])) * part
+            out[m, n] = float(tot)
+    return out
+
+
+def test_grouped_gemm_exact_small():
+    rng = np.random.default_rng(9)
+    K, N = 256, 128
+    aq = rng.integers(0, 0x7E, (5, K)).astype(np.uint8) | (rng.integers(0, 2, (5, K)) << 7).astype(np.uint8)
+    bq = rng.integers(0, 0x7E, (2, N, K)).astype(np.uint8)
+    sa = rng.uniform(0.01, 2, (5, 2)).astype(np.float32)
+    sb = rng.uniform(0.01, 2, (2, 1, 2)).astype(np.float32)
+    offs = np.array([0, 2, 5])
+    got = O.grouped_gemm(aq, sa, bq, sb, offs)
+    cols = [0, 1, 77, 127]
+    want0 = _exact_block_gemm(aq[:2], sa[:2], bq[0][cols], sb[0])
+    want1 = _exact_block_gemm(aq[2:], sa[2:], bq[1][cols], sb[1])
+    assert np.allclose(got[:2][:, cols], want0, rtol=1e-13, atol=1e-13)
+    assert np.allclose(got[2:][:, cols], want1, rtol=1e-13, atol=1e-13)
+
+
+def test_grouped_gemm_integer_operands_exact():
+    # codes whose E4M3 values are small integers, unit scales: exact integers
+    rng = np.random.default_rng(11)
+    ints = {int(v): c for c, v in zip(range(0x7F), O.e4m3_decode(np.arange(0x7F, dtype=np.uint8)))
+            if float(v).is_integer() and 0 < v <= 8}
+    keys = sorted(ints)
+    av = rng.choice(keys, (3, 128))
+    bv = rng.choice(keys, (1, 128, 128))
+    aq = np.vectorize(ints.get)(av).astype(np.uint8)
+    bq = np.vectorize(ints.get)(bv).astype(np.uint8)
+    got = O.grouped_gemm(aq, np.ones((3, 1), np.float32), bq, np.ones((1, 1, 1), np.float32), [0, 3])
+    want = av.astype(np.int64) @ bv[0].T.astype(np.int64)
+    assert np.array_equal(got, want.astype(np.float64))
+
+
+def test_empty_segments_leave_rows_zero():
+    aq = np.full((4, 128), 0x38, np.uint8)       # all 1.0
+    bq = np.full((3, 128, 128), 0x38, np.uint8)
+    sa = np.ones((4, 1), np.float32)
+    sb = np.stack([np.full((1, 1), 2.0 ** i, np.float32) for i in range(3)])
+    got = O.grouped_gemm(aq, sa, bq, sb, [0, 0, 4, 4])
+    assert np.all(got == 128.0 * 2.0)             # every row in segment 1 (scale 2)
+
+
+# ----------------------------------------------------------------- SwiGLU --
+def test_swiglu_layout_and_values():
+    rng = np.random.default_rng(12)
+    I = 256
+    gu = rng.normal(0, 2, (3, 2 * I))
+    h = O.swiglu(gu, I)
+    for r in range(3):
+        for c in (0, 5, 127, 128, 200, 255):
+            j, o = divmod(c, 128)
+            g = gu[r, 256 * j + o]
+            u = gu[r, 256 * j + 128 + o]
+            assert math.isclose(h[r, c], g / (1 + math.exp(-g)) * u, rel_tol=1e-14)
+    assert O.silu(0.0) == 0.0
+    assert math.isclose(float(O.silu(40.0)), 40.0, rel_tol=1e-15)
+    assert abs(float(O.silu(-40.0))) < 1e-15
+
+
+def test_swiglu_quant_roundtrip():
+    rng = np.random.default_rng(13)
+    gu = rng.normal(0, 1, (4, 512)).astype(np.float32)
+    q, s = O.swiglu_quant(gu, 256)
+    assert q.shape == (4, 256) and s.shape == (4, 2)
+    h = O.swiglu(gu, 256)
+    deq = O.dequant_1x128(q, s)
+    assert np.all(np.abs(deq - h) <= np.abs(h) * 2.0 ** -4 + np.repeat(s, 128, 1) * 2.0 ** -9)
+
+
+# ---------------------------------------------------------------- combine --
+def test_combine_bruteforce():
+    rng = np.random.default_rng(14)
+    T, K, d = 5, 3, 8
+    Y = rng.normal(0, 1, (T * K, d))
+    Ys = rng.normal(0, 1, (T, d))
+    u = rng.normal(0, 1, (T, d))
+    dst = np.stack([rng.permutation(T * K)[:K] for _ in range(T)])
+    gate = rng.uniform(0, 1, (T, K))
+    out = O.combine(Y, dst, gate, Ys, u)
+    for t in range(T):
+        for j in range(d):
+            want = u[t, j] + Ys[t, j] + sum(gate[t, k] * Y[dst[t, k], j] for k in range(K))
+            assert math.isclose(out[t, j], want, rel_tol=1e-13, abs_tol=1e-13)
+    # gates summing to 1 over identical rows reproduce that row
+    Yc = np.tile(rng.normal(0, 1, (1, d)), (T * K, 1))
+    g1 = gate / gate.sum(1, keepdims=True)
+    assert np.allclose(O.combine(Yc, dst, g1, None, np.zeros((T, d))), np.tile(Yc[:1], (T, 1)))
+
+
+# ------------------------------------------------------------ bias update --
+def test_bias_update_hand_example():
+    counts = np.array([3, 1, 2, 2])               # T=2, K=4, E=4: mean load 2
+    b = np.array([0.01, -0.02, 0.03, 0.0], np.float32)
+    nb = O.bias_update(counts, 2, 4, 0.001, b)
+    g = np.float32(0.001)
+    assert nb.dtype == np.float32
+    assert nb[0] == np.float32(b[0] - g)          # overloaded: minus gamma
+    assert nb[1] == np.float32(b[1] + g)          # underloaded: plus gamma
+    assert nb[2] == b[2] and nb[3] == b[3]        # at the mean: unchanged
+
+
+def test_bias_update_fp32_exact():
+    rng = np.random.default_rng(15)
+    E = 256
+    counts = rng.integers(0, 300, E)
+    b = rng.uniform(-0.05, 0.05, E).astype(np.float32)
+    nb = O.bias_update(counts, 4096, 8, 0.001, b)
+    mean = 4096 * 8 / E
+    for i in range(E):
+        if counts[i] > mean:
+            assert nb[i] == np.float32(b[i]) - np.float32(0.001)
+        elif counts[i] < mean:
+            assert nb[i] == np.float32(b[i]) + np.float32(0.001)
+        else:
+            assert nb[i] == b[i]
+
+
+# ----------------------------------------------------------- whole layer --
+def test_tiny_layer_invariants():
+    from fp8_block_scaled_sigmoid_b200 import configs, inputs
+    cfg = configs.TINY
+    inp = inputs.draw_layer(cfg)
+    u = inp["u"].float().numpy()
+    w1q, w1s, w2q, w2s = O.quantise_weights(inp["w1"].float().numpy(), inp["w2"].float().numpy())
+    r = O.moe_layer(u, inp["centroids"].float().numpy(), inp["bias"].numpy(),
+                    w1q, w1s, w2q, w2s, cfg.G, cfg.M, cfg.K, cfg.gamma)
+    T, K = cfg.T, cfg.K
+    assert r["counts"].sum() == T * K
+    assert np.allclose(r["gate"].sum(1), 1.0)
+    # eq. (12) rebuilt from the per-row expert outputs
+    Y = r["Y"]
+    out = u.astype(np.float64) + Y[T * K:]
+    for t in range(T):
+        for k in range(K):
+            out[t] += r["gate"][t, k] * Y[r["dst_of"][t, k]]
+    assert np.allclose(out, r["out"], rtol=1e-12, atol=1e-12)
+    # the expert outputs of token t under expert e equal the dense FFN of t
+    t, k = 3, 1
+    e = r["idx"][t, k]
+    x = O.dequant_1x128(r["xq_tok"][t:t + 1], r["xs_tok"][t:t + 1])
+    gu = x @ O.dequant_128x128(w1q[e], w1s[e]).T
+    hq, hs = O.swiglu_quant(gu, cfg.I)
+    y = O.dequant_1x128(hq, hs) @ O.dequant_128x128(w2q[e], w2s[e]).T
+    assert np.allclose(y[0], Y[r["dst_of"][t, k]], rtol=1e-12, atol=1e-12)
