@@ -1,0 +1,431 @@
+"""Benchmark: MoE-layer tokens/s of the V3-shaped prefill layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config v3_prefill]
+                    [--impl reference] [--no-cpu-baseline]
+
+One step = one forward pass of the whole layer (route, 1x128 quantisation,
+permutation, grouped GEMM 1 with fused SwiGLU + requantisation, grouped
+GEMM 2, combine, bias update) over one batch of T tokens, with the FP8
+weights already resident (they are quantised once, before timing).  With N
+GPUs (torchrun, one process per GPU) every rank runs its own batch of T
+tokens over the full expert set and the per-expert load counts are summed
+with an NCCL all-reduce before the bias update (weak scaling).
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream; between steps a 512 MB buffer is overwritten to
+flush the 126 MB L2 (outside the events).  The reported time is the max over
+ranks of the summed step times.  Clocks are sampled with nvidia-smi during
+the timed region.
+
+``--impl reference`` times the CPU oracle instead (rank 0 only) on a bounded
+sample of the same workload and prints the same JSON line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s on 1 B200; grouped FP8 GEMM TFLOPS as % of peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_name(cfg) -> str:
+    lim = f"G={cfg.G} M={cfg.M}" if cfg.M < cfg.G else "no group limit"
+    return (f"{cfg.name}: DeepSeekMoE layer forward, T={cfg.T} d={cfg.d} E={cfg.E} routed "
+            f"({lim}) top-{cfg.K} +{cfg.n_shared} shared, SwiGLU I={cfg.I}, FP8 E4M3 1x128 "
+            f"activations / 128x128 weights")
+
+
+# --------------------------------------------------------------- clocks ---
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------- CPU oracle leg ---
+def oracle_sample_rate(cfg, u_host, cent_host, bias_host, expert_weights, route_tokens,
+                       ffn_tokens):
+    """Time the oracle on a bounded sample of the layer and return
+    (seconds per token, description).  Route + 1x128 quantisation +
+    permutation + bias update run over ``route_tokens`` tokens; the expert
+    FFNs (routed and shared) and the combine over ``ffn_tokens`` of them.
+    ``expert_weights(e)`` returns the quantised (w1q, w1s, w2q, w2s) of one
+    expert as numpy arrays (weight preparation is not timed, as on the GPU)."""
+    import numpy as np
+    from oracle import moe_oracle as O
+
+    ur = u_host[:route_tokens]
+    t0 = time.perf_counter()
+    idx, gate, _ = O.route(ur, cent_host, bias_host, cfg.G, cfg.M, cfg.K)
+    xq, xs = O.quant_1x128(ur)
+    counts, offsets, src_row, dst_of = O.permute(idx, cfg.E)
+    _ = xq[src_row], xs[src_row]
+    O.bias_update(counts, route_tokens, cfg.K, cfg.gamma, bias_host)
+    t_route = time.perf_counter() - t0
+    # expert FFNs of the sampled tokens, one expert at a time
+    t_ffn = 0.0
+    for t in ffn_tokens:
+        x = O.dequant_1x128(xq[t:t + 1], xs[t:t + 1])
+        ys = []
+        for e in [cfg.E] + list(idx[t]):
+            w1q, w1s, w2q, w2s = expert_weights(int(e))
+            t1 = time.perf_counter()
+            gu = x @ O.dequant_128x128(w1q, w1s).T
+            hq, hs = O.swiglu_quant(gu, cfg.I)
+            ys.append(O.dequant_1x128(hq, hs) @ O.dequant_128x128(w2q, w2s).T)
+            t_ffn += time.perf_counter() - t1
+        t1 = time.perf_counter()
+        Y = np.concatenate(ys[1:])
+        O.combine(Y, np.arange(cfg.K)[None, :], gate[t:t + 1], ys[0], ur[t:t + 1])
+        t_ffn += time.perf_counter() - t1
+    per_token = t_route / route_tokens + t_ffn / len(ffn_tokens)
+    desc = (f"route+quant+permute+bias-update over {route_tokens} tokens "
+            f"({t_route:.2f} s); expert FFNs ({cfg.K} routed + 1 shared) + combine for "
+            f"{len(ffn_tokens)} token(s) ({t_ffn:.2f} s); rate = 1/(route time per token + "
+            f"FFN time per token)")
+    return per_token, desc
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------- GPU arm ---
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from fp8_block_scaled_sigmoid_b200 import _abi, configs, inputs
+    from fp8_block_scaled_sigmoid_b200.layer import MoELayer, make_fp8_weights
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist.group.WORLD
+
+    cfg = configs.PRESETS[args.config]
+    cfg_rank = cfg.with_(seed=cfg.seed + rank)       # each rank its own token batch
+    w1q, w1s, w2q, w2s = make_fp8_weights(cfg, dev)  # same weights on every rank
+    cent = inputs.draw_centroids(cfg, dev)
+    bias = inputs.draw_bias(cfg, dev)
+    u = inputs.draw_u(cfg_rank, dev)
+    layer = MoELayer(cfg, cent, bias.clone(), w1q, w1s, w2q, w2s, process_group=pg)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+
+    def barrier():
+        if pg is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        layer.forward(u)
+    barrier()
+    layer.check()
+
+    names = ["route", "quant", "permute", "gemm1", "gemm2", "combine", "bias"]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+          for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    barrier()
+    lc0 = _abi.launch_count
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e = ev[i]
+        e[0].record(st)
+        layer.step_route(u)
+        e[1].record(st)
+        layer.step_quant(u)
+        e[2].record(st)
+        layer.step_permute()
+        e[3].record(st)
+        layer.step_gemm1()
+        e[4].record(st)
+        layer.step_gemm2()
+        e[5].record(st)
+        layer.step_combine(u)
+        e[6].record(st)
+        layer.step_bias_update()
+        e[7].record(st)
+    barrier()
+    launches = _abi.launch_count - lc0
+    clocks = sampler.stop() if sampler else None
+    layer.check()
+    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
+    per_kernel = {n: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)) / args.steps
+                  for j, n in enumerate(names)}
+    total_ms = sum(step_ms)
+    if pg is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    tokens = cfg.T * world * args.steps
+    value = tokens / (total_ms / 1e3)
+
+    # end to end through the public API with pinned host buffers
+    u_host = u.cpu().pin_memory()
+    out_host = torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory()
+    for _ in range(2):
+        layer.forward_host(u_host, out_host)
+    barrier()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e2e_ev[i][0].record(st)
+        layer.forward_host(u_host, out_host)
+        e2e_ev[i][1].record(st)
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    if pg is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = tokens / (e2e_ms / 1e3)
+
+    # roofline of the dominant kernel (grouped GEMM 1 with the SwiGLU epilogue)
+    counts = layer.perm["counts"].cpu()
+    active = int((counts > 0).sum()) + cfg.n_shared
+    rows = cfg.pairs + cfg.T
+    w1_bytes = active * 2 * cfg.I * cfg.d * (1 + 4.0 / (128 * 128))
+    a_bytes = rows * cfg.d * (1 + 4.0 / 128)
+    h_bytes = rows * cfg.I * (1 + 4.0 / 128)
+    g1_bytes = w1_bytes + a_bytes + h_bytes
+    w2_bytes = active * cfg.I * cfg.d * (1 + 4.0 / (128 * 128))
+    g2_bytes = w2_bytes + rows * cfg.I * (1 + 4.0 / 128) + rows * cfg.d * 4
+    g1_flops = 2.0 * rows * cfg.d * 2 * cfg.I
+    g2_flops = 2.0 * rows * cfg.I * cfg.d
+    t1 = per_kernel["gemm1"] / 1e3
+    t2 = per_kernel["gemm2"] / 1e3
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fp8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = g1_bytes / t1 / 1e9
+    traffic = read_traffic("grouped_gemm_fp8", cfg.name)
+    roofline = {"kernel": "grouped_gemm_fp8 (GEMM 1, SwiGLU+quant epilogue)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": traffic,
+                "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured"
+                else "fallback 6650 GB/s",
+                "algorithmic_bytes": int(g1_bytes)}
+    gemm = {"gemm1_tflops": round(g1_flops / t1 / 1e12, 1),
+            "gemm2_tflops": round(g2_flops / t2 / 1e12, 1),
+            "gemm1_gbs": round(achieved, 1), "gemm2_gbs": round(g2_bytes / t2 / 1e9, 1),
+            "layer_gemm_tflops": round((g1_flops + g2_flops) / (t1 + t2) / 1e12, 1),
+            "fp8_peak_tflops": fp8_peak,
+            "frac_fp8_peak": round((g1_flops + g2_flops) / (t1 + t2) / 1e12 / fp8_peak, 4),
+            "fp8_peak_note": "2 x measured bf16 burst (nominal fp8:bf16 ratio)"}
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
+        "data": "synthetic (seeded; random-init weights of the V3-shaped layer)",
+        "config": {"workload": workload_name(cfg), "tokens_per_gpu": cfg.T,
+                   "parallelism": f"dp{world} (full expert set per GPU, load counts all-reduced)"
+                   if world > 1 else "single GPU",
+                   "l2": "512 MB buffer written between timed steps; FP8 weights (11.3 GB) > L2"},
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(u_host.numel() * u_host.element_size()),
+                "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size())},
+        "gpu_launches": launches,
+        "roofline": roofline,
+        "gemm": gemm,
+        "kernel_ms": {k: round(v, 4) for k, v in per_kernel.items()},
+        "loads": {"max": int(counts.max()), "mean": float(counts.float().mean()),
+                  "active_experts": active - cfg.n_shared},
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cfg, layer, u, bias)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if pg is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def read_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(f"{kernel}/{workload}")
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "fp8_block_scaled_sigmoid_b200", "csrc", ent.get("source", ""))
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return ent["bytes_per_launch"] if h == ent.get("source_sha256_16") else None
+
+
+def cpu_baseline(cfg, layer, u, bias):
+    import numpy as np
+    import torch
+    u_h = u.float().cpu().numpy()
+    cent_h = layer.centroids.float().cpu().numpy()
+    b_h = bias.cpu().numpy()
+
+    def weights(e):
+        return (layer.w1q[e].cpu().numpy(), layer.w1s[e].cpu().numpy(),
+                layer.w2q[e].cpu().numpy(), layer.w2s[e].cpu().numpy())
+
+    route_tokens = min(cfg.T, 2048)
+    per_token, desc = oracle_sample_rate(cfg, u_h, cent_h, b_h, weights, route_tokens, [0])
+    return {"value": round(1.0 / per_token, 3), "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle", "sample": desc}
+
+
+# ------------------------------------------------------- reference arm ---
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    from fp8_block_scaled_sigmoid_b200 import configs, inputs
+    from oracle import moe_oracle as O
+
+    cfg = configs.PRESETS[args.config]
+    u = inputs.draw_u(cfg).float().numpy()
+    cent = inputs.draw_centroids(cfg).float().numpy()
+    bias = inputs.draw_bias(cfg).numpy()
+    cache = {}
+
+    def weights(e):
+        if e not in cache:       # weight preparation (not timed)
+            w1 = inputs.draw_w1(cfg, e).float().numpy()
+            w2 = inputs.draw_w2(cfg, e).float().numpy()
+            cache[e] = O.quant_128x128(w1) + O.quant_128x128(w2)
+        return cache[e]
+
+    route_tokens = min(cfg.T, 256)
+    # prepare the sampled token's experts before timing
+    idx0, _, _ = O.route(u[:1], cent, bias, cfg.G, cfg.M, cfg.K)
+    for e in [cfg.E] + list(idx0[0]):
+        weights(int(e))
+    times, desc = [], ""
+    for i in range(args.warmup + args.steps):
+        per_token, desc = oracle_sample_rate(cfg, u, cent, bias, weights, route_tokens, [0])
+        if i >= args.warmup:
+            times.append(per_token)
+    per_token = sum(times) / len(times)
+    value = 1.0 / per_token
+    cb = {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+          "sample": desc}
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(per_token * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": workload_name(cfg), "tokens_per_gpu": cfg.T,
+                   "parallelism": "CPU oracle, rank 0 only"},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="v3_prefill")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,296 @@
+"""ctypes binding of libmoefp8.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+tensors that already live on the GPU, passes their raw pointers and sizes,
+and raises MoEError on a non-zero status.  Output tensors are allocated with
+torch when the caller does not pass them (device memory is torch's job; all
+arithmetic happens in the library's kernels).  There is no fallback: if the
+library is missing or a CUDA device is absent the call fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoefp8.so")
+
+_c = ctypes
+_p = _c.c_void_p
+_i = _c.c_int
+_i64 = _c.c_int64
+_sz = _c.c_size_t
+_f = _c.c_float
+
+_SIGS = {
+    "moe_status_string": (_c.c_char_p, [_i]),
+    "moe_abi_version": (_i, []),
+    "fp8_quant_1x128": (_i, [_p, _i64, _i, _i, _p, _p, _p]),
+    "fp8_quant_128x128": (_i, [_p, _i64, _i, _i, _p, _p, _p]),
+    "moe_route_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
+    "moe_route": (_i, [_p, _i64, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _sz, _p, _p]),
+    "moe_max_m_tiles": (_i, [_i, _i, _i, _i]),
+    "moe_permute_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
+    "moe_permute": (_i, [_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                         _p, _sz, _p, _p]),
+    "moe_tile_table": (_i, [_p, _i, _i, _p, _p, _p, _p, _p]),
+    "grouped_gemm_fp8_blockscaled": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
+                                          _i, _p, _p, _p, _p]),
+    "swiglu_quant": (_i, [_p, _i, _i, _p, _p, _p]),
+    "moe_combine": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
+    "moe_bias_update": (_i, [_p, _i, _i64, _i, _f, _p, _p]),
+}
+
+EP_F32 = 0
+EP_SWIGLU_QUANT = 1
+DEVERR = {0: "none", 1: "bounded wait timed out", 2: "inconsistent segment table",
+          3: "expert index out of range"}
+
+_lib = None
+
+# Kernels each entry point launches (for the benchmark's launch count).
+LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant": 1,
+                     "moe_route": 2, "moe_permute": 4, "moe_tile_table": 1,
+                     "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1}
+launch_count = 0
+
+
+def _count(name: str) -> None:
+    global launch_count
+    launch_count += LAUNCHES_PER_CALL[name]
+
+
+class MoEError(RuntimeError):
+    pass
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoefp8.so (built in-tree by ``python -m fp8_block_scaled_sigmoid_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise MoEError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m fp8_block_scaled_sigmoid_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def exported_symbols() -> list[str]:
+    return list(_SIGS)
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        msg = lib().moe_status_string(status).decode()
+        raise MoEError(f"{what}: status {status} ({msg})")
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise MoEError("expected a CUDA tensor")
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dev(t):
+    return t.device
+
+
+# ----------------------------------------------------------------- quant ---
+def fp8_quant_1x128(x, q=None, scale=None, stream=None):
+    """x bf16 [rows][cols] (row stride may exceed cols) -> (q uint8, scale fp32)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    q = torch.empty(rows, cols, dtype=torch.uint8, device=_dev(x)) if q is None else q
+    scale = torch.empty(rows, cols // 128, dtype=torch.float32, device=_dev(x)) if scale is None else scale
+    _count("fp8_quant_1x128")
+    _check(lib().fp8_quant_1x128(_ptr(x), x.stride(0), rows, cols, _ptr(q), _ptr(scale),
+                                 _stream(stream)), "fp8_quant_1x128")
+    return q, scale
+
+
+def fp8_quant_128x128(w, q=None, scale=None, stream=None):
+    """w bf16 [rows][cols] or a stack [G][N][K] (N % 128 == 0) -> (q, scale)
+    with scale [ceil(rows/128)][cols/128] (stack: [G][N/128][K/128])."""
+    assert w.dtype == torch.bfloat16 and w.stride(-1) == 1
+    shape = w.shape
+    w2 = w.reshape(-1, shape[-1])
+    rows, cols = w2.shape
+    if w.dim() == 3:
+        assert shape[1] % 128 == 0
+        sshape = (shape[0], shape[1] // 128, cols // 128)
+    else:
+        sshape = ((rows + 127) // 128, cols // 128)
+    q = torch.empty(shape, dtype=torch.uint8, device=_dev(w)) if q is None else q
+    scale = torch.empty(sshape, dtype=torch.float32, device=_dev(w)) if scale is None else scale
+    _count("fp8_quant_128x128")
+    _check(lib().fp8_quant_128x128(_ptr(w2), w2.stride(0), rows, cols, _ptr(q), _ptr(scale),
+                                   _stream(stream)), "fp8_quant_128x128")
+    return q, scale
+
+
+def swiglu_quant(gu, I, h=None, h_scale=None, stream=None):
+    rows = gu.shape[0]
+    h = torch.empty(rows, I, dtype=torch.uint8, device=_dev(gu)) if h is None else h
+    h_scale = torch.empty(rows, I // 128, dtype=torch.float32, device=_dev(gu)) if h_scale is None else h_scale
+    _count("swiglu_quant")
+    _check(lib().swiglu_quant(_ptr(gu), rows, I, _ptr(h), _ptr(h_scale), _stream(stream)),
+           "swiglu_quant")
+    return h, h_scale
+
+
+# ----------------------------------------------------------------- route ---
+def moe_route_workspace_size(T, d, E) -> int:
+    n = _sz(0)
+    _check(lib().moe_route_workspace_size(T, d, E, ctypes.byref(n)), "moe_route_workspace_size")
+    return n.value
+
+
+def moe_route(u, centroids, bias, G, M, K, topk_idx=None, topk_gate=None, logits_out=None,
+              ws=None, dev_err=None, stream=None):
+    T, d = u.shape
+    E = centroids.shape[0]
+    dev = _dev(u)
+    topk_idx = torch.empty(T, K, dtype=torch.int32, device=dev) if topk_idx is None else topk_idx
+    topk_gate = torch.empty(T, K, dtype=torch.float32, device=dev) if topk_gate is None else topk_gate
+    need = moe_route_workspace_size(T, d, E)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _count("moe_route")
+    _check(lib().moe_route(_ptr(u), u.stride(0), _ptr(centroids), _ptr(bias), T, d, E, G, M, K,
+                           _ptr(topk_idx), _ptr(topk_gate), _ptr(logits_out), _ptr(ws),
+                           ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream)),
+           "moe_route")
+    return topk_idx, topk_gate
+
+
+# --------------------------------------------------------------- permute ---
+def moe_max_m_tiles(T, K, E, with_shared) -> int:
+    return lib().moe_max_m_tiles(T, K, E, int(bool(with_shared)))
+
+
+def moe_permute_workspace_size(T, K, E) -> int:
+    n = _sz(0)
+    _check(lib().moe_permute_workspace_size(T, K, E, ctypes.byref(n)), "moe_permute_workspace_size")
+    return n.value
+
+
+def moe_permute(topk_idx, E, xq, xscale, with_shared=True, out=None, ws=None, dev_err=None,
+                stream=None):
+    """Returns a dict of the outputs (allocated here unless ``out`` holds them).
+    xq_perm needs T*K rows at least; for the layer the caller passes a buffer
+    of T*K+T rows whose tail already holds xq."""
+    T, K = topk_idx.shape
+    d = xq.shape[1]
+    dev = _dev(topk_idx)
+    groups = E + (1 if with_shared else 0)
+    o = {} if out is None else out
+    mt = moe_max_m_tiles(T, K, E, with_shared)
+
+    def get(name, shape, dtype):
+        if name not in o:
+            o[name] = torch.empty(shape, dtype=dtype, device=dev)
+        return o[name]
+
+    counts = get("counts", (E,), torch.int32)
+    offsets = get("offsets", (groups + 1,), torch.int32)
+    src_row = get("src_row", (T * K,), torch.int32)
+    dst_of = get("dst_of", (T, K), torch.int32)
+    xq_perm = get("xq_perm", (T * K, d), torch.uint8)
+    xs_perm = get("xs_perm", (T * K, d // 128), torch.float32)
+    tile_group = get("tile_group", (max(mt, 1),), torch.int32)
+    tile_start = get("tile_start", (groups + 1,), torch.int32)
+    n_tiles = get("n_tiles", (1,), torch.int32)
+    need = moe_permute_workspace_size(T, K, E)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _count("moe_permute")
+    _check(lib().moe_permute(_ptr(topk_idx), T, K, E, int(bool(with_shared)), _ptr(xq),
+                             _ptr(xscale), d, _ptr(counts), _ptr(offsets), _ptr(src_row),
+                             _ptr(dst_of), _ptr(xq_perm), _ptr(xs_perm), _ptr(tile_group),
+                             _ptr(tile_start), _ptr(n_tiles), _ptr(ws),
+                             ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream)),
+           "moe_permute")
+    o["max_tiles"] = mt
+    return o
+
+
+def moe_tile_table(offsets, max_tiles, tile_group=None, tile_start=None, n_tiles=None,
+                   dev_err=None, stream=None):
+    groups = offsets.numel() - 1
+    dev = _dev(offsets)
+    tile_group = torch.empty(max(max_tiles, 1), dtype=torch.int32, device=dev) if tile_group is None else tile_group
+    tile_start = torch.empty(groups + 1, dtype=torch.int32, device=dev) if tile_start is None else tile_start
+    n_tiles = torch.empty(1, dtype=torch.int32, device=dev) if n_tiles is None else n_tiles
+    _count("moe_tile_table")
+    _check(lib().moe_tile_table(_ptr(offsets), groups, max_tiles, _ptr(tile_group),
+                                _ptr(tile_start), _ptr(n_tiles), _ptr(dev_err), _stream(stream)),
+           "moe_tile_table")
+    return tile_group, tile_start, n_tiles
+
+
+# ------------------------------------------------------------------ GEMM ---
+def grouped_gemm_fp8_blockscaled(A, sa, B, sb, offsets, tile_group, tile_start, n_tiles,
+                                 max_tiles, ep=EP_F32, D=None, d_scale=None, dev_err=None,
+                                 stream=None):
+    """A uint8 [rows][K], sa fp32 [rows][K/128], B uint8 [G][N][K], sb fp32
+    [G][N/128][K/128].  ep=EP_F32 -> D fp32 [rows][N]; ep=EP_SWIGLU_QUANT ->
+    (h uint8 [rows][N/2], h_scale fp32 [rows][N/256])."""
+    rows, K = A.shape
+    G, N, _ = B.shape
+    dev = _dev(A)
+    if ep == EP_F32:
+        D = torch.zeros(rows, N, dtype=torch.float32, device=dev) if D is None else D
+    else:
+        D = torch.empty(rows, N // 2, dtype=torch.uint8, device=dev) if D is None else D
+        d_scale = torch.empty(rows, N // 256, dtype=torch.float32, device=dev) if d_scale is None else d_scale
+    _count("grouped_gemm_fp8_blockscaled")
+    _check(lib().grouped_gemm_fp8_blockscaled(_ptr(A), _ptr(sa), rows, _ptr(B), _ptr(sb),
+                                              _ptr(offsets), _ptr(tile_group), _ptr(tile_start),
+                                              _ptr(n_tiles), max_tiles, G, N, K, ep, _ptr(D),
+                                              _ptr(d_scale), _ptr(dev_err), _stream(stream)),
+           "grouped_gemm_fp8_blockscaled")
+    return D if ep == EP_F32 else (D, d_scale)
+
+
+# --------------------------------------------------------- combine / bias ---
+def moe_combine(Y, dst_of, topk_gate, Y_shared, u, out=None, stream=None):
+    T, d = u.shape
+    K = dst_of.shape[1]
+    out = torch.empty(T, d, dtype=torch.float32, device=_dev(u)) if out is None else out
+    _count("moe_combine")
+    _check(lib().moe_combine(_ptr(Y), _ptr(dst_of), _ptr(topk_gate), _ptr(Y_shared), _ptr(u),
+                             T, K, d, _ptr(out), _stream(stream)), "moe_combine")
+    return out
+
+
+def moe_bias_update(counts, T, K, gamma, bias, stream=None):
+    E = counts.numel()
+    _count("moe_bias_update")
+    _check(lib().moe_bias_update(_ptr(counts), E, T, K, float(gamma), _ptr(bias),
+                                 _stream(stream)), "moe_bias_update")
+    return bias
+
+
+def read_dev_err(dev_err) -> int:
+    v = int(dev_err.item())
+    return v
+
+
+def raise_dev_err(dev_err) -> None:
+    v = read_dev_err(dev_err)
+    if v != 0:
+        raise MoEError(f"device-side error {v}: {DEVERR.get(v, 'unknown')}")

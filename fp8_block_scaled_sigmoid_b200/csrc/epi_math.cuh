@@ -1,0 +1,42 @@
+// Element arithmetic shared by every kernel that quantises to E4M3 or applies
+// SwiGLU, so that fused and standalone paths give identical bytes.  Each step
+// uses an explicitly rounded fp32 intrinsic: no contraction into FMAs can
+// make two call sites differ.
+#pragma once
+
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr float kE4M3Max = 448.0f;
+constexpr float kQuantEps = 1e-4f;
+
+// Dequantisation multiplier of a tile with max |x| = amax ("Online
+// Quantization": s = Q_max / max(A_max, eps); stored as its inverse).
+__device__ __forceinline__ float quant_scale(float amax) {
+  return __fdiv_rn(fmaxf(amax, kQuantEps), kE4M3Max);
+}
+
+// Two fp32 values -> two E4M3 bytes (lo in the low byte), round to nearest
+// even, saturating to +-448 (hardware cvt.rn.satfinite.e4m3x2).
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+  return static_cast<uint16_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  return static_cast<uint32_t>(e4m3x2(a, b)) | (static_cast<uint32_t>(e4m3x2(c, d)) << 16);
+}
+
+// SiLU(g) * u with Swish beta = 1.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  const float den = __fadd_rn(1.0f, expf(-g));
+  return __fmul_rn(__fdiv_rn(g, den), u);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
+  return __uint_as_float(bits16 << 16);
+}
+
+}  // namespace moe

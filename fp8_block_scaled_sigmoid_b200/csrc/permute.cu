@@ -1,0 +1,298 @@
+// Local permutation of (token, expert) pairs by expert -- the single-GPU
+// stand-in for the dispatch step ("DeepSeek_V3_Report：Annotation",
+// "Low-Precision Communication": tokens are quantised to FP8 first and the
+// FP8 rows are what moves; "No Token-Dropping": no capacity limit).
+//
+// Deterministic and stable without atomics deciding any order:
+//  1. count   -- per chunk of kChunkT tokens, a shared-memory histogram
+//                (order-free integer adds) -> ws[chunk][E].
+//  2. scan    -- one CTA: per expert a running sum over chunks (chunk bases),
+//                then an exclusive scan over experts -> offsets, and the
+//                128-row tile table of every segment.
+//  3. scatter -- per chunk, one warp walks its tokens in order, several
+//                tokens per step (lane = (token, k)); lanes that picked the
+//                same expert are ranked with __match_any_sync in lane order,
+//                which is token order, so each expert's rows stay in
+//                ascending token order.
+//  4. gather  -- one warp per destination row copies the FP8 row (16-byte
+//                vectors, coalesced) and its 1x128 scales.
+#include "moe_common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kChunkT = 128;
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(256) perm_count_kernel(const int32_t* __restrict__ idx, int T,
+                                                         int K, int E, int32_t* __restrict__ ccount,
+                                                         int32_t* dev_err) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * kChunkT;
+  const int nt = min(kChunkT, T - t0);
+  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) {
+    const int e = idx[static_cast<int64_t>(t0) * K + p];
+    if (e < 0 || e >= E) {
+      set_dev_err(dev_err, MOE_DEVERR_BAD_INDEX);
+      continue;
+    }
+    atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    ccount[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
+}
+
+// Exclusive block scan of one int per thread (kScanThreads threads).
+__device__ int block_excl_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += n;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+    int wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += n;
+    }
+    warp_sums[lane] = wi - w;  // exclusive prefix of the warp sums
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  const int r = warp_sums[warp] + incl - v;
+  __syncthreads();
+  return r;
+}
+
+// Offsets and tile table from per-group row counts (one thread per group).
+__device__ void write_tables(int cnt, int g, int groups, int32_t* offsets, int32_t* tile_group,
+                             int32_t* tile_start, int32_t* n_tiles, int max_tiles,
+                             int32_t* dev_err, int* smem) {
+  int* warp_sums = smem;
+  int* totals = smem + 32;
+  const bool in = g < groups;
+  const int off = block_excl_scan(in ? cnt : 0, warp_sums, &totals[0]);
+  const int mt = in ? (cnt + 127) / 128 : 0;
+  const int mstart = block_excl_scan(mt, warp_sums, &totals[1]);
+  const int total_rows = totals[0];
+  const int total_tiles = totals[1];
+  const bool fits = total_tiles <= max_tiles;
+  if (in) {
+    offsets[g] = off;
+    tile_start[g] = mstart;
+    if (fits)
+      for (int j = 0; j < mt; ++j) tile_group[mstart + j] = g;
+  }
+  if (threadIdx.x == 0) {
+    offsets[groups] = total_rows;
+    tile_start[groups] = total_tiles;
+    *n_tiles = fits ? total_tiles : 0;
+    if (!fits) set_dev_err(dev_err, MOE_DEVERR_BAD_TABLE);
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) perm_scan_kernel(
+    int32_t* __restrict__ ccount, int n_chunks, int E, int T, int with_shared,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ tile_group,
+    int32_t* __restrict__ tile_start, int32_t* __restrict__ n_tiles, int max_tiles,
+    int32_t* dev_err) {
+  __shared__ int smem[40];
+  __shared__ int eoff[kScanThreads];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+    // running sum over chunks; loads batched so they overlap
+    int c = 0;
+    for (; c + 8 <= n_chunks; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = ccount[static_cast<int64_t>(c + j) * E + e];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        ccount[static_cast<int64_t>(c + j) * E + e] = run;
+        run += v[j];
+      }
+    }
+    for (; c < n_chunks; ++c) {
+      const int v = ccount[static_cast<int64_t>(c) * E + e];
+      ccount[static_cast<int64_t>(c) * E + e] = run;
+      run += v;
+    }
+    counts[e] = run;
+  }
+  const int groups = E + (with_shared ? 1 : 0);
+  const int cnt = (e < E) ? run : ((with_shared && e == E) ? T : 0);
+  write_tables(cnt, e, groups, offsets, tile_group, tile_start, n_tiles, max_tiles, dev_err, smem);
+  __syncthreads();
+  if (e < E) eoff[e] = offsets[e];
+  __syncthreads();
+  // chunk bases become absolute row positions
+  if (e < E) {
+    const int base = eoff[e];
+    for (int c = 0; c < n_chunks; ++c) ccount[static_cast<int64_t>(c) * E + e] += base;
+  }
+}
+
+__global__ void __launch_bounds__(32) perm_scatter_kernel(const int32_t* __restrict__ idx, int T,
+                                                          int K, int E,
+                                                          const int32_t* __restrict__ cbase,
+                                                          int32_t* __restrict__ src_row,
+                                                          int32_t* __restrict__ dst_of) {
+  extern __shared__ int32_t sm[];
+  int32_t* cursor = sm;       // [E]
+  int32_t* sidx = sm + E;     // [kChunkT * K]
+  const int lane = threadIdx.x;
+  const int t0 = blockIdx.x * kChunkT;
+  const int nt = min(kChunkT, T - t0);
+  for (int e = lane; e < E; e += 32) cursor[e] = cbase[static_cast<int64_t>(blockIdx.x) * E + e];
+  for (int p = lane; p < nt * K; p += 32) sidx[p] = idx[static_cast<int64_t>(t0) * K + p];
+  __syncwarp();
+  const int tpi = 32 / K;  // tokens per step
+  const int tl = lane / K, k = lane - (lane / K) * K;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int tb = 0; tb < nt; tb += tpi) {
+    const int tt = tb + tl;
+    int e = -1;
+    if (tl < tpi && tt < nt) e = sidx[tt * K + k];
+    const bool active = e >= 0 && e < E;
+    const unsigned amask = __ballot_sync(0xffffffffu, active);
+    unsigned peers = 0;
+    int pos = 0;
+    if (active) {
+      peers = __match_any_sync(amask, e);
+      pos = cursor[e] + __popc(peers & lt_mask);
+    }
+    __syncwarp();
+    if (active && lane == __ffs(peers) - 1) cursor[e] += __popc(peers);
+    __syncwarp();
+    if (active) {
+      const int t = t0 + tt;
+      src_row[pos] = t;
+      dst_of[static_cast<int64_t>(t) * K + k] = pos;
+    } else if (tl < tpi && tt < nt) {
+      dst_of[static_cast<int64_t>(t0 + tt) * K + k] = -1;  // flagged bad index: no row
+    }
+  }
+}
+
+// One warp per destination row: d bytes of FP8 plus d/128 fp32 scales.
+__global__ void __launch_bounds__(256) perm_gather_kernel(
+    const int32_t* __restrict__ src_row, int rows, int T, const uint8_t* __restrict__ xq,
+    const float* __restrict__ xs, int d, uint8_t* __restrict__ xq_perm,
+    float* __restrict__ xs_perm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int64_t s = src_row[r];
+  // rows left unassigned after a flagged bad expert index hold no token
+  if (s < 0 || s >= T) return;
+  const uint4* src = reinterpret_cast<const uint4*>(xq + s * d);
+  uint4* dst = reinterpret_cast<uint4*>(xq_perm + r * d);
+  const int nv = d / 16;
+  for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+  const int ns = d / 128;
+  for (int v = lane; v < ns; v += 32) xs_perm[r * ns + v] = __ldg(xs + s * ns + v);
+}
+
+__global__ void __launch_bounds__(kScanThreads) tile_table_kernel(
+    const int32_t* __restrict__ offsets, int groups, int max_tiles, int32_t* __restrict__ tile_group,
+    int32_t* __restrict__ tile_start, int32_t* __restrict__ n_tiles, int32_t* dev_err) {
+  __shared__ int smem[40];
+  __shared__ int32_t offs_copy[kScanThreads + 1];
+  const int g = threadIdx.x;
+  int cnt = 0;
+  if (g < groups) {
+    cnt = offsets[g + 1] - offsets[g];
+    if (cnt < 0 || offsets[g] < 0) {
+      set_dev_err(dev_err, MOE_DEVERR_BAD_TABLE);
+      cnt = 0;
+    }
+  }
+  // the caller's offsets are kept; only the tile table is written
+  write_tables(cnt, g, groups, offs_copy, tile_group, tile_start, n_tiles, max_tiles, dev_err,
+               smem);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int n_chunks_of(int T) { return (T + kChunkT - 1) / kChunkT; }
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_max_m_tiles(int T, int K, int E, int with_shared) {
+  if (T < 0 || K < 0 || E < 0) return 0;
+  const int64_t pairs = static_cast<int64_t>(T) * K;
+  int64_t n = (pairs + static_cast<int64_t>(E) * 127) / 128;  // sum of ceil(c_e/128)
+  if (with_shared) n += (T + 127) / 128;
+  return static_cast<int>(n);
+}
+
+extern "C" moe_status moe_permute_workspace_size(int T, int K, int E, size_t* bytes) {
+  if (!bytes || T < 0 || K <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+  const size_t b = static_cast<size_t>(moe::n_chunks_of(T)) * E * sizeof(int32_t);
+  *bytes = (b + 255) / 256 * 256;
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_permute(const int32_t* topk_idx, int T, int K, int E, int with_shared,
+                                  const uint8_t* xq, const float* xscale, int d, int32_t* counts,
+                                  int32_t* offsets, int32_t* src_row, int32_t* dst_of,
+                                  uint8_t* xq_perm, float* xscale_perm, int32_t* tile_group,
+                                  int32_t* tile_start, int32_t* n_tiles, void* ws,
+                                  size_t ws_bytes, int32_t* dev_err, moe_stream_t stream) {
+  using namespace moe;
+  if (T < 0 || K <= 0 || E <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+  if (d % 128 != 0) return MOE_ERR_SHAPE;
+  if (K > 32 || K > E || E + (with_shared ? 1 : 0) > kScanThreads) return MOE_ERR_UNSUPPORTED;
+  if (!counts || !offsets || !tile_start || !n_tiles || !tile_group) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_idx || !xq || !xscale || !src_row || !dst_of || !xq_perm || !xscale_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(xq_perm)) return MOE_ERR_ALIGN;
+  size_t need = 0;
+  moe_permute_workspace_size(T, K, E, &need);
+  if (ws_bytes < need || (!ws && need)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nch = n_chunks_of(T);
+  int32_t* ccount = static_cast<int32_t*>(ws);
+  const int max_tiles = moe_max_m_tiles(T, K, E, with_shared);
+  if (nch > 0) {
+    perm_count_kernel<<<nch, 256, E * sizeof(int32_t), st>>>(topk_idx, T, K, E, ccount, dev_err);
+    MOE_CUDA_CHECK_LAUNCH();
+  }
+  perm_scan_kernel<<<1, kScanThreads, 0, st>>>(ccount, nch, E, T, with_shared, counts, offsets,
+                                               tile_group, tile_start, n_tiles, max_tiles, dev_err);
+  MOE_CUDA_CHECK_LAUNCH();
+  if (nch > 0) {
+    const size_t sm = (static_cast<size_t>(E) + kChunkT * K) * sizeof(int32_t);
+    perm_scatter_kernel<<<nch, 32, sm, st>>>(topk_idx, T, K, E, ccount, src_row, dst_of);
+    MOE_CUDA_CHECK_LAUNCH();
+    const int rows = T * K;
+    perm_gather_kernel<<<(rows + 7) / 8, 256, 0, st>>>(src_row, rows, T, xq, xscale, d, xq_perm,
+                                                       xscale_perm);
+    MOE_CUDA_CHECK_LAUNCH();
+  }
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_tile_table(const int32_t* offsets, int groups, int max_tiles,
+                                     int32_t* tile_group, int32_t* tile_start, int32_t* n_tiles,
+                                     int32_t* dev_err, moe_stream_t stream) {
+  using namespace moe;
+  if (groups <= 0 || max_tiles < 0 || !offsets || !tile_group || !tile_start || !n_tiles)
+    return MOE_ERR_INVALID_ARG;
+  if (groups > kScanThreads) return MOE_ERR_UNSUPPORTED;
+  tile_table_kernel<<<1, kScanThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      offsets, groups, max_tiles, tile_group, tile_start, n_tiles, dev_err);
+  MOE_CUDA_CHECK_LAUNCH();
+  return MOE_OK;
+}

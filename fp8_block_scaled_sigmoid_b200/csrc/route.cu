@@ -1,0 +1,330 @@
+// Sigmoid router with bias-based, group-limited top-K selection.
+// "DeepSeek_V3_Report：Annotation", eqs. (13)-(16), "Node-Limited Routing" and
+// "Auxiliary-Loss-Free Load Balancing".
+//
+// Two kernels:
+//  1. router_logits_kernel -- z = u . e^T as a bf16 x bf16 -> fp32 tcgen05 GEMM
+//     (TMA-fed 128-byte-swizzled smem ring, accumulator in TMEM).  The gating
+//     stays in high precision, never FP8.  K is split over blockIdx.z so that
+//     a T=4096 batch still covers the SMs; the partial sums land in the
+//     caller's workspace and are added in split order (deterministic).
+//  2. route_select_kernel -- one warp per token, experts spread over lanes,
+//     everything in registers and warp shuffles: sigmoid, biased scores,
+//     group scores (sum of each group's top K/M), top-M groups, top-K experts
+//     within them (ties to the lower index), gates from the raw scores.
+#include <algorithm>
+#include <climits>
+
+#include "moe_common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kRtStages = 4;
+constexpr int kRtBK = 64;                 // bf16 elements per stage (128 bytes)
+constexpr int kRtABytes = 128 * 128;      // 128 rows x 128 bytes
+constexpr int kRtThreads = 128;
+
+struct RouterTiling {
+  int m_tiles, n_tiles, BN, KB, splits, kb_per_split;
+};
+
+RouterTiling router_tiling(int T, int d, int E) {
+  RouterTiling r;
+  r.m_tiles = (T + 127) / 128;
+  r.n_tiles = (E + 255) / 256;
+  r.BN = ((E + r.n_tiles - 1) / r.n_tiles + 15) / 16 * 16;
+  r.KB = d / kRtBK;
+  const int tiles = std::max(1, r.m_tiles * r.n_tiles);
+  int splits = (moe_num_sms() + tiles - 1) / tiles;
+  splits = std::max(1, std::min(std::min(splits, 16), r.KB));
+  r.kb_per_split = (r.KB + splits - 1) / splits;
+  r.splits = (r.KB + r.kb_per_split - 1) / r.kb_per_split;  // no empty split
+  return r;
+}
+
+size_t router_smem_bytes(int BN) {
+  return 1024 + static_cast<size_t>(kRtStages) * (kRtABytes + BN * 128) + 256;
+}
+
+__global__ void __launch_bounds__(kRtThreads, 1) router_logits_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    float* __restrict__ part, int T, int E, int BN, int KB, int kb_per_split,
+    int32_t* dev_err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sA = base;
+  uint8_t* sB = base + kRtStages * kRtABytes;
+  const int b_bytes = BN * 128;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kRtStages * b_bytes);
+  uint64_t* empty = full + kRtStages;
+  uint64_t* done = empty + kRtStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN, split = blockIdx.z;
+  const int kb0 = split * kb_per_split;
+  const int nkb = min(KB, kb0 + kb_per_split) - kb0;
+  const uint32_t ncols = BN <= 32 ? 32u : (BN <= 64 ? 64u : (BN <= 128 ? 128u : 256u));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRtStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abort_v = abort_flag;
+
+  if (warp == 0 && lane == 0) {
+    // TMA producer
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % kRtStages;
+      const uint32_t ph = (i / kRtStages) & 1;
+      if (!mbar_wait(&empty[s], ph ^ 1, abort_v, dev_err)) break;
+      mbar_arrive_expect_tx(&full[s], kRtABytes + b_bytes);
+      tma_load_2d(sA + s * kRtABytes, &tmA, &full[s], (kb0 + i) * kRtBK, m0);
+      tma_load_2d(sB + s * b_bytes, &tmB, &full[s], (kb0 + i) * kRtBK, n0);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // single-thread MMA issuer: 4 x (K=16) per 64-element stage
+    const uint32_t idesc = instr_desc(kFmtBF16, kFmtBF16, 128, BN);
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % kRtStages;
+      const uint32_t ph = (i / kRtStages) & 1;
+      if (!mbar_wait(&full[s], ph, abort_v, dev_err)) break;
+      tc_fence_after();
+      const uint64_t ad = smem_desc_sw128(smem_u32(sA + s * kRtABytes));
+      const uint64_t bd = smem_desc_sw128(smem_u32(sB + s * b_bytes));
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_f16(tmem, ad + 2 * k, bd + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
+      mma_commit(&empty[s]);
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+  // warp-uniform outcome: the TMEM loads below are warp-collective
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_v, dev_err));
+  tc_fence_after();
+  if (ok && *abort_v == 0) {
+    const int row = m0 + warp * 32 + lane;
+    float* dst = part + (static_cast<int64_t>(split) * T + row) * E;
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c, v);
+      tmem_ld_wait();
+      if (row < T) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (n0 + c + j < E) dst[n0 + c + j] = v[j];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
+// --------------------------------------------------------------- selection --
+struct Cand {
+  float v;  // biased score
+  int i;    // expert
+  float s;  // raw score
+};
+
+__device__ __forceinline__ bool better(float v1, int i1, float v2, int i2) {
+  return v1 > v2 || (v1 == v2 && i1 < i2);
+}
+
+__device__ __forceinline__ Cand warp_best(Cand c) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float v = __shfl_xor_sync(0xffffffffu, c.v, off);
+    const int i = __shfl_xor_sync(0xffffffffu, c.i, off);
+    const float s = __shfl_xor_sync(0xffffffffu, c.s, off);
+    if (better(v, i, c.v, c.i)) {
+      c.v = v;
+      c.i = i;
+      c.s = s;
+    }
+  }
+  return c;
+}
+
+constexpr int kSelThreads = 256;
+
+// P = experts per lane (lane l owns experts l*P .. l*P+P-1).
+template <int P>
+__global__ void __launch_bounds__(kSelThreads) route_select_kernel(
+    const float* __restrict__ part, int splits, int T, int E, int G, int M, int K,
+    const float* __restrict__ bias, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+    float* __restrict__ logits_out) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (kSelThreads / 32) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int e0 = lane * P;
+  const int gs = E / G;
+  float beta[P], sc[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    const int e = e0 + i;
+    beta[i] = -INFINITY;
+    sc[i] = 0.f;
+    if (e < E) {
+      float z = part[static_cast<int64_t>(t) * E + e];
+      for (int sp = 1; sp < splits; ++sp)
+        z = __fadd_rn(z, part[(static_cast<int64_t>(sp) * T + t) * E + e]);
+      if (logits_out) logits_out[static_cast<int64_t>(t) * E + e] = z;
+      sc[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z)));
+      beta[i] = __fadd_rn(sc[i], bias[e]);
+    }
+  }
+
+  // groups a token may use (bit g set = allowed)
+  uint32_t allowed = 0xffffffffu;
+  if (M < G) {
+    const int n_top = K / M;
+    float my_score = -INFINITY;
+    for (int g = 0; g < G; ++g) {
+      uint32_t tk = 0;
+      float sum = 0.f;
+      for (int r = 0; r < n_top; ++r) {
+        Cand c{-INFINITY, INT_MAX, 0.f};
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+          const int e = e0 + i;
+          if (e < E && e / gs == g && !((tk >> i) & 1u) && better(beta[i], e, c.v, c.i)) {
+            c.v = beta[i];
+            c.i = e;
+          }
+        }
+        c = warp_best(c);
+        if (c.i / P == lane) tk |= 1u << (c.i - e0);
+        sum = __fadd_rn(sum, c.v);
+      }
+      if (lane == g) my_score = sum;
+    }
+    int rank = 0;
+    for (int g = 0; g < G; ++g) {
+      const float v = __shfl_sync(0xffffffffu, my_score, g);
+      if (better(v, g, my_score, lane)) ++rank;
+    }
+    allowed = __ballot_sync(0xffffffffu, lane < G && rank < M);
+  }
+
+  uint32_t taken = 0;
+  float ssum = 0.f, my_s = 0.f;
+  int my_idx = 0;
+  for (int k = 0; k < K; ++k) {
+    Cand c{-INFINITY, INT_MAX, 0.f};
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+      const int e = e0 + i;
+      if (e < E && ((allowed >> (e / gs)) & 1u) && !((taken >> i) & 1u) &&
+          better(beta[i], e, c.v, c.i)) {
+        c.v = beta[i];
+        c.i = e;
+        c.s = sc[i];
+      }
+    }
+    c = warp_best(c);
+    if (c.i / P == lane) taken |= 1u << (c.i - e0);
+    ssum = __fadd_rn(ssum, c.s);
+    if (lane == k) {
+      my_idx = c.i;
+      my_s = c.s;
+    }
+  }
+  if (lane < K) {
+    idx_out[static_cast<int64_t>(t) * K + lane] = my_idx;
+    gate_out[static_cast<int64_t>(t) * K + lane] = __fdiv_rn(my_s, ssum);
+  }
+}
+
+template <int P>
+void launch_select(int blocks, cudaStream_t st, const float* part, int splits, int T, int E,
+                   int G, int M, int K, const float* bias, int32_t* idx, float* gate,
+                   float* logits) {
+  route_select_kernel<P><<<blocks, kSelThreads, 0, st>>>(part, splits, T, E, G, M, K, bias, idx,
+                                                          gate, logits);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_route_workspace_size(int T, int d, int E, size_t* bytes) {
+  if (!bytes || T < 0 || d <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+  if (d % 128 != 0) return MOE_ERR_SHAPE;
+  const moe::RouterTiling r = moe::router_tiling(T, d, E);
+  const size_t b = static_cast<size_t>(r.splits) * T * E * sizeof(float);
+  *bytes = (b + 255) / 256 * 256;
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* centroids,
+                                const float* bias, int T, int d, int E, int G, int M, int K,
+                                int32_t* topk_idx, float* topk_gate, float* logits_out, void* ws,
+                                size_t ws_bytes, int32_t* dev_err, moe_stream_t stream) {
+  using namespace moe;
+  if (T < 0 || d <= 0 || E <= 0 || G <= 0 || M <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (d % 128 != 0 || E % 16 != 0 || E % G != 0 || M > G || K > E || ldu < d) return MOE_ERR_SHAPE;
+  if (E > 1024 || G > 32 || K > 32) return MOE_ERR_UNSUPPORTED;
+  if (M < G && (K % M != 0 || M * (E / G) < K)) return MOE_ERR_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!u || !centroids || !bias || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(u) || !aligned16(centroids) || ldu % 8 != 0) return MOE_ERR_ALIGN;
+  size_t need = 0;
+  moe_route_workspace_size(T, d, E, &need);
+  if (ws_bytes < need || (!ws && need)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_ALIGN;
+
+  const RouterTiling r = router_tiling(T, d, E);
+  CUtensorMap tmA, tmB;
+  if (!moe_make_tmap_2d(&tmA, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, T, ldu * 2, kRtBK, 128) ||
+      !moe_make_tmap_2d(&tmB, centroids, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, E, d * 2, kRtBK,
+                        r.BN))
+    return MOE_ERR_CUDA;
+  const size_t smem = router_smem_bytes(r.BN);
+  static int configured = 0;
+  if (!configured) {
+    if (cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(router_smem_bytes(256))) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured = 1;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* part = static_cast<float*>(ws);
+  dim3 grid(r.m_tiles, r.n_tiles, r.splits);
+  router_logits_kernel<<<grid, kRtThreads, smem, st>>>(tmA, tmB, part, T, E, r.BN, r.KB,
+                                                       r.kb_per_split, dev_err);
+  MOE_CUDA_CHECK_LAUNCH();
+
+  const int blocks = (T + kSelThreads / 32 - 1) / (kSelThreads / 32);
+  const int P = (E + 31) / 32;
+  if (P <= 1) launch_select<1>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
+  else if (P <= 2) launch_select<2>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
+  else if (P <= 4) launch_select<4>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
+  else if (P <= 8) launch_select<8>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
+  else if (P <= 12) launch_select<12>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
+  else if (P <= 16) launch_select<16>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
+  else launch_select<32>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
+  MOE_CUDA_CHECK_LAUNCH();
+  return MOE_OK;
+}

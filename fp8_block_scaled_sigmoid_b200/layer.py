@@ -1,0 +1,155 @@
+"""One DeepSeekMoE layer forward, composed from the C-ABI calls.
+
+The steps ("DeepSeek_V3_Report：Annotation", eqs. (12)-(16); quantise before
+dispatch per "Low-Precision Communication"):
+
+    moe_route -> fp8_quant_1x128(u) -> moe_permute
+      -> grouped GEMM 1 (W1, fused SwiGLU + 1x128 requantisation)
+      -> grouped GEMM 2 (W2, fp32 rows) -> moe_combine -> moe_bias_update
+
+All of it is queued on one CUDA stream with no host synchronisation: the
+ragged expert segments travel through device-side offsets and the tile
+table.  This module only owns buffers (torch allocations) and the call order;
+every step runs in libmoefp8.so.
+
+Row layout of the permuted activations (and of h and Y): rows [0, T*K) are
+the routed pairs sorted by expert, rows [T*K, T*K+T) are the T tokens in
+order, which the shared expert (group E of the grouped GEMMs) consumes.  The
+quantiser writes the tokens straight into that tail and the permutation
+gathers the routed rows from it, so the shared expert costs no copy.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _abi
+from .configs import MoEConfig
+from . import inputs as _inputs
+
+
+def quantise_weight_stack(w_bf16: torch.Tensor, q=None, s=None):
+    """128x128 block quantisation of a [G][N][K] bf16 stack on the device."""
+    return _abi.fp8_quant_128x128(w_bf16, q, s)
+
+
+def make_fp8_weights(cfg: MoEConfig, device, chunk: int = 16):
+    """Draw the bf16 expert weights (seeded, per expert) and quantise them on
+    the device a few experts at a time; only the FP8 stacks stay resident."""
+    G = cfg.E + cfg.n_shared
+    w1q = torch.empty(G, 2 * cfg.I, cfg.d, dtype=torch.uint8, device=device)
+    w1s = torch.empty(G, 2 * cfg.I // 128, cfg.d // 128, dtype=torch.float32, device=device)
+    w2q = torch.empty(G, cfg.d, cfg.I, dtype=torch.uint8, device=device)
+    w2s = torch.empty(G, cfg.d // 128, cfg.I // 128, dtype=torch.float32, device=device)
+    for e0 in range(0, G, chunk):
+        e1 = min(G, e0 + chunk)
+        w1 = torch.stack([_inputs.draw_w1(cfg, e, device) for e in range(e0, e1)])
+        w2 = torch.stack([_inputs.draw_w2(cfg, e, device) for e in range(e0, e1)])
+        _abi.fp8_quant_128x128(w1, w1q[e0:e1], w1s[e0:e1])
+        _abi.fp8_quant_128x128(w2, w2q[e0:e1], w2s[e0:e1])
+        del w1, w2
+    return w1q, w1s, w2q, w2s
+
+
+class MoELayer:
+    """Device buffers and call sequence of one layer for a fixed batch size T."""
+
+    def __init__(self, cfg: MoEConfig, centroids: torch.Tensor, bias: torch.Tensor,
+                 w1q, w1s, w2q, w2s, T: int | None = None, process_group=None):
+        self.cfg = cfg
+        self.T = cfg.T if T is None else T
+        self.dev = centroids.device
+        self.centroids = centroids
+        self.bias = bias
+        self.w1q, self.w1s, self.w2q, self.w2s = w1q, w1s, w2q, w2s
+        self.pg = process_group
+        T, d, K, E, I = self.T, cfg.d, cfg.K, cfg.E, cfg.I
+        P = T * K
+        self.pairs = P
+        dev = self.dev
+        i32, f32, u8 = torch.int32, torch.float32, torch.uint8
+        self.idx = torch.empty(T, K, dtype=i32, device=dev)
+        self.gate = torch.empty(T, K, dtype=f32, device=dev)
+        self.route_ws = torch.empty(max(_abi.moe_route_workspace_size(T, d, E), 16), dtype=u8, device=dev)
+        self.Xq = torch.empty(P + T, d, dtype=u8, device=dev)
+        self.Xs = torch.empty(P + T, d // 128, dtype=f32, device=dev)
+        self.perm = {
+            "xq_perm": self.Xq[:P], "xs_perm": self.Xs[:P],
+        }
+        self.perm_ws = torch.empty(max(_abi.moe_permute_workspace_size(T, K, E), 16), dtype=u8, device=dev)
+        self.H = torch.empty(P + T, I, dtype=u8, device=dev)
+        self.Hs = torch.empty(P + T, I // 128, dtype=f32, device=dev)
+        self.Y = torch.empty(P + T, d, dtype=f32, device=dev)
+        self.out = torch.empty(T, d, dtype=f32, device=dev)
+        self.dev_err = torch.zeros(1, dtype=i32, device=dev)
+        self.u_dev = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        # first permute allocates the index/tile buffers inside self.perm
+        self.max_tiles = _abi.moe_max_m_tiles(T, K, E, True)
+
+    # -- individual steps (also used by the benchmark to time them) --------
+    def step_route(self, u):
+        c = self.cfg
+        _abi.moe_route(u, self.centroids, self.bias, c.G, c.M, c.K, self.idx, self.gate,
+                       ws=self.route_ws, dev_err=self.dev_err)
+
+    def step_quant(self, u):
+        _abi.fp8_quant_1x128(u, self.Xq[self.pairs:], self.Xs[self.pairs:])
+
+    def step_permute(self):
+        c = self.cfg
+        _abi.moe_permute(self.idx, c.E, self.Xq[self.pairs:], self.Xs[self.pairs:], True,
+                         out=self.perm, ws=self.perm_ws, dev_err=self.dev_err)
+
+    def step_gemm1(self):
+        p = self.perm
+        _abi.grouped_gemm_fp8_blockscaled(self.Xq, self.Xs, self.w1q, self.w1s, p["offsets"],
+                                          p["tile_group"], p["tile_start"], p["n_tiles"],
+                                          self.max_tiles, _abi.EP_SWIGLU_QUANT, self.H, self.Hs,
+                                          dev_err=self.dev_err)
+
+    def step_gemm2(self):
+        p = self.perm
+        _abi.grouped_gemm_fp8_blockscaled(self.H, self.Hs, self.w2q, self.w2s, p["offsets"],
+                                          p["tile_group"], p["tile_start"], p["n_tiles"],
+                                          self.max_tiles, _abi.EP_F32, self.Y,
+                                          dev_err=self.dev_err)
+
+    def step_combine(self, u):
+        P = self.pairs
+        _abi.moe_combine(self.Y, self.perm["dst_of"], self.gate, self.Y[P:], u, self.out)
+
+    def step_bias_update(self):
+        counts = self.perm["counts"]
+        T_all = self.T
+        if self.pg is not None:
+            import torch.distributed as dist
+            counts = counts.clone()
+            dist.all_reduce(counts, group=self.pg)
+            T_all = self.T * dist.get_world_size(self.pg)
+        _abi.moe_bias_update(counts, T_all, self.cfg.K, self.cfg.gamma, self.bias)
+
+    # -- whole layer --------------------------------------------------------
+    def forward(self, u: torch.Tensor, update_bias: bool = True) -> torch.Tensor:
+        """u bf16 [T][d] on the device -> out fp32 [T][d] (self.out)."""
+        assert u.shape == (self.T, self.cfg.d) and u.dtype == torch.bfloat16
+        self.step_route(u)
+        self.step_quant(u)
+        self.step_permute()
+        self.step_gemm1()
+        self.step_gemm2()
+        self.step_combine(u)
+        if update_bias:
+            self.step_bias_update()
+        return self.out
+
+    def forward_host(self, u_host: torch.Tensor, out_host: torch.Tensor,
+                     update_bias: bool = True) -> torch.Tensor:
+        """End-to-end call with host buffers: copy u in (pinned host ->
+        device), run the layer, copy the output back (device -> pinned host)."""
+        self.u_dev.copy_(u_host, non_blocking=True)
+        self.forward(self.u_dev, update_bias)
+        out_host.copy_(self.out, non_blocking=True)
+        return out_host
+
+    def check(self) -> None:
+        """Raise if a kernel recorded a device-side error (synchronises)."""
+        _abi.raise_dev_err(self.dev_err)

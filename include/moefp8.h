@@ -1,0 +1,227 @@
+/*
+ * moefp8.h -- C ABI of libmoefp8.so: the forward pass of one DeepSeekMoE layer
+ * with FP8 (E4M3) block-scaled expert GEMMs, as hand-written sm_100a kernels.
+ *
+ * Sources (web pages on DeepSeek-V3/V4):
+ *   [ANN]   "DeepSeek_V3_Report：Annotation" -- eqs. (12)-(16), "Node-Limited
+ *           Routing", "Auxiliary-Loss-Free Load Balancing", "Fine-Grained
+ *           Quantization", "Online Quantization", "Low-Precision Communication",
+ *           SwiGLU operator notes.
+ *   [INFRA] "DeepSeek V3 / V4 Infra：把 all-to-all 藏进计算" -- 6hd FLOPs per
+ *           token-expert pair (gate, up, down projections).
+ *
+ * Conventions shared by every call:
+ *   - All pointers are DEVICE pointers unless stated.  The caller owns every
+ *     buffer; the library allocates nothing and keeps no state between calls
+ *     (scratch comes from the caller through `ws`, sized by the matching
+ *     *_workspace_size query).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and returns a moe_status.  Argument, shape and
+ *     alignment errors are detected on the host before anything is launched
+ *     and returned synchronously; a failed launch returns MOE_ERR_CUDA.
+ *   - Faults that only the device can see (inconsistent segment tables, a
+ *     bounded wait that ran out) are recorded in the caller's `dev_err`
+ *     (one int32 in device memory, 0 = none; first error wins) and read by
+ *     the caller after synchronising.  `dev_err` may be NULL, which drops them.
+ *   - bf16 tensors are passed as uint16_t bit patterns.  FP8 tensors are
+ *     E4M3 bytes (bias 7, max 448, no infinities).
+ *   - Device pointers must be 16-byte aligned; leading dimensions are in
+ *     elements and must keep every row 16-byte aligned.  Widths that are
+ *     tiled by 128 (d, I, N, K) must be multiples of 128.
+ *   - Scales are fp32 dequantisation multipliers: x ~= e4m3_value * scale,
+ *     scale = max(amax, 1e-4) / 448 computed in fp32, and the stored byte is
+ *     E4M3(x / scale) with the division in fp32 (IEEE, round to nearest even)
+ *     and round-to-nearest-even, saturating conversion.
+ *   - No call throws; no exception crosses the ABI.
+ */
+#ifndef MOEFP8_H
+#define MOEFP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* NULL where a buffer is required, negative size */
+  MOE_ERR_SHAPE = 2,       /* a width not a multiple of 128, K % M != 0, ... */
+  MOE_ERR_ALIGN = 3,       /* pointer or leading dimension not 16-byte aligned */
+  MOE_ERR_UNSUPPORTED = 4, /* shape outside the kernels' limits (e.g. E > 1024) */
+  MOE_ERR_CUDA = 5,        /* a CUDA call or kernel launch failed */
+  MOE_ERR_WORKSPACE = 6    /* workspace smaller than the size query returned */
+} moe_status;
+
+typedef enum {
+  MOE_EP_F32 = 0,         /* D is fp32 [rows][N] */
+  MOE_EP_SWIGLU_QUANT = 1 /* D is E4M3 [rows][N/2] with d_scale fp32 [rows][N/256] */
+} moe_epilogue;
+
+/* Codes the kernels write into dev_err. */
+#define MOE_DEVERR_TIMEOUT 1   /* a bounded wait gave up; results are invalid */
+#define MOE_DEVERR_BAD_TABLE 2 /* segment offsets / tile table inconsistent */
+#define MOE_DEVERR_BAD_INDEX 3 /* an expert index outside [0, E) */
+
+typedef void* moe_stream_t; /* cudaStream_t */
+
+/* Human-readable text for a status (static storage, never NULL). */
+const char* moe_status_string(moe_status s);
+
+/* ABI version of this header (bumped on any incompatible change). */
+int moe_abi_version(void);
+
+/* ---------------------------------------------------------------------------
+ * fp8_quant_1x128 -- online 1x128 activation quantisation.
+ * [ANN] "Fine-Grained Quantization" (activations grouped and scaled per token
+ * per 128 channels) and "Online Quantization" (scale from the tile's own
+ * max |x|, s = Q_max / max(A_max, eps), Q_max = 448 for E4M3).
+ *   x     bf16 [rows][ldx], first `cols` columns used; ldx >= cols, ldx % 8 == 0
+ *   q     E4M3 [rows][cols] (dense, row stride cols)
+ *   scale fp32 [rows][cols/128]
+ * cols % 128 == 0; rows >= 0 (rows == 0 launches nothing).
+ */
+moe_status fp8_quant_1x128(const uint16_t* x, int64_t ldx, int rows, int cols, uint8_t* q,
+                           float* scale, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * fp8_quant_128x128 -- online 128x128 weight-block quantisation.
+ * [ANN] "Fine-Grained Quantization" (weights grouped per 128 input x 128
+ * output channels) and "Online Quantization".
+ *   w     bf16 [rows][ldw] in nn.Linear layout (output channels x input
+ *         channels, input channels contiguous); stacks of experts are passed
+ *         as rows = experts * N when N % 128 == 0
+ *   q     E4M3 [rows][cols];  scale fp32 [ceil(rows/128)][cols/128]
+ * cols % 128 == 0; a ragged last row-block takes its amax over its real rows.
+ */
+moe_status fp8_quant_128x128(const uint16_t* w, int64_t ldw, int rows, int cols, uint8_t* q,
+                             float* scale, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_route -- sigmoid router with bias-based, group-limited top-K selection.
+ * [ANN] eqs. (13)-(16): s_{i,t} = Sigmoid(u_t . e_i); the top-K is taken over
+ * s_{i,t} + b_i, the gate g_{i,t} = s_{i,t} / sum of the chosen s; "Node-
+ * Limited Routing": at most M of G groups, groups ranked by the sum of their
+ * top K/M biased scores.  Ties go to the lower index (groups and experts);
+ * the K outputs of a token are ordered by biased score, descending.
+ * The logits are a bf16 x bf16 -> fp32 tensor-core GEMM; everything after
+ * them runs in fp32.
+ *   u          bf16 [T][ldu];  centroids bf16 [E][d];  bias fp32 [E]
+ *   topk_idx   int32 [T][K];   topk_gate fp32 [T][K]
+ *   logits_out fp32 [T][E] or NULL (the logits the selection used)
+ *   ws         scratch of moe_route_workspace_size() bytes (may be NULL if 0)
+ * Limits: d % 128 == 0, E % 16 == 0, 16 <= E <= 1024, E % G == 0,
+ * 1 <= M <= G <= 32, K <= E, K % M == 0 when M < G, K <= 32.
+ */
+moe_status moe_route_workspace_size(int T, int d, int E, size_t* bytes);
+moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* centroids,
+                     const float* bias, int T, int d, int E, int G, int M, int K,
+                     int32_t* topk_idx, float* topk_gate, float* logits_out, void* ws,
+                     size_t ws_bytes, int32_t* dev_err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_permute -- local permutation of (token, expert) pairs by expert, the
+ * single-GPU stand-in for the dispatch step.  [ANN] "Low-Precision
+ * Communication" (activations are quantised to FP8 before dispatch, so the
+ * permutation moves FP8 rows and their scales) and "No Token-Dropping" (no
+ * capacity limit: every pair gets a row).
+ * Pair (t, k) goes to row dst_of[t][k]; rows of expert e are
+ * [offsets[e], offsets[e+1]) in ascending token order.  With with_shared != 0
+ * the shared expert is group E whose T rows [T*K, T*K+T) the caller fills
+ * with the unpermuted quantised tokens (offsets has E+2 entries then).
+ *   topk_idx int32 [T][K] (each token's experts distinct, in [0, E))
+ *   xq E4M3 [T][d], xscale fp32 [T][d/128]   (the quantised tokens)
+ *   counts int32 [E] (routed pairs per expert), offsets int32 [E+1 (+1)]
+ *   src_row int32 [T*K], dst_of int32 [T][K]
+ *   xq_perm E4M3 [T*K][d], xscale_perm fp32 [T*K][d/128]  (rows 0..T*K-1)
+ *   tile_group int32 [moe_max_m_tiles()], tile_start int32 [groups+1],
+ *   n_tiles int32 [1]: the 128-row tiles of every segment, for the grouped
+ *   GEMM (tile j covers rows of group tile_group[j]).
+ * An out-of-range expert index records MOE_DEVERR_BAD_INDEX.
+ */
+int moe_max_m_tiles(int T, int K, int E, int with_shared);
+moe_status moe_permute_workspace_size(int T, int K, int E, size_t* bytes);
+moe_status moe_permute(const int32_t* topk_idx, int T, int K, int E, int with_shared,
+                       const uint8_t* xq, const float* xscale, int d, int32_t* counts,
+                       int32_t* offsets, int32_t* src_row, int32_t* dst_of, uint8_t* xq_perm,
+                       float* xscale_perm, int32_t* tile_group, int32_t* tile_start,
+                       int32_t* n_tiles, void* ws, size_t ws_bytes, int32_t* dev_err,
+                       moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_tile_table -- the 128-row tile table of arbitrary segment offsets (for
+ * grouped GEMM calls whose segments do not come from moe_permute).
+ *   offsets int32 [groups+1], non-decreasing, device
+ *   tile_group int32 [max_tiles], tile_start int32 [groups+1], n_tiles int32 [1]
+ * Inconsistent offsets or too small a max_tiles record MOE_DEVERR_BAD_TABLE.
+ */
+moe_status moe_tile_table(const int32_t* offsets, int groups, int max_tiles,
+                          int32_t* tile_group, int32_t* tile_start, int32_t* n_tiles,
+                          int32_t* dev_err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * grouped_gemm_fp8_blockscaled -- D_g = A_g . B_g^T for every segment g, with
+ * FP8 operands, per-128-K block scales and fp32 accumulation.
+ * [ANN] "Fine-Grained Quantization" (per-group scales along the inner
+ * dimension K) and "Increasing Accumulation Precision" (partial results
+ * promoted to fp32 and scaled every 128 elements of K).  Here each 128-wide
+ * K block is one tensor-core (tcgen05) accumulation in TMEM, which is then
+ * scaled by sa * sb and added to an fp32 register accumulator.
+ *   A  E4M3 [a_rows][K], sa fp32 [a_rows][K/128]  (1x128 tiles)
+ *   B  E4M3 [groups][N][K], sb fp32 [groups][N/128][K/128] (128x128 blocks)
+ *   offsets int32 [groups+1] (segment g = rows [offsets[g], offsets[g+1]))
+ *   tile_group / tile_start / n_tiles: as written by moe_permute or
+ *   moe_tile_table; max_tiles = capacity of tile_group.
+ *   ep == MOE_EP_F32:  D fp32 [a_rows][N] (rows outside every segment are
+ *                      left untouched); d_scale unused.
+ *   ep == MOE_EP_SWIGLU_QUANT: B rows are gate/up block-interleaved (rows
+ *      [256j, 256j+128) gate channels 128j.., the next 128 the matching up
+ *      channels); D is E4M3 h [a_rows][N/2] with h = SiLU(gate) * up
+ *      ([ANN] SwiGLU operator notes, Swish with beta = 1) quantised 1x128 as
+ *      in fp8_quant_1x128, d_scale fp32 [a_rows][N/256].
+ * Limits: K % 128 == 0, N % 256 == 0.
+ */
+moe_status grouped_gemm_fp8_blockscaled(const uint8_t* A, const float* sa, int64_t a_rows,
+                                        const uint8_t* B, const float* sb,
+                                        const int32_t* offsets, const int32_t* tile_group,
+                                        const int32_t* tile_start, const int32_t* n_tiles,
+                                        int max_tiles, int groups, int N, int K,
+                                        moe_epilogue ep, void* D, float* d_scale,
+                                        int32_t* dev_err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * swiglu_quant -- standalone SwiGLU + 1x128 quantisation of fp32 GEMM output
+ * in the block-interleaved layout above; bit-identical to the fused epilogue
+ * on identical input.
+ *   gu fp32 [rows][2I];  h E4M3 [rows][I];  h_scale fp32 [rows][I/128]
+ */
+moe_status swiglu_quant(const float* gu, int rows, int I, uint8_t* h, float* h_scale,
+                        moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_combine -- [ANN] eq. (12): out_t = u_t + FFN_shared(u_t)
+ *                                        + sum_k gate[t][k] * Y[dst_of[t][k]],
+ * summed in fp32 in that order (k ascending), deterministic.
+ *   Y fp32 [>= T*K][d] (routed expert outputs by permuted row)
+ *   Y_shared fp32 [T][d] or NULL;  u bf16 [T][d];  out fp32 [T][d]
+ */
+moe_status moe_combine(const float* Y, const int32_t* dst_of, const float* topk_gate,
+                       const float* Y_shared, const uint16_t* u, int T, int K, int d,
+                       float* out, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_bias_update -- [ANN] "Auxiliary-Loss-Free Load Balancing": after the
+ * step, b_i -= gamma for an expert loaded above the batch mean T*K/E, b_i +=
+ * gamma below it, unchanged at it (fp32).  counts are routed pairs per
+ * expert over the whole batch of T tokens (sum over data-parallel ranks).
+ *   counts int32 [E], bias fp32 [E] (updated in place)
+ */
+moe_status moe_bias_update(const int32_t* counts, int E, int64_t T, int K, float gamma,
+                           float* bias, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEFP8_H */
