@@ -59,7 +59,12 @@ V3_DECODE = MoEConfig("v3_decode", T=256, d=7168, E=256, G=8, M=4, K=8, I=2048,
 V4_PRO = MoEConfig("v4_pro", T=16384, d=7168, E=384, G=1, M=1, K=6, I=3072,
                    load_shape="hot", bias_lo=-0.01, bias_hi=0.01)
 
-PRESETS = {c.name: c for c in (TINY, V3_PREFILL, V3_DECODE, V4_PRO)}
+# Profiling case: V3 prefill's per-expert shapes (~128 rows per expert,
+# d=7168, I=2048) with 32 experts, so an ncu capture holds ~1.5 GB.
+V3_PREFILL_E32 = MoEConfig("v3_prefill_e32", T=512, d=7168, E=32, G=8, M=4, K=8, I=2048,
+                           bias_lo=-0.05, bias_hi=0.05)
+
+PRESETS = {c.name: c for c in (TINY, V3_PREFILL, V3_DECODE, V4_PRO, V3_PREFILL_E32)}
 
 
 @dataclass(frozen=True)
