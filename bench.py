@@ -167,7 +167,7 @@ def run_gpu(args):
     import torch.distributed as dist
 
     from fp8_block_scaled_sigmoid_b200 import _abi, configs, inputs
-    from fp8_block_scaled_sigmoid_b200.layer import MoELayer, make_fp8_weights
+    from fp8_block_scaled_sigmoid_b200.layer import MoELayer, make_fp8_weights, max_over_ranks
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -235,11 +235,7 @@ def run_gpu(args):
     step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
     per_kernel = {n: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)) / args.steps
                   for j, n in enumerate(names)}
-    total_ms = sum(step_ms)
-    if pg is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev, pg)
     tokens = cfg.T * world * args.steps
     value = tokens / (total_ms / 1e3)
 
@@ -257,11 +253,7 @@ def run_gpu(args):
         layer.forward_host(u_host, out_host)
         e2e_ev[i][1].record(st)
     barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    if pg is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), dev, pg)
     e2e_value = tokens / (e2e_ms / 1e3)
 
     # roofline of the dominant kernel (grouped GEMM 1 with the SwiGLU epilogue)

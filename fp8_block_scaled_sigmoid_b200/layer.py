@@ -27,6 +27,30 @@ from .configs import MoEConfig
 from . import inputs as _inputs
 
 
+def reduce_load_counts(counts: torch.Tensor, tokens_per_rank: int, process_group=None):
+    """Sum the per-expert routed-pair counts over the data-parallel ranks.
+
+    The bias update needs the load of the whole batch ("Auxiliary-Loss-Free
+    Load Balancing": loads are monitored over the whole batch of each step),
+    so every rank applies the same +-gamma.  Returns (counts, total tokens)."""
+    if process_group is None:
+        return counts, tokens_per_rank
+    import torch.distributed as dist
+    total = counts.clone()
+    dist.all_reduce(total, op=dist.ReduceOp.SUM, group=process_group)
+    return total, tokens_per_rank * dist.get_world_size(process_group)
+
+
+def max_over_ranks(value: float, device, process_group=None) -> float:
+    """Largest value over the ranks (a time: the job finishes with its slowest rank)."""
+    if process_group is None:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=process_group)
+    return float(t.item())
+
+
 def quantise_weight_stack(w_bf16: torch.Tensor, q=None, s=None):
     """128x128 block quantisation of a [G][N][K] bf16 stack on the device."""
     return _abi.fp8_quant_128x128(w_bf16, q, s)
@@ -118,13 +142,7 @@ class MoELayer:
         _abi.moe_combine(self.Y, self.perm["dst_of"], self.gate, self.Y[P:], u, self.out)
 
     def step_bias_update(self):
-        counts = self.perm["counts"]
-        T_all = self.T
-        if self.pg is not None:
-            import torch.distributed as dist
-            counts = counts.clone()
-            dist.all_reduce(counts, group=self.pg)
-            T_all = self.T * dist.get_world_size(self.pg)
+        counts, T_all = reduce_load_counts(self.perm["counts"], self.T, self.pg)
         _abi.moe_bias_update(counts, T_all, self.cfg.K, self.cfg.gamma, self.bias)
 
     # -- whole layer --------------------------------------------------------
