@@ -40,9 +40,9 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 384;       // 3 warpgroups
 constexpr int kEpiThreads = 256;    // warpgroups 1 and 2
 // Register split (setmaxnreg), checked against the launch budget of
-// 384 threads x 168 registers = 64512: 128 x 40 + 256 x 232 = 64512.
-constexpr int kRegsCtl = 40;
-constexpr int kRegsEpi = 232;
+// 384 threads x 168 registers = 64512: 128 x 56 + 256 x 224 = 64512.
+constexpr int kRegsCtl = 56;
+constexpr int kRegsEpi = 224;
 constexpr uint32_t kTmemCols = 512;
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 4096;
 
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(
         }
       }
       // every issued copy lands before the CTA can exit
-      const int first = std::max(0, it - kStages);
+      const int first = it > kStages ? it - kStages : 0;
       for (int i = first; i < it; ++i)
         mbar_wait(&full[i % kStages], (i / kStages) & 1, nullptr, args.dev_err);
     } else if (warp == 1 && lane == 0) {
@@ -220,9 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(
     for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
       const Work t = decode_work(w, nN, args);
       if (!t.ok) continue;
-      float acc[128];
+      // 128 fp32 accumulators as 64 packed pairs (packed fp32x2 FMA)
+      float2 acc[64];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
       const int64_t arow = static_cast<int64_t>(t.row0) + r_in;
       const int64_t arow_c = arow < args.a_rows ? arow : args.a_rows - 1;
       const float* sa_row = args.sa + arow_c * KB;
@@ -230,12 +231,28 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(
       const float* sb1 = sb0 + KB;
       const float* sb_lo = (EP == MOE_EP_F32) ? (g ? sb1 : sb0) : sb0;
       const float* sb_hi = (EP == MOE_EP_F32) ? (g ? sb1 : sb0) : sb1;
+      // the scales of the next two K blocks are in flight while this one is
+      // folded in (their global-load latency would otherwise stall every block)
+      float a_n0 = __ldg(sa_row), lo_n0 = __ldg(sb_lo), hi_n0 = __ldg(sb_hi);
+      float a_n1 = 0.f, lo_n1 = 0.f, hi_n1 = 0.f;
+      if (KB > 1) {
+        a_n1 = __ldg(sa_row + 1);
+        lo_n1 = __ldg(sb_lo + 1);
+        hi_n1 = __ldg(sb_hi + 1);
+      }
       for (int kb = 0; kb < KB; ++kb, ++tit) {
         const int p = tit & 1;
         const uint32_t tph = (tit >> 1) & 1;
-        const float s_a = __ldg(sa_row + kb);
-        const float f_lo = __fmul_rn(s_a, __ldg(sb_lo + kb));
-        const float f_hi = __fmul_rn(s_a, __ldg(sb_hi + kb));
+        const float f_lo = __fmul_rn(a_n0, lo_n0);
+        const float f_hi = __fmul_rn(a_n0, hi_n0);
+        a_n0 = a_n1;
+        lo_n0 = lo_n1;
+        hi_n0 = hi_n1;
+        if (kb + 2 < KB) {
+          a_n1 = __ldg(sa_row + kb + 2);
+          lo_n1 = __ldg(sb_lo + kb + 2);
+          hi_n1 = __ldg(sb_hi + kb + 2);
+        }
         // warp-uniform outcome: the TMEM loads below are warp-collective
         if (!__all_sync(0xffffffffu, mbar_wait(&tfull[p], tph, abort_v, args.dev_err))) {
           live = false;
@@ -243,26 +260,29 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(
         }
         tc_fence_after();
         const uint32_t ta = tmem + lane_base + static_cast<uint32_t>(p * kBN);
-        float v[32];
-        tmem_ld32(ta + c_lo, v);
+        // two 32-column loads in flight per wait
+        float v0[32], v1[32];
+        tmem_ld32(ta + c_lo, v0);
+        tmem_ld32(ta + c_lo + 32, v1);
         tmem_ld_wait();
+        const float2 flo = make_float2(f_lo, f_lo);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = fmaf(v[i], f_lo, acc[i]);
-        tmem_ld32(ta + c_lo + 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[32 + i] = fmaf(v[i], f_lo, acc[32 + i]);
-        tmem_ld32(ta + c_hi, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[64 + i] = fmaf(v[i], f_hi, acc[64 + i]);
-        tmem_ld32(ta + c_hi + 32, v);
+        for (int i = 0; i < 16; ++i) {
+          acc[i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), flo, acc[i]);
+          acc[16 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), flo, acc[16 + i]);
+        }
+        tmem_ld32(ta + c_hi, v0);
+        tmem_ld32(ta + c_hi + 32, v1);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[p]);
+        const float2 fhi = make_float2(f_hi, f_hi);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[96 + i] = fmaf(v[i], f_hi, acc[96 + i]);
+        for (int i = 0; i < 16; ++i) {
+          acc[32 + i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), fhi, acc[32 + i]);
+          acc[48 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), fhi, acc[48 + i]);
+        }
       }
       if (!live) break;
       const bool row_ok = r_in < t.rows;
@@ -272,16 +292,19 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             reinterpret_cast<float4*>(dst)[i] =
-                make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+                make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x, acc[2 * i + 1].y);
         }
       } else {
         // h = SiLU(gate) * up for this thread's 64 channels, then the 1x128
         // tile amax is shared with the partner thread of the other half.
+        // gate channels are acc[0..31] (packed pairs), the matching up channels acc[32..63]
+        float h[64];
         float amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          acc[i] = silu_mul(acc[i], acc[64 + i]);
-          amax = fmaxf(amax, fabsf(acc[i]));
+        for (int i = 0; i < 32; ++i) {
+          h[2 * i] = silu_mul(acc[i].x, acc[32 + i].x);
+          h[2 * i + 1] = silu_mul(acc[i].y, acc[32 + i].y);
+          amax = fmaxf(amax, fmaxf(fabsf(h[2 * i]), fabsf(h[2 * i + 1])));
         }
         const int xb = xtile & 1;
         amax_x[(xb * 2 + g) * 128 + r_in] = amax;
@@ -297,14 +320,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 o;
-            o.x = e4m3x4(__fdiv_rn(acc[16 * i + 0], s), __fdiv_rn(acc[16 * i + 1], s),
-                         __fdiv_rn(acc[16 * i + 2], s), __fdiv_rn(acc[16 * i + 3], s));
-            o.y = e4m3x4(__fdiv_rn(acc[16 * i + 4], s), __fdiv_rn(acc[16 * i + 5], s),
-                         __fdiv_rn(acc[16 * i + 6], s), __fdiv_rn(acc[16 * i + 7], s));
-            o.z = e4m3x4(__fdiv_rn(acc[16 * i + 8], s), __fdiv_rn(acc[16 * i + 9], s),
-                         __fdiv_rn(acc[16 * i + 10], s), __fdiv_rn(acc[16 * i + 11], s));
-            o.w = e4m3x4(__fdiv_rn(acc[16 * i + 12], s), __fdiv_rn(acc[16 * i + 13], s),
-                         __fdiv_rn(acc[16 * i + 14], s), __fdiv_rn(acc[16 * i + 15], s));
+            o.x = e4m3x4(__fdiv_rn(h[16 * i + 0], s), __fdiv_rn(h[16 * i + 1], s),
+                         __fdiv_rn(h[16 * i + 2], s), __fdiv_rn(h[16 * i + 3], s));
+            o.y = e4m3x4(__fdiv_rn(h[16 * i + 4], s), __fdiv_rn(h[16 * i + 5], s),
+                         __fdiv_rn(h[16 * i + 6], s), __fdiv_rn(h[16 * i + 7], s));
+            o.z = e4m3x4(__fdiv_rn(h[16 * i + 8], s), __fdiv_rn(h[16 * i + 9], s),
+                         __fdiv_rn(h[16 * i + 10], s), __fdiv_rn(h[16 * i + 11], s));
+            o.w = e4m3x4(__fdiv_rn(h[16 * i + 12], s), __fdiv_rn(h[16 * i + 13], s),
+                         __fdiv_rn(h[16 * i + 14], s), __fdiv_rn(h[16 * i + 15], s));
             reinterpret_cast<uint4*>(dst)[i] = o;
           }
           if (g == 0) args.d_scale[arow * (I / 128) + t.n_idx] = s;

@@ -129,9 +129,16 @@ __global__ void __launch_bounds__(kRtThreads, 1) router_logits_kernel(
       tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c, v);
       tmem_ld_wait();
       if (row < T) {
+        if (n0 + c + 16 <= E) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (n0 + c + j < E) dst[n0 + c + j] = v[j];
+          for (int j = 0; j < 4; ++j)
+            reinterpret_cast<float4*>(dst + n0 + c)[j] =
+                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (n0 + c + j < E) dst[n0 + c + j] = v[j];
+        }
       }
     }
   }
@@ -199,8 +206,10 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
   uint32_t allowed = 0xffffffffu;
   if (M < G) {
     const int n_top = K / M;
-    float my_score = -INFINITY;
-    for (int g = 0; g < G; ++g) {
+    const int L = gs / P;  // lanes per group when a group spans whole lanes
+    if (gs % P == 0 && L > 0 && L <= 32 && (L & (L - 1)) == 0) {
+      // every group sits on L consecutive lanes: all groups at once with
+      // segmented (xor < L) reductions
       uint32_t tk = 0;
       float sum = 0.f;
       for (int r = 0; r < n_top; ++r) {
@@ -208,23 +217,59 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
 #pragma unroll
         for (int i = 0; i < P; ++i) {
           const int e = e0 + i;
-          if (e < E && e / gs == g && !((tk >> i) & 1u) && better(beta[i], e, c.v, c.i)) {
+          if (e < E && !((tk >> i) & 1u) && better(beta[i], e, c.v, c.i)) {
             c.v = beta[i];
             c.i = e;
           }
         }
-        c = warp_best(c);
+        for (int off = 1; off < L; off <<= 1) {
+          const float v = __shfl_xor_sync(0xffffffffu, c.v, off);
+          const int i = __shfl_xor_sync(0xffffffffu, c.i, off);
+          if (better(v, i, c.v, c.i)) {
+            c.v = v;
+            c.i = i;
+          }
+        }
         if (c.i / P == lane) tk |= 1u << (c.i - e0);
         sum = __fadd_rn(sum, c.v);
       }
-      if (lane == g) my_score = sum;
+      const int my_g = lane / L;
+      int rank = 0;
+      for (int g = 0; g < G; ++g) {
+        const float v = __shfl_sync(0xffffffffu, sum, g * L);
+        if (better(v, g, sum, my_g)) ++rank;
+      }
+      const uint32_t lead = __ballot_sync(0xffffffffu, (lane % L) == 0 && my_g < G && rank < M);
+      allowed = 0;
+      for (int g = 0; g < G; ++g) allowed |= ((lead >> (g * L)) & 1u) << g;
+    } else {
+      float my_score = -INFINITY;
+      for (int g = 0; g < G; ++g) {
+        uint32_t tk = 0;
+        float sum = 0.f;
+        for (int r = 0; r < n_top; ++r) {
+          Cand c{-INFINITY, INT_MAX, 0.f};
+#pragma unroll
+          for (int i = 0; i < P; ++i) {
+            const int e = e0 + i;
+            if (e < E && e / gs == g && !((tk >> i) & 1u) && better(beta[i], e, c.v, c.i)) {
+              c.v = beta[i];
+              c.i = e;
+            }
+          }
+          c = warp_best(c);
+          if (c.i / P == lane) tk |= 1u << (c.i - e0);
+          sum = __fadd_rn(sum, c.v);
+        }
+        if (lane == g) my_score = sum;
+      }
+      int rank = 0;
+      for (int g = 0; g < G; ++g) {
+        const float v = __shfl_sync(0xffffffffu, my_score, g);
+        if (better(v, g, my_score, lane)) ++rank;
+      }
+      allowed = __ballot_sync(0xffffffffu, lane < G && rank < M);
     }
-    int rank = 0;
-    for (int g = 0; g < G; ++g) {
-      const float v = __shfl_sync(0xffffffffu, my_score, g);
-      if (better(v, g, my_score, lane)) ++rank;
-    }
-    allowed = __ballot_sync(0xffffffffu, lane < G && rank < M);
   }
 
   uint32_t taken = 0;
