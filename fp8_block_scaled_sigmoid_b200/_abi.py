@@ -35,6 +35,8 @@ _SIGS = {
     "moe_permute_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
     "moe_permute": (_i, [_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                          _p, _sz, _p, _p]),
+    "moe_permute_noalloc": (_i, [_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p,
+                                 _p, _p, _p, _p]),
     "moe_tile_table": (_i, [_p, _i, _i, _p, _p, _p, _p, _p]),
     "grouped_gemm_fp8_blockscaled": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
                                           _i, _p, _p, _p, _p]),
@@ -52,7 +54,8 @@ _lib = None
 
 # Kernels each entry point launches (for the benchmark's launch count).
 LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant": 1,
-                     "moe_route": 2, "moe_permute": 4, "moe_tile_table": 1,
+                     "moe_route": 2, "moe_permute": 4, "moe_permute_noalloc": 4,
+                     "moe_tile_table": 1,
                      "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1}
 launch_count = 0
 
@@ -224,6 +227,43 @@ def moe_permute(topk_idx, E, xq, xscale, with_shared=True, out=None, ws=None, de
                              _ptr(tile_start), _ptr(n_tiles), _ptr(ws),
                              ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream)),
            "moe_permute")
+    o["max_tiles"] = mt
+    return o
+
+
+def moe_permute_noalloc(topk_idx, E, xq, xscale, with_shared=True, out=None, dev_err=None,
+                        stream=None):
+    """moe_permute without a workspace argument: the library's fixed 1 MiB
+    device scratch array is used instead (for callers that cannot allocate;
+    calls must not overlap on the GPU).  Returns the same dict as moe_permute."""
+    T, K = topk_idx.shape
+    d = xq.shape[1]
+    dev = _dev(topk_idx)
+    groups = E + (1 if with_shared else 0)
+    o = {} if out is None else out
+    mt = moe_max_m_tiles(T, K, E, with_shared)
+
+    def get(name, shape, dtype):
+        if name not in o:
+            o[name] = torch.empty(shape, dtype=dtype, device=dev)
+        return o[name]
+
+    counts = get("counts", (E,), torch.int32)
+    offsets = get("offsets", (groups + 1,), torch.int32)
+    src_row = get("src_row", (T * K,), torch.int32)
+    dst_of = get("dst_of", (T, K), torch.int32)
+    xq_perm = get("xq_perm", (T * K, d), torch.uint8)
+    xs_perm = get("xs_perm", (T * K, d // 128), torch.float32)
+    tile_group = get("tile_group", (max(mt, 1),), torch.int32)
+    tile_start = get("tile_start", (groups + 1,), torch.int32)
+    n_tiles = get("n_tiles", (1,), torch.int32)
+    _count("moe_permute_noalloc")
+    _check(lib().moe_permute_noalloc(_ptr(topk_idx), T, K, E, int(bool(with_shared)), _ptr(xq),
+                                     _ptr(xscale), d, _ptr(counts), _ptr(offsets), _ptr(src_row),
+                                     _ptr(dst_of), _ptr(xq_perm), _ptr(xs_perm),
+                                     _ptr(tile_group), _ptr(tile_start), _ptr(n_tiles),
+                                     _ptr(dev_err), _stream(stream)),
+           "moe_permute_noalloc")
     o["max_tiles"] = mt
     return o
 

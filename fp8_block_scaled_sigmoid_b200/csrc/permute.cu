@@ -16,6 +16,8 @@
 //                ascending token order.
 //  4. gather  -- one warp per destination row copies the FP8 row (16-byte
 //                vectors, coalesced) and its 1x128 scales.
+#include <mutex>
+
 #include "moe_common.cuh"
 
 namespace moe {
@@ -295,4 +297,71 @@ extern "C" moe_status moe_tile_table(const int32_t* offsets, int groups, int max
       offsets, groups, max_tiles, tile_group, tile_start, n_tiles, dev_err);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: moe_permute for callers that cannot allocate device
+// memory at call time.  Inference-runtime plugins whose host framework owns
+// and plans all device memory (and offers the plugin no workspace), and
+// latency-critical paths that must not hit cudaMalloc's implicit device-wide
+// synchronisation, can still run the permutation: its scratch (per-chunk
+// expert counts) lives in a fixed file-scope device array instead of a
+// caller buffer.
+//
+// The array is kNoAllocScratchInts int32 (1 MiB) and exists on every device
+// that loads the library, for as long as the library stays loaded.  Every
+// call shares it and it keeps the last call's contents; nothing in it needs
+// clearing, because the count kernel overwrites every entry the later kernels
+// read.  Calls that overlap on the GPU (two streams, or two host threads)
+// race on the array and must be serialised by the caller.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchInts = size_t(1) << 18;
+static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocScratchInts];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64] = {nullptr};
+
+// Device address of the array for the current device; looked up once per
+// device (host code may not use the symbol's name as a device pointer).
+void* scratch_for_current_device(moe_status* st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *st = MOE_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p) {
+      *st = MOE_ERR_CUDA;
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = p;
+  }
+  *st = MOE_OK;
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" moe_status moe_permute_noalloc(const int32_t* topk_idx, int T, int K, int E,
+                                          int with_shared, const uint8_t* xq,
+                                          const float* xscale, int d, int32_t* counts,
+                                          int32_t* offsets, int32_t* src_row, int32_t* dst_of,
+                                          uint8_t* xq_perm, float* xscale_perm,
+                                          int32_t* tile_group, int32_t* tile_start,
+                                          int32_t* n_tiles, int32_t* dev_err,
+                                          moe_stream_t stream) {
+  size_t need = 0;
+  const moe_status q = moe_permute_workspace_size(T, K, E, &need);
+  if (q != MOE_OK) return q;
+  if (need > kNoAllocScratchInts * sizeof(int32_t)) return MOE_ERR_UNSUPPORTED;
+  moe_status st = MOE_OK;
+  void* ws = scratch_for_current_device(&st);
+  if (st != MOE_OK) return st;
+  return moe_permute(topk_idx, T, K, E, with_shared, xq, xscale, d, counts, offsets, src_row,
+                     dst_of, xq_perm, xscale_perm, tile_group, tile_start, n_tiles, ws,
+                     kNoAllocScratchInts * sizeof(int32_t), dev_err, stream);
 }

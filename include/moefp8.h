@@ -150,6 +150,31 @@ moe_status moe_permute(const int32_t* topk_idx, int T, int K, int E, int with_sh
                        moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_permute_noalloc -- moe_permute without a caller workspace.  The pages
+ * have no counterpart: it is a deployment convenience.  It serves callers
+ * that cannot allocate device memory at call time -- plugins of inference
+ * runtimes whose host framework owns and plans all device memory and gives
+ * the plugin no workspace, and latency-critical paths that must not incur
+ * cudaMalloc's implicit device-wide synchronisation.
+ * Arguments, outputs and errors are those of moe_permute minus ws/ws_bytes.
+ * Its scratch is a fixed 1 MiB file-scope device array (262144 int32), held
+ * by every device that loads the library until the library is unloaded; a
+ * batch whose moe_permute_workspace_size exceeds 1 MiB (ceil(T/128) * E int32
+ * entries) returns MOE_ERR_UNSUPPORTED before anything is launched.  The
+ * first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the array and it keeps the last call's contents (nothing in
+ * it needs clearing); calls that overlap on the GPU race on it, so the caller
+ * must serialise them.  It allocates nothing.
+ */
+moe_status moe_permute_noalloc(const int32_t* topk_idx, int T, int K, int E, int with_shared,
+                               const uint8_t* xq, const float* xscale, int d, int32_t* counts,
+                               int32_t* offsets, int32_t* src_row, int32_t* dst_of,
+                               uint8_t* xq_perm, float* xscale_perm, int32_t* tile_group,
+                               int32_t* tile_start, int32_t* n_tiles, int32_t* dev_err,
+                               moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_tile_table -- the 128-row tile table of arbitrary segment offsets (for
  * grouped GEMM calls whose segments do not come from moe_permute).
  *   offsets int32 [groups+1], non-decreasing, device
