@@ -402,6 +402,56 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_gemm(args):
+    """Standalone block-scaled GEMM: A 4096x7168 (1x128 tiles, 1% outliers
+    x50) times B^T, B 7168x2048 (128x128 blocks), fp32 out."""
+    import torch
+
+    from fp8_block_scaled_sigmoid_b200 import _abi, configs, inputs
+
+    dev = torch.device("cuda", 0)
+    cfg = configs.STANDALONE_GEMM
+    a, bt = inputs.draw_gemm(cfg, dev)
+    aq, sa = _abi.fp8_quant_1x128(a)
+    bq, sb = _abi.fp8_quant_128x128(bt.unsqueeze(0))
+    offs = torch.tensor([0, cfg.M], dtype=torch.int32, device=dev)
+    mt = cfg.M // 128
+    tg, ts, nt = _abi.moe_tile_table(offs, mt)
+    D = torch.empty(cfg.M, cfg.N, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        _abi.grouped_gemm_fp8_blockscaled(aq, sa, bq, sb, offs, tg, ts, nt, mt, D=D)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    times = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        _abi.grouped_gemm_fp8_blockscaled(aq, sa, bq, sb, offs, tg, ts, nt, mt, D=D)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    clocks = sampler.stop()
+    peaks, src = load_peaks()
+    fp8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    ms = statistics.median(times)
+    tf = cfg.flops / (ms / 1e3) / 1e12
+    print(json.dumps({
+        "metric": "standalone block-scaled FP8 GEMM TFLOP/s", "value": round(tf, 1),
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "dtype": "fp8_e4m3",
+        "config": {"workload": f"{cfg.name}: A {cfg.M}x{cfg.K} (1x128 scales, 1% outliers x50) "
+                               f"x B^T {cfg.N}x{cfg.K} (128x128 scales), fp32 out",
+                   "l2": "512 MB buffer written between timed launches"},
+        "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": fp8_peak,
+                     "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4),
+                     "peak_source": f"2 x {src} bf16_tflops (nominal fp8:bf16 ratio)"},
+        "clocks": clocks}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -410,11 +460,15 @@ def main():
     ap.add_argument("--config", default="v3_prefill")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm", action="store_true",
+                    help="time the standalone 4096x7168x2048 block-scaled GEMM instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.gemm:
+        run_gemm(args)
     else:
         run_gpu(args)
 

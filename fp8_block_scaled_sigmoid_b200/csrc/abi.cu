@@ -45,7 +45,7 @@ EncodeTiledFn get_encode_fn() {
 
 bool moe_make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                       uint64_t inner_elems, uint64_t outer_rows, uint64_t row_stride_bytes,
-                      uint32_t box_inner, uint32_t box_outer) {
+                      uint32_t box_inner, uint32_t box_outer, int swizzle_bytes) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner_elems, outer_rows};
@@ -53,7 +53,10 @@ bool moe_make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                      : (swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                             : CU_TENSOR_MAP_SWIZZLE_128B),
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

@@ -7,36 +7,58 @@
 // partial sums to fp32 registers every N_C = 128 elements and apply the
 // scales there.  On Blackwell the same contract maps onto:
 //
-//   * one 128x256x128 block product per K-block = 4 tcgen05.mma (K=32 each)
-//     from a TMA-fed, 128-byte-swizzled shared-memory ring into a fresh TMEM
+//   * one 128x256x128 block product per K block = 4 tcgen05.mma (K=32 each)
+//     from a TMA-fed, swizzled shared-memory ring into a fresh TMEM
 //     accumulator (two 256-column buffers, ping-pong);
 //   * two epilogue warpgroups drain each finished buffer with tcgen05.ld and
 //     fold it into fp32 register accumulators: acc += (sa[row,kb] *
-//     sb[nblk,kb]) * partial, while the tensor core fills the other buffer;
-//   * a persistent grid (one CTA per SM) walks the (expert, n-tile, m-tile)
-//     work list derived on the device from the segment tile table, so the
-//     ragged expert segments need no host synchronisation; the m-tiles of one
-//     expert that share a weight tile run next to each other for L2 reuse.
+//     sb[nblk,kb]) * partial (packed fp32x2 FMA), while the tensor core fills
+//     the other buffer;
+//   * a persistent grid walks the (expert, n-tile, m-tile) work list derived
+//     on the device from the segment offsets, so the ragged expert segments
+//     need no host synchronisation; the m-tiles of one expert that share a
+//     weight tile run next to each other for L2 reuse.
+//
+// The shared-memory ring is staged in K slices of SK bytes (128, or 64 with
+// the 64-byte swizzle): a stage is released as soon as the MMAs of its slice
+// complete.  Measured on V3-prefill shapes, 128-byte slices are faster (the
+// 64-byte ones halve the contiguous bytes each weight row contributes to a
+// TMA box), so 128 is the default.
+//
+// Two forms of the mainloop share the epilogue:
+//   gemm1sm  -- one CTA computes a 128 x 256 tile (tcgen05 cta_group::1);
+//   gemm2sm  -- a CTA pair (cluster of 2) computes a 256 x 256 tile with
+//               tcgen05.mma.cta_group::2: each CTA stages its 128 rows of A
+//               and 128 of the 256 weight rows, a weight tile is streamed
+//               once per pair, and each CTA's TMEM holds its rows' partial.
+//               It does more padded work when experts hold ~128 rows (V3
+//               prefill), where the 1-SM form is faster; it is kept for
+//               segments of 256+ rows.
 //
 // Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
-// TMEM owner, warps 2-3 idle (the first warpgroup gives its registers to the
-// other two), warps 4..11 = epilogue (warp w reads TMEM lanes 32*(w%4)..).
-// Epilogues: fp32 rows, or SwiGLU + 1x128 E4M3 requantisation of h (the W1
-// rows are gate/up block-interleaved so one 256-wide tile holds 128 gate and
-// the matching 128 up channels).
+// TMEM owner, warp 2 builds the work list then idles with warp 3 (the first
+// warpgroup gives registers to the other two), warps 4..11 = epilogue (warp w
+// reads TMEM lanes 32*(w%4)..).  Epilogues: fp32 rows, or SwiGLU + 1x128 E4M3
+// requantisation of h (the W1 rows are gate/up block-interleaved so one
+// 256-wide tile holds 128 gate and the matching 128 up channels).  Every
+// wait is bounded (MOE_DEVERR_TIMEOUT).
 #include <algorithm>
 
 #include "epi_math.cuh"
 #include "moe_common.cuh"
 
+// Mainloop form and stage width (build-time choices).
+#ifndef MOE_GEMM_PAIR
+#define MOE_GEMM_PAIR 0
+#endif
+#ifndef MOE_GEMM_SK
+#define MOE_GEMM_SK 128
+#endif
+
 namespace moe {
 namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;
-constexpr int kStages = 4;
-constexpr int kABytes = kBM * kBK;
-constexpr int kBBytes = kBN * kBK;
-constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 384;       // 3 warpgroups
 constexpr int kEpiThreads = 256;    // warpgroups 1 and 2
 // Register split (setmaxnreg), checked against the launch budget of
@@ -44,7 +66,9 @@ constexpr int kEpiThreads = 256;    // warpgroups 1 and 2
 constexpr int kRegsCtl = 56;
 constexpr int kRegsEpi = 224;
 constexpr uint32_t kTmemCols = 512;
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 4096;
+constexpr int kRingBytes = 192 * 1024;
+constexpr int kMaxGroups = 1024;
+constexpr size_t kSmemBytes = 1024 + kRingBytes + 512 + (kMaxGroups + 1) * 4 + 2048 + 64;
 
 struct GemmArgs {
   const float* sa;
@@ -61,86 +85,280 @@ struct GemmArgs {
 };
 
 struct Work {
-  int e, n_idx, row0, rows;
+  int e, n_idx, row0, rows;  // row0 / rows: the rows this CTA owns
   bool ok;
 };
 
-// Work item w -> (expert, n-tile, m-tile).  The items of expert e occupy
-// [nN*tile_start[e], nN*tile_start[e+1]); inside, the m-tile varies fastest.
-__device__ __forceinline__ Work decode_work(int w, int nN, const GemmArgs& a) {
+template <int SK>
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
+  static_assert(SK == 128 || SK == 64, "stage K width");
+  return SK == 128 ? smem_desc_sw128(addr) : smem_desc_sw64(addr);
+}
+
+// rstart[g] = number of RT-row tiles of the groups before g (one warp).
+template <int RT>
+__device__ void build_tile_prefix(const GemmArgs& a, int* rstart, int lane) {
+  const int G = a.groups;
+  const int per = (G + 31) / 32;
+  const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+  int mine = 0;
+  for (int g = g0; g < g1; ++g) {
+    const int c = __ldg(a.offsets + g + 1) - __ldg(a.offsets + g);
+    if (c < 0) set_dev_err(a.dev_err, MOE_DEVERR_BAD_TABLE);
+    mine += c > 0 ? (c + RT - 1) / RT : 0;
+  }
+  int incl = mine;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += n;
+  }
+  int run = incl - mine;
+  for (int g = g0; g < g1; ++g) {
+    rstart[g] = run;
+    const int c = __ldg(a.offsets + g + 1) - __ldg(a.offsets + g);
+    run += c > 0 ? (c + RT - 1) / RT : 0;
+  }
+  if (lane == 31) rstart[G] = incl;
+}
+
+// Work item w -> (expert, n-tile, RT-row tile); the items of expert e occupy
+// [nN*rstart[e], nN*rstart[e+1]) and the row tile varies fastest inside.
+// `sub` selects this CTA's 128-row half of a 256-row pair tile.
+template <int RT>
+__device__ __forceinline__ Work decode_work(int w, int nN, const int* rstart, const GemmArgs& a,
+                                            int sub) {
   Work t{0, 0, 0, 0, false};
   const int j = w / nN;
-  const int e = __ldg(a.tile_group + j);
-  if (e < 0 || e >= a.groups) return t;
-  const int ms = __ldg(a.tile_start + e);
-  const int mc = __ldg(a.tile_start + e + 1) - ms;
-  if (mc <= 0 || j < ms || j >= ms + mc) return t;
-  const int local = w - nN * ms;
-  t.n_idx = local / mc;
-  const int m_loc = local - t.n_idx * mc;
-  const int r0 = __ldg(a.offsets + e) + kBM * m_loc;
-  const int r1 = __ldg(a.offsets + e + 1);
-  t.rows = min(kBM, r1 - r0);
-  if (t.rows <= 0 || r0 < 0 || r1 > a.a_rows || t.n_idx >= nN) return t;
+  int lo = 0, hi = a.groups - 1;
+  while (lo < hi) {  // last group whose first tile index is <= j
+    const int mid = (lo + hi + 1) >> 1;
+    if (rstart[mid] <= j) lo = mid;
+    else hi = mid - 1;
+  }
+  const int e = lo;
+  const int tc = rstart[e + 1] - rstart[e];
+  if (tc <= 0 || j < rstart[e] || j >= rstart[e] + tc) return t;
+  const int local = w - nN * rstart[e];
+  t.n_idx = local / tc;
+  const int mt = local - t.n_idx * tc;
+  const int seg0 = __ldg(a.offsets + e), seg1 = __ldg(a.offsets + e + 1);
+  const int tile0 = seg0 + RT * mt;
+  if (tile0 >= seg1 || seg1 > a.a_rows || t.n_idx >= nN) return t;
+  t.row0 = tile0 + 128 * sub;
+  t.rows = max(0, min(128, seg1 - t.row0));
   t.e = e;
-  t.row0 = r0;
   t.ok = true;
   return t;
 }
 
-template <int EP>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(
+// ------------------------------------------------------------------ epilogue
+// Promotes every K block of one tile into fp32 registers and writes the
+// tile.  Returns false if a bounded wait gave up.  PAIR: the TMEM buffer is
+// released on the even CTA's barrier.
+template <int EP, bool PAIR>
+__device__ __forceinline__ bool epilogue_tile(const GemmArgs& args, const Work& t, uint32_t tmem,
+                                              int warp, int lane, int KB, int N, int& tit,
+                                              int& xtile, uint64_t* tfull, uint64_t* tempty,
+                                              uint64_t* xbar, float* amax_x,
+                                              volatile int* abort_v) {
+  const int g = (warp - 4) >> 2;   // which half of the columns
+  const int q = warp & 3;          // TMEM lane quarter this warp may read
+  const int r_in = q * 32 + lane;  // row inside the tile
+  const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+  // columns of the 256-wide tile this thread accumulates (two runs of 64)
+  const int c_lo = (EP == MOE_EP_F32) ? 128 * g : 64 * g;
+  const int c_hi = (EP == MOE_EP_F32) ? 128 * g + 64 : 128 + 64 * g;
+  // 128 fp32 accumulators as 64 packed pairs (packed fp32x2 FMA)
+  float2 acc[64];
+#pragma unroll
+  for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
+  const int64_t arow = static_cast<int64_t>(t.row0) + r_in;
+  const int64_t arow_c = arow < args.a_rows ? arow : args.a_rows - 1;
+  const float* sa_row = args.sa + arow_c * KB;
+  const float* sb0 = args.sb + (static_cast<int64_t>(t.e) * (N / 128) + t.n_idx * 2) * KB;
+  const float* sb1 = sb0 + KB;
+  const float* sb_lo = (EP == MOE_EP_F32) ? (g ? sb1 : sb0) : sb0;
+  const float* sb_hi = (EP == MOE_EP_F32) ? (g ? sb1 : sb0) : sb1;
+  // the scales of the next two K blocks are in flight while this one is
+  // folded in
+  float a_n0 = __ldg(sa_row), lo_n0 = __ldg(sb_lo), hi_n0 = __ldg(sb_hi);
+  float a_n1 = 0.f, lo_n1 = 0.f, hi_n1 = 0.f;
+  if (KB > 1) {
+    a_n1 = __ldg(sa_row + 1);
+    lo_n1 = __ldg(sb_lo + 1);
+    hi_n1 = __ldg(sb_hi + 1);
+  }
+  for (int kb = 0; kb < KB; ++kb, ++tit) {
+    const int p = tit & 1;
+    const uint32_t tph = (tit >> 1) & 1;
+    const float f_lo = __fmul_rn(a_n0, lo_n0);
+    const float f_hi = __fmul_rn(a_n0, hi_n0);
+    a_n0 = a_n1;
+    lo_n0 = lo_n1;
+    hi_n0 = hi_n1;
+    if (kb + 2 < KB) {
+      a_n1 = __ldg(sa_row + kb + 2);
+      lo_n1 = __ldg(sb_lo + kb + 2);
+      hi_n1 = __ldg(sb_hi + kb + 2);
+    }
+    // warp-uniform outcome: the TMEM loads below are warp-collective
+    if (!__all_sync(0xffffffffu, mbar_wait(&tfull[p], tph, abort_v, args.dev_err))) return false;
+    tc_fence_after();
+    const uint32_t ta = tmem + lane_base + static_cast<uint32_t>(p * kBN);
+    // two 32-column loads in flight per wait
+    float v0[32], v1[32];
+    tmem_ld32(ta + c_lo, v0);
+    tmem_ld32(ta + c_lo + 32, v1);
+    tmem_ld_wait();
+    const float2 flo = make_float2(f_lo, f_lo);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      acc[i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), flo, acc[i]);
+      acc[16 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), flo, acc[16 + i]);
+    }
+    tmem_ld32(ta + c_hi, v0);
+    tmem_ld32(ta + c_hi + 32, v1);
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      if (PAIR) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[p]), 0));
+      else mbar_arrive(&tempty[p]);
+    }
+    const float2 fhi = make_float2(f_hi, f_hi);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      acc[32 + i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), fhi, acc[32 + i]);
+      acc[48 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), fhi, acc[48 + i]);
+    }
+  }
+  const bool row_ok = r_in < t.rows;
+  if (EP == MOE_EP_F32) {
+    if (row_ok) {
+      float* dst = static_cast<float*>(args.D) + arow * N + t.n_idx * kBN + 128 * g;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        reinterpret_cast<float4*>(dst)[i] =
+            make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x, acc[2 * i + 1].y);
+    }
+  } else {
+    // h = SiLU(gate) * up overwrites the gate accumulators: h[2i], h[2i+1]
+    // are acc[i].x, acc[i].y; the up channels are acc[32..63]
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      acc[i].x = silu_mul(acc[i].x, acc[32 + i].x);
+      acc[i].y = silu_mul(acc[i].y, acc[32 + i].y);
+      amax = fmaxf(amax, fmaxf(fabsf(acc[i].x), fabsf(acc[i].y)));
+    }
+    // the 1x128 tile amax is shared with the partner thread of the other half
+    const int xb = xtile & 1;
+    amax_x[(xb * 2 + g) * 128 + r_in] = amax;
+    mbar_arrive(&xbar[xb]);
+    if (!__all_sync(0xffffffffu, mbar_wait(&xbar[xb], (xtile >> 1) & 1, abort_v, args.dev_err)))
+      return false;
+    amax = fmaxf(amax_x[(xb * 2 + 0) * 128 + r_in], amax_x[(xb * 2 + 1) * 128 + r_in]);
+    ++xtile;
+    const float sq = quant_scale(amax);
+    if (row_ok) {
+      const int I = N / 2;
+      uint8_t* dst = static_cast<uint8_t*>(args.D) + arow * I + t.n_idx * 128 + 64 * g;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2* hp = acc + 8 * i;  // h[16i .. 16i+15]
+        uint4 o;
+        o.x = e4m3x4(__fdiv_rn(hp[0].x, sq), __fdiv_rn(hp[0].y, sq), __fdiv_rn(hp[1].x, sq),
+                     __fdiv_rn(hp[1].y, sq));
+        o.y = e4m3x4(__fdiv_rn(hp[2].x, sq), __fdiv_rn(hp[2].y, sq), __fdiv_rn(hp[3].x, sq),
+                     __fdiv_rn(hp[3].y, sq));
+        o.z = e4m3x4(__fdiv_rn(hp[4].x, sq), __fdiv_rn(hp[4].y, sq), __fdiv_rn(hp[5].x, sq),
+                     __fdiv_rn(hp[5].y, sq));
+        o.w = e4m3x4(__fdiv_rn(hp[6].x, sq), __fdiv_rn(hp[6].y, sq), __fdiv_rn(hp[7].x, sq),
+                     __fdiv_rn(hp[7].y, sq));
+        reinterpret_cast<uint4*>(dst)[i] = o;
+      }
+      if (g == 0) args.d_scale[arow * (I / 128) + t.n_idx] = sq;
+    }
+  }
+  return true;
+}
+
+// Shared-memory layout after the 1024-aligned ring.
+struct Ctl {
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  uint64_t* done;
+  uint64_t* xbar;
+  uint32_t* tmem_slot;
+  int* abort_flag;
+  int* rstart;
+  float* amax_x;  // [2][2][128]
+};
+
+template <int STAGES>
+__device__ __forceinline__ Ctl carve(uint8_t* base) {
+  Ctl c;
+  c.full = reinterpret_cast<uint64_t*>(base + kRingBytes);
+  c.empty = c.full + STAGES;
+  c.tfull = c.empty + STAGES;
+  c.tempty = c.tfull + 2;
+  c.done = c.tempty + 2;
+  c.xbar = c.done + 1;
+  c.tmem_slot = reinterpret_cast<uint32_t*>(c.xbar + 2);
+  c.abort_flag = reinterpret_cast<int*>(c.tmem_slot + 1);
+  c.rstart = reinterpret_cast<int*>(base + kRingBytes + 512);
+  c.amax_x = reinterpret_cast<float*>(c.rstart + kMaxGroups + 1);
+  return c;
+}
+
+// =========================================================== 1-SM mainloop
+template <int EP, int SK>
+__global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const GemmArgs args) {
+  constexpr int kSub = kBK / SK;                 // stages per K block
+  constexpr int kA = kBM * SK, kB = kBN * SK;    // stage bytes of A and B
+  constexpr int kStage = kA + kB;
+  constexpr int kStages = kRingBytes / kStage;
+  static_assert((2 * kStages + 8) * 8 + 8 <= 512, "barrier area");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* done = tempty + 2;
-  uint64_t* xbar = done + 1;  // [2] amax exchange between the two epilogue halves
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 2);
-  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  float* amax_x = reinterpret_cast<float*>(base + kStages * kStageBytes + 256);  // [2][2][128]
-
+  const Ctl c = carve<kStages>(base);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = args.N, KB = args.K / kBK, nN = N / kBN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], 1);
     }
     for (int p = 0; p < 2; ++p) {
-      mbar_init(&tfull[p], 1);
-      mbar_init(&tempty[p], kEpiThreads / 32);
+      mbar_init(&c.tfull[p], 1);
+      mbar_init(&c.tempty[p], kEpiThreads / 32);
     }
-    mbar_init(done, 1);
-    mbar_init(&xbar[0], kEpiThreads);
-    mbar_init(&xbar[1], kEpiThreads);
-    *abort_flag = 0;
+    mbar_init(c.done, 1);
+    mbar_init(&c.xbar[0], kEpiThreads);
+    mbar_init(&c.xbar[1], kEpiThreads);
+    *c.abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
+  if (warp == 2) build_tile_prefix<128>(args, c.rstart, lane);
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(c.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  volatile int* abort_v = abort_flag;
-
-  int n_mt = __ldg(args.n_tiles);
-  if (n_mt < 0 || n_mt > args.max_tiles) {
-    if (threadIdx.x == 0) set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
-    n_mt = 0;
-  }
-  const int total = n_mt * nN;
+  const uint32_t tmem = *c.tmem_slot;
+  volatile int* abort_v = c.abort_flag;
+  const int total = c.rstart[args.groups] * nN;
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
@@ -149,195 +367,228 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(
       int it = 0;
       bool live = true;
       for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
-        const Work t = decode_work(w, nN, args);
+        const Work t = decode_work<128>(w, nN, c.rstart, args, 0);
         if (!t.ok) {
           set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
           continue;
         }
         const int brow = t.e * N + t.n_idx * kBN;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int kk = 0; kk < KB * kSub; ++kk, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
-          if (!mbar_wait(&empty[s], ph ^ 1, abort_v, args.dev_err)) {
+          if (!mbar_wait(&c.empty[s], ph ^ 1, abort_v, args.dev_err)) {
             live = false;
             break;
           }
-          uint8_t* sA = base + s * kStageBytes;
-          mbar_arrive_expect_tx(&full[s], kStageBytes);
-          tma_load_2d(sA, &tmA, &full[s], kb * kBK, t.row0);
-          tma_load_2d(sA + kABytes, &tmB, &full[s], kb * kBK, brow);
+          uint8_t* sA = base + s * kStage;
+          mbar_arrive_expect_tx(&c.full[s], kStage);
+          tma_load_2d(sA, &tmA, &c.full[s], kk * SK, t.row0);
+          tma_load_2d(sA + kA, &tmB, &c.full[s], kk * SK, brow);
         }
       }
       // every issued copy lands before the CTA can exit
       const int first = it > kStages ? it - kStages : 0;
       for (int i = first; i < it; ++i)
-        mbar_wait(&full[i % kStages], (i / kStages) & 1, nullptr, args.dev_err);
+        mbar_wait(&c.full[i % kStages], (i / kStages) & 1, nullptr, args.dev_err);
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------- MMA issuer
       const uint32_t idesc = instr_desc(kFmtE4M3, kFmtE4M3, kBM, kBN);
       int it = 0, tit = 0;
       bool live = true;
       for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
-        const Work t = decode_work(w, nN, args);
+        const Work t = decode_work<128>(w, nN, c.rstart, args, 0);
         if (!t.ok) continue;
-        for (int kb = 0; kb < KB; ++kb, ++it, ++tit) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
+        for (int kb = 0; kb < KB && live; ++kb, ++tit) {
           const int p = tit & 1;
-          const uint32_t tph = (tit >> 1) & 1;
-          if (!mbar_wait(&tempty[p], tph ^ 1, abort_v, args.dev_err) ||
-              !mbar_wait(&full[s], ph, abort_v, args.dev_err)) {
+          if (!mbar_wait(&c.tempty[p], ((tit >> 1) & 1) ^ 1, abort_v, args.dev_err)) {
             live = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t sA = smem_u32(base + s * kStageBytes);
-          const uint64_t ad = smem_desc_sw128(sA);
-          const uint64_t bd = smem_desc_sw128(sA + kABytes);
           const uint32_t dt = tmem + static_cast<uint32_t>(p * kBN);
+          for (int h = 0; h < kSub; ++h, ++it) {
+            const int s = it % kStages;
+            if (!mbar_wait(&c.full[s], (it / kStages) & 1, abort_v, args.dev_err)) {
+              live = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sA = smem_u32(base + s * kStage);
+            const uint64_t ad = kmajor_desc<SK>(sA);
+            const uint64_t bd = kmajor_desc<SK>(sA + kA);
 #pragma unroll
-          for (int k = 0; k < kBK / 32; ++k) mma_f8f6f4(dt, ad + 2 * k, bd + 2 * k, idesc, k > 0);
-          mma_commit(&empty[s]);
-          mma_commit(&tfull[p]);
+            for (int k = 0; k < SK / 32; ++k)
+              mma_f8f6f4(dt, ad + 2 * k, bd + 2 * k, idesc, (h > 0 || k > 0) ? 1u : 0u);
+            mma_commit(&c.empty[s]);
+          }
+          if (live) mma_commit(&c.tfull[p]);
         }
       }
-      mma_commit(done);
-      mbar_wait(done, 0, nullptr, args.dev_err);
+      mma_commit(c.done);
+      mbar_wait(c.done, 0, nullptr, args.dev_err);
     }
+    __syncwarp();
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
-    // ------------------------------------------------------------ epilogue
-    const int ew = warp - 4;
-    const int g = ew >> 2;          // which half of the columns
-    const int q = warp & 3;         // TMEM lane quarter this warp may read
-    const int r_in = q * 32 + lane; // row inside the tile
-    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    // columns of the 256-wide tile this thread accumulates (two runs of 64)
-    const int c_lo = (EP == MOE_EP_F32) ? 128 * g : 64 * g;
-    const int c_hi = (EP == MOE_EP_F32) ? 128 * g + 64 : 128 + 64 * g;
     int tit = 0, xtile = 0;
-    bool live = true;
-    for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
-      const Work t = decode_work(w, nN, args);
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      const Work t = decode_work<128>(w, nN, c.rstart, args, 0);
       if (!t.ok) continue;
-      // 128 fp32 accumulators as 64 packed pairs (packed fp32x2 FMA)
-      float2 acc[64];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
-      const int64_t arow = static_cast<int64_t>(t.row0) + r_in;
-      const int64_t arow_c = arow < args.a_rows ? arow : args.a_rows - 1;
-      const float* sa_row = args.sa + arow_c * KB;
-      const float* sb0 = args.sb + (static_cast<int64_t>(t.e) * (N / 128) + t.n_idx * 2) * KB;
-      const float* sb1 = sb0 + KB;
-      const float* sb_lo = (EP == MOE_EP_F32) ? (g ? sb1 : sb0) : sb0;
-      const float* sb_hi = (EP == MOE_EP_F32) ? (g ? sb1 : sb0) : sb1;
-      // the scales of the next two K blocks are in flight while this one is
-      // folded in (their global-load latency would otherwise stall every block)
-      float a_n0 = __ldg(sa_row), lo_n0 = __ldg(sb_lo), hi_n0 = __ldg(sb_hi);
-      float a_n1 = 0.f, lo_n1 = 0.f, hi_n1 = 0.f;
-      if (KB > 1) {
-        a_n1 = __ldg(sa_row + 1);
-        lo_n1 = __ldg(sb_lo + 1);
-        hi_n1 = __ldg(sb_hi + 1);
-      }
-      for (int kb = 0; kb < KB; ++kb, ++tit) {
-        const int p = tit & 1;
-        const uint32_t tph = (tit >> 1) & 1;
-        const float f_lo = __fmul_rn(a_n0, lo_n0);
-        const float f_hi = __fmul_rn(a_n0, hi_n0);
-        a_n0 = a_n1;
-        lo_n0 = lo_n1;
-        hi_n0 = hi_n1;
-        if (kb + 2 < KB) {
-          a_n1 = __ldg(sa_row + kb + 2);
-          lo_n1 = __ldg(sb_lo + kb + 2);
-          hi_n1 = __ldg(sb_hi + kb + 2);
-        }
-        // warp-uniform outcome: the TMEM loads below are warp-collective
-        if (!__all_sync(0xffffffffu, mbar_wait(&tfull[p], tph, abort_v, args.dev_err))) {
-          live = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t ta = tmem + lane_base + static_cast<uint32_t>(p * kBN);
-        // two 32-column loads in flight per wait
-        float v0[32], v1[32];
-        tmem_ld32(ta + c_lo, v0);
-        tmem_ld32(ta + c_lo + 32, v1);
-        tmem_ld_wait();
-        const float2 flo = make_float2(f_lo, f_lo);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          acc[i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), flo, acc[i]);
-          acc[16 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), flo, acc[16 + i]);
-        }
-        tmem_ld32(ta + c_hi, v0);
-        tmem_ld32(ta + c_hi + 32, v1);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[p]);
-        const float2 fhi = make_float2(f_hi, f_hi);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          acc[32 + i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), fhi, acc[32 + i]);
-          acc[48 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), fhi, acc[48 + i]);
-        }
-      }
-      if (!live) break;
-      const bool row_ok = r_in < t.rows;
-      if (EP == MOE_EP_F32) {
-        if (row_ok) {
-          float* dst = static_cast<float*>(args.D) + arow * N + t.n_idx * kBN + 128 * g;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            reinterpret_cast<float4*>(dst)[i] =
-                make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x, acc[2 * i + 1].y);
-        }
-      } else {
-        // h = SiLU(gate) * up for this thread's 64 channels, then the 1x128
-        // tile amax is shared with the partner thread of the other half.
-        // gate channels are acc[0..31] (packed pairs), the matching up channels acc[32..63]
-        float h[64];
-        float amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          h[2 * i] = silu_mul(acc[i].x, acc[32 + i].x);
-          h[2 * i + 1] = silu_mul(acc[i].y, acc[32 + i].y);
-          amax = fmaxf(amax, fmaxf(fabsf(h[2 * i]), fabsf(h[2 * i + 1])));
-        }
-        const int xb = xtile & 1;
-        amax_x[(xb * 2 + g) * 128 + r_in] = amax;
-        mbar_arrive(&xbar[xb]);
-        if (!__all_sync(0xffffffffu, mbar_wait(&xbar[xb], (xtile >> 1) & 1, abort_v, args.dev_err)))
-          break;
-        amax = fmaxf(amax_x[(xb * 2 + 0) * 128 + r_in], amax_x[(xb * 2 + 1) * 128 + r_in]);
-        ++xtile;
-        const float s = quant_scale(amax);
-        if (row_ok) {
-          const int I = N / 2;
-          uint8_t* dst = static_cast<uint8_t*>(args.D) + arow * I + t.n_idx * 128 + 64 * g;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 o;
-            o.x = e4m3x4(__fdiv_rn(h[16 * i + 0], s), __fdiv_rn(h[16 * i + 1], s),
-                         __fdiv_rn(h[16 * i + 2], s), __fdiv_rn(h[16 * i + 3], s));
-            o.y = e4m3x4(__fdiv_rn(h[16 * i + 4], s), __fdiv_rn(h[16 * i + 5], s),
-                         __fdiv_rn(h[16 * i + 6], s), __fdiv_rn(h[16 * i + 7], s));
-            o.z = e4m3x4(__fdiv_rn(h[16 * i + 8], s), __fdiv_rn(h[16 * i + 9], s),
-                         __fdiv_rn(h[16 * i + 10], s), __fdiv_rn(h[16 * i + 11], s));
-            o.w = e4m3x4(__fdiv_rn(h[16 * i + 12], s), __fdiv_rn(h[16 * i + 13], s),
-                         __fdiv_rn(h[16 * i + 14], s), __fdiv_rn(h[16 * i + 15], s));
-            reinterpret_cast<uint4*>(dst)[i] = o;
-          }
-          if (g == 0) args.d_scale[arow * (I / 128) + t.n_idx] = s;
-        }
-      }
+      if (!epilogue_tile<EP, false>(args, t, tmem, warp, lane, KB, N, tit, xtile, c.tfull,
+                                    c.tempty, c.xbar, c.amax_x, abort_v))
+        break;
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// =========================================================== 2-SM mainloop
+// Barrier protocol of a CTA pair:
+//   full[s]   (even CTA)  armed by the even CTA's producer for both CTAs'
+//                         bytes; both CTAs' TMA loads complete on it
+//   empty[s]  (each CTA)  the even CTA's MMA commit, multicast to both
+//   tfull[p]  (each CTA)  the even CTA's MMA commit, multicast to both
+//   tempty[p] (even CTA)  16 arrivals: 8 epilogue warps of each CTA
+template <int EP, int SK>
+__global__ void __launch_bounds__(kThreads, 1) gemm2sm_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const GemmArgs args) {
+  constexpr int kSub = kBK / SK;
+  constexpr int kHalf = 128 * SK;                 // one CTA's share of A or of B
+  constexpr int kStage = 2 * kHalf;
+  constexpr int kStages = kRingBytes / kStage;
+  static_assert((2 * kStages + 8) * 8 + 8 <= 512, "barrier area");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const Ctl c = carve<kStages>(base);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+  const int N = args.N, KB = args.K / kBK, nN = N / kBN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], 1);
+    }
+    for (int p = 0; p < 2; ++p) {
+      mbar_init(&c.tfull[p], 1);
+      mbar_init(&c.tempty[p], 2 * (kEpiThreads / 32));
+    }
+    mbar_init(c.done, 1);
+    mbar_init(&c.xbar[0], kEpiThreads);
+    mbar_init(&c.xbar[1], kEpiThreads);
+    *c.abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 2) build_tile_prefix<256>(args, c.rstart, lane);
+  if (warp == 1) {
+    tmem_alloc_pair(c.tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *c.tmem_slot;
+  volatile int* abort_v = c.abort_flag;
+  const int total = c.rstart[args.groups] * nN;
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------- TMA producer (each CTA)
+      int it = 0;
+      bool live = true;
+      for (int w = cluster; w < total && live; w += n_clusters) {
+        const Work t = decode_work<256>(w, nN, c.rstart, args, static_cast<int>(rank));
+        if (!t.ok) {
+          set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
+          continue;
+        }
+        const int brow = t.e * N + t.n_idx * kBN + 128 * static_cast<int>(rank);
+        for (int kk = 0; kk < KB * kSub; ++kk, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!mbar_wait(&c.empty[s], ph ^ 1, abort_v, args.dev_err)) {
+            live = false;
+            break;
+          }
+          uint8_t* sA = base + s * kStage;
+          if (rank == 0) mbar_arrive_expect_tx(&c.full[s], 2 * kStage);
+          tma_load_2d_pair(sA, &tmA, &c.full[s], kk * SK, t.row0);
+          tma_load_2d_pair(sA + kHalf, &tmB, &c.full[s], kk * SK, brow);
+        }
+      }
+      if (rank == 0) {
+        // every issued copy (of both CTAs) lands before either CTA can exit
+        const int first = it > kStages ? it - kStages : 0;
+        for (int i = first; i < it; ++i)
+          mbar_wait(&c.full[i % kStages], (i / kStages) & 1, nullptr, args.dev_err);
+      }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+      // ------------------------------------- MMA issuer (even CTA only)
+      const uint32_t idesc = instr_desc(kFmtE4M3, kFmtE4M3, 256, kBN);
+      int it = 0, tit = 0;
+      bool live = true;
+      for (int w = cluster; w < total && live; w += n_clusters) {
+        const Work t = decode_work<256>(w, nN, c.rstart, args, 0);
+        if (!t.ok) continue;
+        for (int kb = 0; kb < KB && live; ++kb, ++tit) {
+          const int p = tit & 1;
+          if (!mbar_wait(&c.tempty[p], ((tit >> 1) & 1) ^ 1, abort_v, args.dev_err)) {
+            live = false;
+            break;
+          }
+          const uint32_t dt = tmem + static_cast<uint32_t>(p * kBN);
+          for (int h = 0; h < kSub; ++h, ++it) {
+            const int s = it % kStages;
+            if (!mbar_wait(&c.full[s], (it / kStages) & 1, abort_v, args.dev_err)) {
+              live = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sA = smem_u32(base + s * kStage);
+            const uint64_t ad = kmajor_desc<SK>(sA);
+            const uint64_t bd = kmajor_desc<SK>(sA + kHalf);
+#pragma unroll
+            for (int k = 0; k < SK / 32; ++k)
+              mma_f8f6f4_pair(dt, ad + 2 * k, bd + 2 * k, idesc, (h > 0 || k > 0) ? 1u : 0u);
+            mma_commit_pair(&c.empty[s], 0x3);
+          }
+          if (live) mma_commit_pair(&c.tfull[p], 0x3);
+        }
+      }
+      mma_commit_pair(c.done, 0x1);
+      mbar_wait(c.done, 0, nullptr, args.dev_err);
+    }
+    __syncwarp();
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
+    int tit = 0, xtile = 0;
+    for (int w = cluster; w < total; w += n_clusters) {
+      const Work t = decode_work<256>(w, nN, c.rstart, args, static_cast<int>(rank));
+      if (!t.ok) continue;
+      if (!epilogue_tile<EP, true>(args, t, tmem, warp, lane, KB, N, tit, xtile, c.tfull,
+                                   c.tempty, c.xbar, c.amax_x, abort_v))
+        break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+}
+
+template <int EP>
+const void* kernel_ptr() {
+  if (MOE_GEMM_PAIR) return reinterpret_cast<const void*>(gemm2sm_kernel<EP, MOE_GEMM_SK>);
+  return reinterpret_cast<const void*>(gemm1sm_kernel<EP, MOE_GEMM_SK>);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -361,10 +612,15 @@ extern "C" moe_status grouped_gemm_fp8_blockscaled(
   if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return MOE_ERR_ALIGN;
   if (a_rows > 0x7FFFFFFF || static_cast<int64_t>(groups) * N > 0x7FFFFFFF)
     return MOE_ERR_UNSUPPORTED;
+  if (groups > kMaxGroups) return MOE_ERR_UNSUPPORTED;
+  constexpr int SK = MOE_GEMM_SK;
+  constexpr bool pair = MOE_GEMM_PAIR != 0;
+  // A: 128-row boxes; B: the 256 weight rows of a tile, or each CTA's 128
+  // of them in the pair form; boxes are SK bytes wide with an SK-byte swizzle
   CUtensorMap tmA, tmB;
-  if (!moe_make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, a_rows, K, kBK, kBM) ||
+  if (!moe_make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, a_rows, K, SK, kBM, SK) ||
       !moe_make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K,
-                        static_cast<uint64_t>(groups) * N, K, kBK, kBN))
+                        static_cast<uint64_t>(groups) * N, K, SK, pair ? 128 : kBN, SK))
     return MOE_ERR_CUDA;
   GemmArgs a;
   a.sa = sa;
@@ -382,23 +638,44 @@ extern "C" moe_status grouped_gemm_fp8_blockscaled(
   a.d_scale = d_scale;
   a.dev_err = dev_err;
   static int configured = 0;
+  static int max_ctas[2] = {0, 0};
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pair ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (!configured) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<MOE_EP_F32>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess ||
-        cudaFuncSetAttribute(grouped_gemm_kernel<MOE_EP_SWIGLU_QUANT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
-      return MOE_ERR_CUDA;
+    for (int i = 0; i < 2; ++i) {
+      const void* f = i == 0 ? kernel_ptr<MOE_EP_F32>() : kernel_ptr<MOE_EP_SWIGLU_QUANT>();
+      if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSmemBytes)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (pair) {
+        cfg.gridDim = dim3(2 * (moe_num_sms() / 2));
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, f, &cfg) != cudaSuccess) return MOE_ERR_CUDA;
+        max_ctas[i] = 2 * clusters;
+      } else {
+        max_ctas[i] = moe_num_sms();
+      }
+    }
     configured = 1;
   }
-  const int64_t work_max = static_cast<int64_t>(max_tiles) * (N / kBN);
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(moe_num_sms(), work_max)));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (ep == MOE_EP_F32)
-    grouped_gemm_kernel<MOE_EP_F32><<<grid, kThreads, kSmemBytes, st>>>(tmA, tmB, a);
-  else
-    grouped_gemm_kernel<MOE_EP_SWIGLU_QUANT><<<grid, kThreads, kSmemBytes, st>>>(tmA, tmB, a);
-  MOE_CUDA_CHECK_LAUNCH();
+  const int mc = max_ctas[ep == MOE_EP_F32 ? 0 : 1];
+  if (mc <= 0) return MOE_ERR_UNSUPPORTED;
+  // no more CTAs than work items (128-row tiles bound the work count)
+  const int64_t work_max = static_cast<int64_t>(max_tiles) * (N / kBN) * (pair ? 2 : 1);
+  int ctas = static_cast<int>(std::max<int64_t>(pair ? 2 : 1, std::min<int64_t>(mc, work_max)));
+  if (pair) ctas &= ~1;
+  cfg.gridDim = dim3(ctas);
+  const void* fn = ep == MOE_EP_F32 ? kernel_ptr<MOE_EP_F32>() : kernel_ptr<MOE_EP_SWIGLU_QUANT>();
+  void* kargs[3] = {&tmA, &tmB, &a};
+  if (cudaLaunchKernelExC(&cfg, fn, kargs) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
