@@ -64,7 +64,13 @@ V4_PRO = MoEConfig("v4_pro", T=16384, d=7168, E=384, G=1, M=1, K=6, I=3072,
 V3_PREFILL_E32 = MoEConfig("v3_prefill_e32", T=512, d=7168, E=32, G=8, M=4, K=8, I=2048,
                            bias_lo=-0.05, bias_hi=0.05)
 
-PRESETS = {c.name: c for c in (TINY, V3_PREFILL, V3_DECODE, V4_PRO, V3_PREFILL_E32)}
+# Profiling case for the token-sized kernels (route, quantisation,
+# permutation, combine): V3 prefill's T, d and top-8, but 32 experts, so the
+# weights take ~1.5 GB and multi-pass captures stay small.
+V3_TOKENS_E32 = MoEConfig("v3_tokens_e32", T=4096, d=7168, E=32, G=8, M=4, K=8, I=2048,
+                          bias_lo=-0.05, bias_hi=0.05)
+
+PRESETS = {c.name: c for c in (TINY, V3_PREFILL, V3_DECODE, V4_PRO, V3_PREFILL_E32, V3_TOKENS_E32)}
 
 
 @dataclass(frozen=True)

@@ -25,15 +25,10 @@
 // 64-byte ones halve the contiguous bytes each weight row contributes to a
 // TMA box), so 128 is the default.
 //
-// Two forms of the mainloop share the epilogue:
-//   gemm1sm  -- one CTA computes a 128 x 256 tile (tcgen05 cta_group::1);
-//   gemm2sm  -- a CTA pair (cluster of 2) computes a 256 x 256 tile with
-//               tcgen05.mma.cta_group::2: each CTA stages its 128 rows of A
-//               and 128 of the 256 weight rows, a weight tile is streamed
-//               once per pair, and each CTA's TMEM holds its rows' partial.
-//               It does more padded work when experts hold ~128 rows (V3
-//               prefill), where the 1-SM form is faster; it is kept for
-//               segments of 256+ rows.
+// One CTA computes a 128 x 256 tile (tcgen05 cta_group::1).  A CTA-pair form
+// (cta_group::2, 256 x 256 tiles, each CTA staging half of A and of the
+// weight tile) was measured slower on every workload here: its cross-CTA
+// handshakes cost more than the halved shared-memory ingress saves.
 //
 // Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
 // TMEM owner, warp 2 builds the work list then idles with warp 3 (the first
@@ -47,10 +42,7 @@
 #include "epi_math.cuh"
 #include "moe_common.cuh"
 
-// Mainloop form and stage width (build-time choices).
-#ifndef MOE_GEMM_PAIR
-#define MOE_GEMM_PAIR 0
-#endif
+// Stage width (build-time choice).
 #ifndef MOE_GEMM_SK
 #define MOE_GEMM_SK 128
 #endif
@@ -85,7 +77,7 @@ struct GemmArgs {
 };
 
 struct Work {
-  int e, n_idx, row0, rows;  // row0 / rows: the rows this CTA owns
+  int e, n_idx, row0, rows;  // expert, n-tile, first row and valid rows of the m-tile
   bool ok;
 };
 
@@ -124,10 +116,8 @@ __device__ void build_tile_prefix(const GemmArgs& a, int* rstart, int lane) {
 
 // Work item w -> (expert, n-tile, RT-row tile); the items of expert e occupy
 // [nN*rstart[e], nN*rstart[e+1]) and the row tile varies fastest inside.
-// `sub` selects this CTA's 128-row half of a 256-row pair tile.
 template <int RT>
-__device__ __forceinline__ Work decode_work(int w, int nN, const int* rstart, const GemmArgs& a,
-                                            int sub) {
+__device__ __forceinline__ Work decode_work(int w, int nN, const int* rstart, const GemmArgs& a) {
   Work t{0, 0, 0, 0, false};
   const int j = w / nN;
   int lo = 0, hi = a.groups - 1;
@@ -145,8 +135,8 @@ __device__ __forceinline__ Work decode_work(int w, int nN, const int* rstart, co
   const int seg0 = __ldg(a.offsets + e), seg1 = __ldg(a.offsets + e + 1);
   const int tile0 = seg0 + RT * mt;
   if (tile0 >= seg1 || seg1 > a.a_rows || t.n_idx >= nN) return t;
-  t.row0 = tile0 + 128 * sub;
-  t.rows = max(0, min(128, seg1 - t.row0));
+  t.row0 = tile0;
+  t.rows = min(RT, seg1 - tile0);
   t.e = e;
   t.ok = true;
   return t;
@@ -154,9 +144,8 @@ __device__ __forceinline__ Work decode_work(int w, int nN, const int* rstart, co
 
 // ------------------------------------------------------------------ epilogue
 // Promotes every K block of one tile into fp32 registers and writes the
-// tile.  Returns false if a bounded wait gave up.  PAIR: the TMEM buffer is
-// released on the even CTA's barrier.
-template <int EP, bool PAIR>
+// tile.  Returns false if a bounded wait gave up.
+template <int EP>
 __device__ __forceinline__ bool epilogue_tile(const GemmArgs& args, const Work& t, uint32_t tmem,
                                               int warp, int lane, int KB, int N, int& tit,
                                               int& xtile, uint64_t* tfull, uint64_t* tempty,
@@ -222,10 +211,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs& args, const Work& 
     tmem_ld_wait();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) {
-      if (PAIR) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[p]), 0));
-      else mbar_arrive(&tempty[p]);
-    }
+    if (lane == 0) mbar_arrive(&tempty[p]);
     const float2 fhi = make_float2(f_hi, f_hi);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -367,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
       int it = 0;
       bool live = true;
       for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
-        const Work t = decode_work<128>(w, nN, c.rstart, args, 0);
+        const Work t = decode_work<128>(w, nN, c.rstart, args);
         if (!t.ok) {
           set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
           continue;
@@ -396,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
       int it = 0, tit = 0;
       bool live = true;
       for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
-        const Work t = decode_work<128>(w, nN, c.rstart, args, 0);
+        const Work t = decode_work<128>(w, nN, c.rstart, args);
         if (!t.ok) continue;
         for (int kb = 0; kb < KB && live; ++kb, ++tit) {
           const int p = tit & 1;
@@ -431,9 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
     int tit = 0, xtile = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
-      const Work t = decode_work<128>(w, nN, c.rstart, args, 0);
+      const Work t = decode_work<128>(w, nN, c.rstart, args);
       if (!t.ok) continue;
-      if (!epilogue_tile<EP, false>(args, t, tmem, warp, lane, KB, N, tit, xtile, c.tfull,
+      if (!epilogue_tile<EP>(args, t, tmem, warp, lane, KB, N, tit, xtile, c.tfull,
                                     c.tempty, c.xbar, c.amax_x, abort_v))
         break;
     }
@@ -443,151 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-// =========================================================== 2-SM mainloop
-// Barrier protocol of a CTA pair:
-//   full[s]   (even CTA)  armed by the even CTA's producer for both CTAs'
-//                         bytes; both CTAs' TMA loads complete on it
-//   empty[s]  (each CTA)  the even CTA's MMA commit, multicast to both
-//   tfull[p]  (each CTA)  the even CTA's MMA commit, multicast to both
-//   tempty[p] (even CTA)  16 arrivals: 8 epilogue warps of each CTA
-template <int EP, int SK>
-__global__ void __launch_bounds__(kThreads, 1) gemm2sm_kernel(
-    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-    const GemmArgs args) {
-  constexpr int kSub = kBK / SK;
-  constexpr int kHalf = 128 * SK;                 // one CTA's share of A or of B
-  constexpr int kStage = 2 * kHalf;
-  constexpr int kStages = kRingBytes / kStage;
-  static_assert((2 * kStages + 8) * 8 + 8 <= 512, "barrier area");
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  const Ctl c = carve<kStages>(base);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
-  const int N = args.N, KB = args.K / kBK, nN = N / kBN;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&c.full[s], 1);
-      mbar_init(&c.empty[s], 1);
-    }
-    for (int p = 0; p < 2; ++p) {
-      mbar_init(&c.tfull[p], 1);
-      mbar_init(&c.tempty[p], 2 * (kEpiThreads / 32));
-    }
-    mbar_init(c.done, 1);
-    mbar_init(&c.xbar[0], kEpiThreads);
-    mbar_init(&c.xbar[1], kEpiThreads);
-    *c.abort_flag = 0;
-    fence_barrier_init();
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-  }
-  if (warp == 2) build_tile_prefix<256>(args, c.rstart, lane);
-  if (warp == 1) {
-    tmem_alloc_pair(c.tmem_slot, kTmemCols);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();
-  tc_fence_after();
-  const uint32_t tmem = *c.tmem_slot;
-  volatile int* abort_v = c.abort_flag;
-  const int total = c.rstart[args.groups] * nN;
-
-  if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
-    if (warp == 0 && lane == 0) {
-      // ------------------------------------------- TMA producer (each CTA)
-      int it = 0;
-      bool live = true;
-      for (int w = cluster; w < total && live; w += n_clusters) {
-        const Work t = decode_work<256>(w, nN, c.rstart, args, static_cast<int>(rank));
-        if (!t.ok) {
-          set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
-          continue;
-        }
-        const int brow = t.e * N + t.n_idx * kBN + 128 * static_cast<int>(rank);
-        for (int kk = 0; kk < KB * kSub; ++kk, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!mbar_wait(&c.empty[s], ph ^ 1, abort_v, args.dev_err)) {
-            live = false;
-            break;
-          }
-          uint8_t* sA = base + s * kStage;
-          if (rank == 0) mbar_arrive_expect_tx(&c.full[s], 2 * kStage);
-          tma_load_2d_pair(sA, &tmA, &c.full[s], kk * SK, t.row0);
-          tma_load_2d_pair(sA + kHalf, &tmB, &c.full[s], kk * SK, brow);
-        }
-      }
-      if (rank == 0) {
-        // every issued copy (of both CTAs) lands before either CTA can exit
-        const int first = it > kStages ? it - kStages : 0;
-        for (int i = first; i < it; ++i)
-          mbar_wait(&c.full[i % kStages], (i / kStages) & 1, nullptr, args.dev_err);
-      }
-    } else if (warp == 1 && lane == 0 && rank == 0) {
-      // ------------------------------------- MMA issuer (even CTA only)
-      const uint32_t idesc = instr_desc(kFmtE4M3, kFmtE4M3, 256, kBN);
-      int it = 0, tit = 0;
-      bool live = true;
-      for (int w = cluster; w < total && live; w += n_clusters) {
-        const Work t = decode_work<256>(w, nN, c.rstart, args, 0);
-        if (!t.ok) continue;
-        for (int kb = 0; kb < KB && live; ++kb, ++tit) {
-          const int p = tit & 1;
-          if (!mbar_wait(&c.tempty[p], ((tit >> 1) & 1) ^ 1, abort_v, args.dev_err)) {
-            live = false;
-            break;
-          }
-          const uint32_t dt = tmem + static_cast<uint32_t>(p * kBN);
-          for (int h = 0; h < kSub; ++h, ++it) {
-            const int s = it % kStages;
-            if (!mbar_wait(&c.full[s], (it / kStages) & 1, abort_v, args.dev_err)) {
-              live = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t sA = smem_u32(base + s * kStage);
-            const uint64_t ad = kmajor_desc<SK>(sA);
-            const uint64_t bd = kmajor_desc<SK>(sA + kHalf);
-#pragma unroll
-            for (int k = 0; k < SK / 32; ++k)
-              mma_f8f6f4_pair(dt, ad + 2 * k, bd + 2 * k, idesc, (h > 0 || k > 0) ? 1u : 0u);
-            mma_commit_pair(&c.empty[s], 0x3);
-          }
-          if (live) mma_commit_pair(&c.tfull[p], 0x3);
-        }
-      }
-      mma_commit_pair(c.done, 0x1);
-      mbar_wait(c.done, 0, nullptr, args.dev_err);
-    }
-    __syncwarp();
-  } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
-    int tit = 0, xtile = 0;
-    for (int w = cluster; w < total; w += n_clusters) {
-      const Work t = decode_work<256>(w, nN, c.rstart, args, static_cast<int>(rank));
-      if (!t.ok) continue;
-      if (!epilogue_tile<EP, true>(args, t, tmem, warp, lane, KB, N, tit, xtile, c.tfull,
-                                   c.tempty, c.xbar, c.amax_x, abort_v))
-        break;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
-}
-
 template <int EP>
 const void* kernel_ptr() {
-  if (MOE_GEMM_PAIR) return reinterpret_cast<const void*>(gemm2sm_kernel<EP, MOE_GEMM_SK>);
   return reinterpret_cast<const void*>(gemm1sm_kernel<EP, MOE_GEMM_SK>);
 }
 
@@ -614,13 +457,12 @@ extern "C" moe_status grouped_gemm_fp8_blockscaled(
     return MOE_ERR_UNSUPPORTED;
   if (groups > kMaxGroups) return MOE_ERR_UNSUPPORTED;
   constexpr int SK = MOE_GEMM_SK;
-  constexpr bool pair = MOE_GEMM_PAIR != 0;
-  // A: 128-row boxes; B: the 256 weight rows of a tile, or each CTA's 128
-  // of them in the pair form; boxes are SK bytes wide with an SK-byte swizzle
+  // A: 128-row boxes; B: the 256 weight rows of a tile; boxes are SK bytes
+  // wide with an SK-byte swizzle
   CUtensorMap tmA, tmB;
   if (!moe_make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, a_rows, K, SK, kBM, SK) ||
       !moe_make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K,
-                        static_cast<uint64_t>(groups) * N, K, SK, pair ? 128 : kBN, SK))
+                        static_cast<uint64_t>(groups) * N, K, SK, kBN, SK))
     return MOE_ERR_CUDA;
   GemmArgs a;
   a.sa = sa;
@@ -638,44 +480,22 @@ extern "C" moe_status grouped_gemm_fp8_blockscaled(
   a.d_scale = d_scale;
   a.dev_err = dev_err;
   static int configured = 0;
-  static int max_ctas[2] = {0, 0};
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = pair ? 2 : 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   if (!configured) {
     for (int i = 0; i < 2; ++i) {
       const void* f = i == 0 ? kernel_ptr<MOE_EP_F32>() : kernel_ptr<MOE_EP_SWIGLU_QUANT>();
       if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kSmemBytes)) != cudaSuccess)
         return MOE_ERR_CUDA;
-      if (pair) {
-        cfg.gridDim = dim3(2 * (moe_num_sms() / 2));
-        int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, f, &cfg) != cudaSuccess) return MOE_ERR_CUDA;
-        max_ctas[i] = 2 * clusters;
-      } else {
-        max_ctas[i] = moe_num_sms();
-      }
     }
     configured = 1;
   }
-  const int mc = max_ctas[ep == MOE_EP_F32 ? 0 : 1];
-  if (mc <= 0) return MOE_ERR_UNSUPPORTED;
-  // no more CTAs than work items (128-row tiles bound the work count)
-  const int64_t work_max = static_cast<int64_t>(max_tiles) * (N / kBN) * (pair ? 2 : 1);
-  int ctas = static_cast<int>(std::max<int64_t>(pair ? 2 : 1, std::min<int64_t>(mc, work_max)));
-  if (pair) ctas &= ~1;
-  cfg.gridDim = dim3(ctas);
+  // persistent: one CTA per SM, no more CTAs than work items
+  const int64_t work_max = static_cast<int64_t>(max_tiles) * (N / kBN);
+  const int ctas = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(moe_num_sms(), work_max)));
   const void* fn = ep == MOE_EP_F32 ? kernel_ptr<MOE_EP_F32>() : kernel_ptr<MOE_EP_SWIGLU_QUANT>();
   void* kargs[3] = {&tmA, &tmB, &a};
-  if (cudaLaunchKernelExC(&cfg, fn, kargs) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaLaunchKernel(fn, dim3(ctas), dim3(kThreads), kargs, kSmemBytes,
+                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
