@@ -18,6 +18,19 @@ __device__ __forceinline__ float quant_scale(float amax) {
   return __fdiv_rn(fmaxf(amax, kQuantEps), kE4M3Max);
 }
 
+// x / s rounded to nearest even, given r = RN(1/s): Markstein's correction
+// step (P. W. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): y = RN(x r),
+// e = x - s y (exact by FMA), q = RN(y + e r).  A zero residual returns y
+// itself, which keeps the sign of a zero quotient.  Used only where x is a
+// bf16 value and s a quantisation scale from a bf16 tile maximum; the tests
+// check it against IEEE division on every such (x, s) pair.
+__device__ __forceinline__ float div_by_scale(float x, float s, float r) {
+  const float y = __fmul_rn(x, r);
+  const float e = __fmaf_rn(-y, s, x);
+  return e == 0.0f ? y : __fmaf_rn(e, r, y);
+}
+
 // Two fp32 values -> two E4M3 bytes (lo in the low byte), round to nearest
 // even, saturating to +-448 (hardware cvt.rn.satfinite.e4m3x2).
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {

@@ -5,7 +5,10 @@
 //
 // All three are HBM-bound streaming kernels: 16-byte vector loads, the amax
 // reduced with warp shuffles, the scale divided out in fp32 and the cast done
-// by the hardware's saturating round-to-nearest-even E4M3 conversion.
+// by the hardware's saturating round-to-nearest-even E4M3 conversion.  For
+// bf16 inputs the division is one correctly rounded reciprocal per tile plus
+// a per-element FMA correction (div_by_scale), which gives the IEEE quotient
+// on every input these kernels can see.
 #include "epi_math.cuh"
 #include "moe_common.cuh"
 
@@ -58,9 +61,12 @@ __global__ void __launch_bounds__(kQ1Threads) quant_1x128_kernel(
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     if (t < total) {
       const float s = quant_scale(amax);
+      const float rs = __frcp_rn(s);
       uint2 out;
-      out.x = e4m3x4(__fdiv_rn(f[0], s), __fdiv_rn(f[1], s), __fdiv_rn(f[2], s), __fdiv_rn(f[3], s));
-      out.y = e4m3x4(__fdiv_rn(f[4], s), __fdiv_rn(f[5], s), __fdiv_rn(f[6], s), __fdiv_rn(f[7], s));
+      out.x = e4m3x4(div_by_scale(f[0], s, rs), div_by_scale(f[1], s, rs),
+                     div_by_scale(f[2], s, rs), div_by_scale(f[3], s, rs));
+      out.y = e4m3x4(div_by_scale(f[4], s, rs), div_by_scale(f[5], s, rs),
+                     div_by_scale(f[6], s, rs), div_by_scale(f[7], s, rs));
       const int64_t r = t / tiles_per_row;
       const int j = static_cast<int>(t - r * tiles_per_row);
       *reinterpret_cast<uint2*>(q + r * cols + j * 128 + lane16 * 8) = out;
@@ -104,6 +110,7 @@ __global__ void __launch_bounds__(kQ2Threads) quant_128x128_kernel(
 #pragma unroll
   for (int k = 1; k < kQ2Threads / 32; ++k) amax = fmaxf(amax, red[k]);
   const float s = quant_scale(amax);
+  const float rs = __frcp_rn(s);
   if (tid == 0) scale[static_cast<int64_t>(bi) * (cols / 128) + bj] = s;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -115,8 +122,8 @@ __global__ void __launch_bounds__(kQ2Threads) quant_128x128_kernel(
     float f[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      f[2 * k] = __fdiv_rn(bf16_bits_to_float(ww[k] & 0xFFFFu), s);
-      f[2 * k + 1] = __fdiv_rn(bf16_bits_to_float(ww[k] >> 16), s);
+      f[2 * k] = div_by_scale(bf16_bits_to_float(ww[k] & 0xFFFFu), s, rs);
+      f[2 * k + 1] = div_by_scale(bf16_bits_to_float(ww[k] >> 16), s, rs);
     }
     uint2 out;
     out.x = e4m3x4(f[0], f[1], f[2], f[3]);
