@@ -22,9 +22,11 @@ __device__ __forceinline__ float quant_scale(float amax) {
 // step (P. W. Markstein, "Computation of elementary functions on the IBM
 // RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): y = RN(x r),
 // e = x - s y (exact by FMA), q = RN(y + e r).  A zero residual returns y
-// itself, which keeps the sign of a zero quotient.  Used only where x is a
-// bf16 value and s a quantisation scale from a bf16 tile maximum; the tests
-// check it against IEEE division on every such (x, s) pair.
+// itself, which keeps the sign of a zero quotient.  For a bf16 x and a scale
+// s from a bf16 tile maximum (the activation and weight quantisers) the tests
+// check it against IEEE division on every such (x, s) pair; the SwiGLU
+// requantisation applies it to fp32 h, where the tests bound the E4M3 bytes
+// against the fp64 reference.
 __device__ __forceinline__ float div_by_scale(float x, float s, float r) {
   const float y = __fmul_rn(x, r);
   const float e = __fmaf_rn(-y, s, x);
@@ -42,10 +44,13 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return static_cast<uint32_t>(e4m3x2(a, b)) | (static_cast<uint32_t>(e4m3x2(c, d)) << 16);
 }
 
-// SiLU(g) * u with Swish beta = 1.
+// SiLU(g) * u with Swish beta = 1, g / (1 + e^-g) evaluated with the
+// hardware exponential and reciprocal approximations (a few fp32 ulps; the
+// result is quantised to E4M3, whose step is 2^20 fp32 ulps).  For g < -87,
+// e^-g overflows and the quotient is a signed zero.
 __device__ __forceinline__ float silu_mul(float g, float u) {
-  const float den = __fadd_rn(1.0f, expf(-g));
-  return __fmul_rn(__fdiv_rn(g, den), u);
+  const float den = __fadd_rn(1.0f, __expf(-g));
+  return __fmul_rn(__fdividef(g, den), u);
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {

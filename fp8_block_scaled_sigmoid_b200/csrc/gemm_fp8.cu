@@ -269,22 +269,19 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs& args, const Work& 
     amax = fmaxf(amax_x[(xb * 2 + 0) * 128 + r_in], amax_x[(xb * 2 + 1) * 128 + r_in]);
     ++xtile;
     const float sq = quant_scale(amax);
+    const float rq = __frcp_rn(sq);
     if (row_ok) {
       const int I = N / 2;
       uint8_t* dst = static_cast<uint8_t*>(args.D) + arow * I + t.n_idx * 128 + 64 * g;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2* hp = acc + 8 * i;  // h[16i .. 16i+15]
-        uint4 o;
-        o.x = e4m3x4(__fdiv_rn(hp[0].x, sq), __fdiv_rn(hp[0].y, sq), __fdiv_rn(hp[1].x, sq),
-                     __fdiv_rn(hp[1].y, sq));
-        o.y = e4m3x4(__fdiv_rn(hp[2].x, sq), __fdiv_rn(hp[2].y, sq), __fdiv_rn(hp[3].x, sq),
-                     __fdiv_rn(hp[3].y, sq));
-        o.z = e4m3x4(__fdiv_rn(hp[4].x, sq), __fdiv_rn(hp[4].y, sq), __fdiv_rn(hp[5].x, sq),
-                     __fdiv_rn(hp[5].y, sq));
-        o.w = e4m3x4(__fdiv_rn(hp[6].x, sq), __fdiv_rn(hp[6].y, sq), __fdiv_rn(hp[7].x, sq),
-                     __fdiv_rn(hp[7].y, sq));
-        reinterpret_cast<uint4*>(dst)[i] = o;
+        uint32_t w4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          w4[j] = e4m3x4(div_by_scale(hp[2 * j].x, sq, rq), div_by_scale(hp[2 * j].y, sq, rq),
+                         div_by_scale(hp[2 * j + 1].x, sq, rq), div_by_scale(hp[2 * j + 1].y, sq, rq));
+        reinterpret_cast<uint4*>(dst)[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
       if (g == 0) args.d_scale[arow * (I / 128) + t.n_idx] = sq;
     }

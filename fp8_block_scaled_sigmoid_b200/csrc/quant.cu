@@ -153,8 +153,9 @@ __global__ void __launch_bounds__(kSwThreads) swiglu_quant_kernel(
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   const float s = quant_scale(amax);
-  const uint32_t packed = e4m3x4(__fdiv_rn(hv[0], s), __fdiv_rn(hv[1], s), __fdiv_rn(hv[2], s),
-                                 __fdiv_rn(hv[3], s));
+  const float rs = __frcp_rn(s);
+  const uint32_t packed = e4m3x4(div_by_scale(hv[0], s, rs), div_by_scale(hv[1], s, rs),
+                                 div_by_scale(hv[2], s, rs), div_by_scale(hv[3], s, rs));
   *reinterpret_cast<uint32_t*>(h + r * I + j * 128 + lane * 4) = packed;
   if (lane == 0) h_scale[tile] = s;
 }
