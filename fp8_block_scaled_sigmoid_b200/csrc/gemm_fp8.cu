@@ -221,34 +221,47 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs& args, const Work& 
   }
   const bool row_ok = r_in < t.rows;
   if (EP == MOE_EP_F32) {
-    // Each lane holds one row.  Lanes 2j and 2j+1 swap half of every
-    // 8-column group so that one store instruction writes 32 contiguous bytes
-    // of row 2j (even lane: columns 8i..8i+3, odd lane: 8i+4..8i+7) and the
-    // next the same of row 2j+1: every 32-byte sector is written whole.
-    const bool odd = lane & 1;
-    const int64_t row_e = static_cast<int64_t>(t.row0) + (r_in & ~1);
-    const bool ok_e = (r_in & ~1) < t.rows, ok_o = (r_in | 1) < t.rows;
-    float* base_e = static_cast<float*>(args.D) + row_e * N + t.n_idx * kBN + 128 * g;
-    float* base_o = base_e + N;
+    // Each lane holds one row (128 columns).  Per 32-column chunk, the 8
+    // lanes of each group (rows rb..rb+7) transpose their 8 x 8 block of
+    // float4 with three xor-butterfly exchange rounds: afterwards lane rb+i
+    // holds columns 4i..4i+3 of every row of the group, so one store
+    // instruction writes 4 rows x 128 contiguous bytes (whole lines).
+    const int li = lane & 7;
+    const int rb = r_in - li;  // first row of this lane's group inside the tile
+    float* base = static_cast<float*>(args.D) + (static_cast<int64_t>(t.row0) + rb) * N +
+                  t.n_idx * kBN + 128 * g + 4 * li;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      // this lane's columns 8i..8i+3 are acc[4i], acc[4i+1]; 8i+4..8i+7 are acc[4i+2], acc[4i+3]
-      const float2 lo0 = acc[4 * i], lo1 = acc[4 * i + 1], hi0 = acc[4 * i + 2], hi1 = acc[4 * i + 3];
-      const float2 send0 = odd ? lo0 : hi0, send1 = odd ? lo1 : hi1;
-      float2 recv0, recv1;
-      recv0.x = __shfl_xor_sync(0xffffffffu, send0.x, 1);
-      recv0.y = __shfl_xor_sync(0xffffffffu, send0.y, 1);
-      recv1.x = __shfl_xor_sync(0xffffffffu, send1.x, 1);
-      recv1.y = __shfl_xor_sync(0xffffffffu, send1.y, 1);
-      // row 2j: even lane its own low half, odd lane the even lane's high half
-      const float4 wa = odd ? make_float4(recv0.x, recv0.y, recv1.x, recv1.y)
-                            : make_float4(lo0.x, lo0.y, lo1.x, lo1.y);
-      // row 2j+1: even lane the odd lane's low half, odd lane its own high half
-      const float4 wb = odd ? make_float4(hi0.x, hi0.y, hi1.x, hi1.y)
-                            : make_float4(recv0.x, recv0.y, recv1.x, recv1.y);
-      const int col = 8 * i + (odd ? 4 : 0);
-      if (ok_e) *reinterpret_cast<float4*>(base_e + col) = wa;
-      if (ok_o) *reinterpret_cast<float4*>(base_o + col) = wb;
+    for (int b = 0; b < 4; ++b) {
+      float4 e[8];  // e[j] = columns 32b + 4j .. 32b + 4j + 3 of this lane's row
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float2 x0 = acc[16 * b + 2 * j], x1 = acc[16 * b + 2 * j + 1];
+        e[j] = make_float4(x0.x, x0.y, x1.x, x1.y);
+      }
+      // round s: for each pair (j0, j0 | s), a lane with bit s set sends e[j0]
+      // and receives its partner's e[j0 | s] into e[j0]; the other sends
+      // e[j0 | s] and receives into it
+#pragma unroll
+      for (int sft = 1; sft < 8; sft <<= 1) {
+        const bool hi = (lane & sft) != 0;
+#pragma unroll
+        for (int j0 = 0; j0 < 8; ++j0) {
+          if (j0 & sft) continue;
+          const int j1 = j0 | sft;
+          const float4 x = hi ? e[j0] : e[j1];
+          float4 y;
+          y.x = __shfl_xor_sync(0xffffffffu, x.x, sft);
+          y.y = __shfl_xor_sync(0xffffffffu, x.y, sft);
+          y.z = __shfl_xor_sync(0xffffffffu, x.z, sft);
+          y.w = __shfl_xor_sync(0xffffffffu, x.w, sft);
+          if (hi) e[j0] = y;
+          else e[j1] = y;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (rb + j < t.rows)
+          *reinterpret_cast<float4*>(base + static_cast<int64_t>(j) * N + 32 * b) = e[j];
     }
   } else {
     // h = SiLU(gate) * up overwrites the gate accumulators: h[2i], h[2i+1]
