@@ -14,8 +14,8 @@ with an NCCL all-reduce before the bias update (weak scaling).
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; between steps a 512 MB buffer is overwritten to
 flush the 126 MB L2 (outside the events).  The reported time is the max over
-ranks of the summed step times.  Clocks are sampled with nvidia-smi during
-the timed region.
+ranks of the summed step times.  Clocks are polled through NVML every 2 ms
+during the timed region.
 
 ``--impl reference`` times the CPU oracle instead (rank 0 only) on a bounded
 sample of the same workload and prints the same JSON line with
@@ -59,16 +59,58 @@ def workload_name(cfg) -> str:
 
 # --------------------------------------------------------------- clocks ---
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU, polled every 2 ms
+    through NVML from a thread while the timed region runs (a 3.5 ms step
+    needs a period far below nvidia-smi's).  The device is matched by PCI
+    bus id, so CUDA_VISIBLE_DEVICES remapping does not pick another GPU.
+    Falls back to ``nvidia-smi -lms 200`` when NVML is unavailable."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
         self.path = None
+        self.nvml = None
+        self.thread = None
+        self.samples = []
+        self.stop_flag = False
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        bus = getattr(torch.cuda.get_device_properties(self.idx), "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(torch.cuda.get_device_properties(self.idx), "pci_domain_id", 0)
+            dev = getattr(torch.cuda.get_device_properties(self.idx), "pci_device_id", 0)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{dev:02x}.0")
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+
+    def _poll(self, pynvml, h):
+        while not self.stop_flag:
+            try:
+                self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                     pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                     pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception:  # noqa: BLE001 - a failed read drops one sample
+                pass
+            time.sleep(0.002)
 
     def start(self):
+        import threading
+        try:
+            pynvml, h = self._nvml_handle()
+            self.nvml = pynvml
+            self.thread = threading.Thread(target=self._poll, args=(pynvml, h), daemon=True)
+            self.thread.start()
+            return
+        except Exception:  # noqa: BLE001 - no NVML: use nvidia-smi
+            self.nvml = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -80,6 +122,20 @@ class ClockSampler:
             self.proc = None
 
     def stop(self) -> dict:
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join()
+            if not self.samples:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"],
+                        "source": "nvml"}
+            reasons = set()
+            for _, _, bits in self.samples:
+                for b, n in self.REASONS.items():
+                    if bits & b:
+                        reasons.add(n)
+            return {"sm_mhz": statistics.median(x[0] for x in self.samples),
+                    "sm_max_mhz": max(x[1] for x in self.samples), "reasons": sorted(reasons),
+                    "samples": len(self.samples), "source": "nvml, 2 ms"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.25)
@@ -105,7 +161,7 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 200 ms"}
 
 
 # ------------------------------------------------------- CPU oracle leg ---
@@ -207,7 +263,8 @@ def run_gpu(args):
     sampler = ClockSampler(local) if rank == 0 else None
     if sampler:
         sampler.start()
-        time.sleep(0.3)
+        if sampler.proc is not None:
+            time.sleep(0.3)  # nvidia-smi needs a moment before its first sample
     barrier()
     lc0 = _abi.launch_count
     for i in range(args.steps):
@@ -434,7 +491,8 @@ def run_gemm(args):
     torch.cuda.synchronize()
     sampler = ClockSampler(0)
     sampler.start()
-    time.sleep(0.3)
+    if sampler.proc is not None:
+        time.sleep(0.3)
     times = []
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
