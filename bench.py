@@ -79,6 +79,8 @@ class ClockSampler:
         self.thread = None
         self.samples = []
         self.stop_flag = False
+        self.win = None
+        self.max_mhz = None
 
     def _nvml_handle(self):
         import pynvml
@@ -92,14 +94,22 @@ class ClockSampler:
         return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.idx)
 
     def _poll(self, pynvml, h):
+        try:
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001
+            self.max_mhz = None
         while not self.stop_flag:
             try:
-                self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
-                                     pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM),
+                self.samples.append((time.perf_counter(),
+                                     pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
                                      pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
             except Exception:  # noqa: BLE001 - a failed read drops one sample
                 pass
             time.sleep(0.002)
+
+    def window(self, t0: float, t1: float):
+        """Keep only samples taken between t0 and t1 (time.perf_counter)."""
+        self.win = (t0, t1)
 
     def start(self):
         import threading
@@ -125,17 +135,20 @@ class ClockSampler:
         if self.thread is not None:
             self.stop_flag = True
             self.thread.join()
-            if not self.samples:
-                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"],
-                        "source": "nvml"}
+            smp = self.samples
+            if self.win is not None:
+                smp = [x for x in smp if self.win[0] <= x[0] <= self.win[1]]
+            if not smp:
+                return {"sm_mhz": None, "sm_max_mhz": self.max_mhz,
+                        "reasons": ["no samples in the timed region"], "source": "nvml"}
             reasons = set()
-            for _, _, bits in self.samples:
+            for _, _, bits in smp:
                 for b, n in self.REASONS.items():
                     if bits & b:
                         reasons.add(n)
-            return {"sm_mhz": statistics.median(x[0] for x in self.samples),
-                    "sm_max_mhz": max(x[1] for x in self.samples), "reasons": sorted(reasons),
-                    "samples": len(self.samples), "source": "nvml, 2 ms"}
+            return {"sm_mhz": statistics.median(x[1] for x in smp), "sm_max_mhz": self.max_mhz,
+                    "reasons": sorted(reasons), "samples": len(smp),
+                    "source": "nvml, polled every 2 ms, samples inside the timed region"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.25)
@@ -266,6 +279,7 @@ def run_gpu(args):
         if sampler.proc is not None:
             time.sleep(0.3)  # nvidia-smi needs a moment before its first sample
     barrier()
+    t_lo = time.perf_counter()
     lc0 = _abi.launch_count
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
@@ -286,7 +300,10 @@ def run_gpu(args):
         layer.step_bias_update()
         e[7].record(st)
     barrier()
+    t_hi = time.perf_counter()
     launches = _abi.launch_count - lc0
+    if sampler:
+        sampler.window(t_lo, t_hi)
     clocks = sampler.stop() if sampler else None
     layer.check()
     step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]

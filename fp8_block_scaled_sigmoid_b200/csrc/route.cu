@@ -36,7 +36,9 @@ RouterTiling router_tiling(int T, int d, int E) {
   r.BN = ((E + r.n_tiles - 1) / r.n_tiles + 15) / 16 * 16;
   r.KB = d / kRtBK;
   const int tiles = std::max(1, r.m_tiles * r.n_tiles);
-  int splits = (moe_num_sms() + tiles - 1) / tiles;
+  // as many K splits as keep every CTA in one wave (a second, partial wave
+  // would double the time)
+  int splits = std::max(1, moe_num_sms() / tiles);
   splits = std::max(1, std::min(std::min(splits, 16), r.KB));
   r.kb_per_split = (r.KB + splits - 1) / splits;
   r.splits = (r.KB + r.kb_per_split - 1) / r.kb_per_split;  // no empty split
@@ -186,19 +188,47 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
   if (t >= T) return;
   const int e0 = lane * P;
   const int gs = E / G;
-  float beta[P], sc[P];
+  float beta[P], sc[P], z[P];
+  if (P % 4 == 0 && e0 + P <= E) {
+    // whole lane in range: 16-byte loads (E % 16 == 0 keeps them aligned)
+#pragma unroll
+    for (int i = 0; i < P; i += 4) {
+      float4 v = __ldg(reinterpret_cast<const float4*>(part + static_cast<int64_t>(t) * E + e0 + i));
+      for (int sp = 1; sp < splits; ++sp) {
+        const float4 w = __ldg(reinterpret_cast<const float4*>(
+            part + (static_cast<int64_t>(sp) * T + t) * E + e0 + i));
+        v = make_float4(__fadd_rn(v.x, w.x), __fadd_rn(v.y, w.y), __fadd_rn(v.z, w.z),
+                        __fadd_rn(v.w, w.w));
+      }
+      z[i] = v.x;
+      z[i + 1] = v.y;
+      z[i + 2] = v.z;
+      z[i + 3] = v.w;
+      if (logits_out)
+        *reinterpret_cast<float4*>(logits_out + static_cast<int64_t>(t) * E + e0 + i) = v;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+      const int e = e0 + i;
+      z[i] = 0.f;
+      if (e < E) {
+        float v = part[static_cast<int64_t>(t) * E + e];
+        for (int sp = 1; sp < splits; ++sp)
+          v = __fadd_rn(v, part[(static_cast<int64_t>(sp) * T + t) * E + e]);
+        if (logits_out) logits_out[static_cast<int64_t>(t) * E + e] = v;
+        z[i] = v;
+      }
+    }
+  }
 #pragma unroll
   for (int i = 0; i < P; ++i) {
     const int e = e0 + i;
     beta[i] = -INFINITY;
     sc[i] = 0.f;
     if (e < E) {
-      float z = part[static_cast<int64_t>(t) * E + e];
-      for (int sp = 1; sp < splits; ++sp)
-        z = __fadd_rn(z, part[(static_cast<int64_t>(sp) * T + t) * E + e]);
-      if (logits_out) logits_out[static_cast<int64_t>(t) * E + e] = z;
-      sc[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z)));
-      beta[i] = __fadd_rn(sc[i], bias[e]);
+      sc[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z[i])));
+      beta[i] = __fadd_rn(sc[i], __ldg(bias + e));
     }
   }
 
@@ -272,27 +302,62 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
     }
   }
 
+  // experts of groups the token may not use drop out of the selection
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+    if (e0 + i < E && !((allowed >> ((e0 + i) / gs)) & 1u)) beta[i] = -INFINITY;
+
+  // each lane keeps its best remaining candidate (local index bi); a round
+  // takes the warp's best (biased score descending, then lower expert) with
+  // one 5-step argmax on (order-preserving key, expert), and only the lane
+  // that owned it looks for its next best
   uint32_t taken = 0;
+  int bi = -1;
+  float bv = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+    if (e0 + i < E && (bi < 0 || beta[i] > bv)) {
+      bi = i;
+      bv = beta[i];
+    }
   float ssum = 0.f, my_s = 0.f;
   int my_idx = 0;
   for (int k = 0; k < K; ++k) {
-    Cand c{-INFINITY, INT_MAX, 0.f};
+    // order-preserving unsigned key of the score (+0 for both zeros)
+    const float v = bv == 0.f ? 0.f : bv;
+    const uint32_t u = __float_as_uint(v);
+    uint32_t key = bi < 0 ? 0u : ((u & 0x80000000u) ? ~u : (u | 0x80000000u));
+    int ex = bi < 0 ? INT_MAX : e0 + bi;
+    float s_mine = 0.f;
 #pragma unroll
-    for (int i = 0; i < P; ++i) {
-      const int e = e0 + i;
-      if (e < E && ((allowed >> (e / gs)) & 1u) && !((taken >> i) & 1u) &&
-          better(beta[i], e, c.v, c.i)) {
-        c.v = beta[i];
-        c.i = e;
-        c.s = sc[i];
+    for (int i = 0; i < P; ++i)
+      if (i == bi) s_mine = sc[i];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const uint32_t ok = __shfl_xor_sync(0xffffffffu, key, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, ex, off);
+      if (ok > key || (ok == key && oe < ex)) {
+        key = ok;
+        ex = oe;
       }
     }
-    c = warp_best(c);
-    if (c.i / P == lane) taken |= 1u << (c.i - e0);
-    ssum = __fadd_rn(ssum, c.s);
+    const int owner = ex / P;
+    const float s_win = __shfl_sync(0xffffffffu, s_mine, owner);
+    if (lane == owner) {
+      taken |= 1u << (ex - e0);
+      bi = -1;
+      bv = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < P; ++i)
+        if (e0 + i < E && !((taken >> i) & 1u) && (bi < 0 || beta[i] > bv)) {
+          bi = i;
+          bv = beta[i];
+        }
+    }
+    ssum = __fadd_rn(ssum, s_win);
     if (lane == k) {
-      my_idx = c.i;
-      my_s = c.s;
+      my_idx = ex;
+      my_s = s_win;
     }
   }
   if (lane < K) {
