@@ -102,7 +102,8 @@ class ClockSampler:
             try:
                 self.samples.append((time.perf_counter(),
                                      pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
-                                     pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                                     pynvml.nvmlDeviceGetCurrentClocksEventReasons(h),
+                                     pynvml.nvmlDeviceGetPowerUsage(h)))
             except Exception:  # noqa: BLE001 - a failed read drops one sample
                 pass
             time.sleep(0.002)
@@ -141,13 +142,16 @@ class ClockSampler:
             if not smp:
                 return {"sm_mhz": None, "sm_max_mhz": self.max_mhz,
                         "reasons": ["no samples in the timed region"], "source": "nvml"}
-            reasons = set()
-            for _, _, bits in smp:
+            reasons, masks = set(), set()
+            for _, _, bits, _ in smp:
+                masks.add(int(bits))
                 for b, n in self.REASONS.items():
                     if bits & b:
                         reasons.add(n)
             return {"sm_mhz": statistics.median(x[1] for x in smp), "sm_max_mhz": self.max_mhz,
                     "reasons": sorted(reasons), "samples": len(smp),
+                    "power_w_median": round(statistics.median(x[3] for x in smp) / 1000.0, 1),
+                    "reason_masks": sorted(hex(m) for m in masks),
                     "source": "nvml, polled every 2 ms, samples inside the timed region"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}

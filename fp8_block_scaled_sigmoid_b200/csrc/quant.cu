@@ -30,19 +30,28 @@ __global__ void __launch_bounds__(kQ1Threads) quant_1x128_kernel(
   const int64_t total = static_cast<int64_t>(rows) * tiles_per_row;
   const int64_t first = (static_cast<int64_t>(blockIdx.x) * (kQ1Threads / 16) + hw) * kTilesPerHW;
   const int cols = tiles_per_row * 128;
+  // (row, tile-in-row) of the first tile; the next ones step along the row
+  // (one division per half-warp, not per tile)
+  const int64_t r0 = first / tiles_per_row;
+  const int j0 = static_cast<int>(first - r0 * tiles_per_row);
 
   uint4 v[kTilesPerHW];
+  {
+    int64_t r = r0;
+    int j = j0;
 #pragma unroll
-  for (int i = 0; i < kTilesPerHW; ++i) {
-    const int64_t t = first + i;
-    v[i] = make_uint4(0, 0, 0, 0);
-    if (t < total) {
-      const int64_t r = t / tiles_per_row;
-      const int j = static_cast<int>(t - r * tiles_per_row);
-      const uint16_t* src = x + r * ldx + j * 128 + lane16 * 8;
-      v[i] = __ldg(reinterpret_cast<const uint4*>(src));
+    for (int i = 0; i < kTilesPerHW; ++i) {
+      v[i] = make_uint4(0, 0, 0, 0);
+      if (first + i < total)
+        v[i] = __ldg(reinterpret_cast<const uint4*>(x + r * ldx + j * 128 + lane16 * 8));
+      if (++j == tiles_per_row) {
+        j = 0;
+        ++r;
+      }
     }
   }
+  int64_t r = r0;
+  int j = j0;
 #pragma unroll
   for (int i = 0; i < kTilesPerHW; ++i) {
     const int64_t t = first + i;
@@ -67,10 +76,12 @@ __global__ void __launch_bounds__(kQ1Threads) quant_1x128_kernel(
                      div_by_scale(f[2], s, rs), div_by_scale(f[3], s, rs));
       out.y = e4m3x4(div_by_scale(f[4], s, rs), div_by_scale(f[5], s, rs),
                      div_by_scale(f[6], s, rs), div_by_scale(f[7], s, rs));
-      const int64_t r = t / tiles_per_row;
-      const int j = static_cast<int>(t - r * tiles_per_row);
       *reinterpret_cast<uint2*>(q + r * cols + j * 128 + lane16 * 8) = out;
       if (lane16 == 0) scale[t] = s;
+    }
+    if (++j == tiles_per_row) {
+      j = 0;
+      ++r;
     }
   }
 }
