@@ -106,6 +106,10 @@ class MoELayer:
         self.out = torch.empty(T, d, dtype=f32, device=dev)
         self.dev_err = torch.zeros(1, dtype=i32, device=dev)
         self.u_dev = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        # second input/output pair and copy streams for forward_host_stream
+        self._u_dev2 = None
+        self._out2 = None
+        self._streams = None
         # first permute allocates the index/tile buffers inside self.perm
         self.max_tiles = _abi.moe_max_m_tiles(T, K, E, True)
 
@@ -137,27 +141,31 @@ class MoELayer:
                                           self.max_tiles, _abi.EP_F32, self.Y,
                                           dev_err=self.dev_err)
 
-    def step_combine(self, u):
+    def step_combine(self, u, out=None):
         P = self.pairs
-        _abi.moe_combine(self.Y, self.perm["dst_of"], self.gate, self.Y[P:], u, self.out)
+        _abi.moe_combine(self.Y, self.perm["dst_of"], self.gate, self.Y[P:], u,
+                         self.out if out is None else out)
 
     def step_bias_update(self):
         counts, T_all = reduce_load_counts(self.perm["counts"], self.T, self.pg)
         _abi.moe_bias_update(counts, T_all, self.cfg.K, self.cfg.gamma, self.bias)
 
     # -- whole layer --------------------------------------------------------
-    def forward(self, u: torch.Tensor, update_bias: bool = True) -> torch.Tensor:
-        """u bf16 [T][d] on the device -> out fp32 [T][d] (self.out)."""
+    def forward(self, u: torch.Tensor, update_bias: bool = True,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+        """u bf16 [T][d] on the device -> out fp32 [T][d] (self.out unless
+        ``out`` is given)."""
         assert u.shape == (self.T, self.cfg.d) and u.dtype == torch.bfloat16
+        out = self.out if out is None else out
         self.step_route(u)
         self.step_quant(u)
         self.step_permute()
         self.step_gemm1()
         self.step_gemm2()
-        self.step_combine(u)
+        self.step_combine(u, out)
         if update_bias:
             self.step_bias_update()
-        return self.out
+        return out
 
     def forward_host(self, u_host: torch.Tensor, out_host: torch.Tensor,
                      update_bias: bool = True) -> torch.Tensor:
@@ -167,6 +175,50 @@ class MoELayer:
         self.forward(self.u_dev, update_bias)
         out_host.copy_(self.out, non_blocking=True)
         return out_host
+
+    def forward_host_stream(self, u_hosts, out_hosts, update_bias: bool = True):
+        """End-to-end calls over a sequence of batches in pinned host memory
+        (u_hosts[i] bf16 [T][d] -> out_hosts[i] fp32 [T][d]), with the copies
+        overlapped: batch i+1's host->device copy and batch i-1's
+        device->host copy run on their own streams while batch i computes on
+        the current stream.  Two device input and output buffers alternate;
+        each batch's layer steps (and its bias update) run in order on the
+        current stream.  Returns out_hosts once every copy has been queued;
+        the caller synchronises (or waits on the current stream, which is
+        made to wait for the last copies)."""
+        import torch as _t
+        assert len(u_hosts) == len(out_hosts)
+        if self._u_dev2 is None:
+            self._u_dev2 = [self.u_dev, _t.empty_like(self.u_dev)]
+            self._out2 = [self.out, _t.empty_like(self.out)]
+            self._streams = (_t.cuda.Stream(self.dev), _t.cuda.Stream(self.dev))
+        s_in, s_out = self._streams
+        comp = _t.cuda.current_stream(self.dev)
+        start = _t.cuda.Event()
+        start.record(comp)
+        in_ready = [None, None]    # input buffer b holds batch data
+        comp_done = [start, start]  # compute that last read u_dev2[b] / wrote out2[b]
+        out_read = [start, start]  # device->host copy that last read out2[b]
+        for i, (uh, oh) in enumerate(zip(u_hosts, out_hosts)):
+            b = i & 1
+            with _t.cuda.stream(s_in):
+                s_in.wait_event(comp_done[b])  # the batch before last is done with u_dev2[b]
+                self._u_dev2[b].copy_(uh, non_blocking=True)
+                in_ready[b] = _t.cuda.Event()
+                in_ready[b].record(s_in)
+            comp.wait_event(in_ready[b])
+            comp.wait_event(out_read[b])      # out2[b] has been copied out
+            self.forward(self._u_dev2[b], update_bias, out=self._out2[b])
+            comp_done[b] = _t.cuda.Event()
+            comp_done[b].record(comp)
+            with _t.cuda.stream(s_out):
+                s_out.wait_event(comp_done[b])
+                oh.copy_(self._out2[b], non_blocking=True)
+                out_read[b] = _t.cuda.Event()
+                out_read[b].record(s_out)
+        comp.wait_event(out_read[0])
+        comp.wait_event(out_read[1])
+        return out_hosts
 
     def check(self) -> None:
         """Raise if a kernel recorded a device-side error (synchronises)."""

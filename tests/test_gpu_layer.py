@@ -123,3 +123,25 @@ def test_layer_v3_prefill_sampled(cuda_dev):
             assert_within_rms(npraw(layer.Y[row]), y[0], what=f"Y row {row}")
             ref_out = ref_out + g * y[0]
         assert_within_rms(outg[t], ref_out, what=f"token {t}")
+
+
+def test_forward_host_stream_matches_forward(cuda_dev):
+    """The overlapped host-to-host call gives, batch by batch, the bytes of
+    the plain device call (same kernels in the same order, the bias updated
+    after every batch), with the copies on their own streams."""
+    cfg = configs.TINY
+    layer, bias0 = _build(cfg, cuda_dev)
+    us = [inputs.draw_u(cfg.with_(seed=cfg.seed + i), cuda_dev) for i in range(5)]
+    ref = [layer.forward(u).clone() for u in us]
+    bias_ref = layer.bias.clone()
+    torch.cuda.synchronize()
+    layer.bias.copy_(bias0)
+    hosts = [u.cpu().pin_memory() for u in us]
+    outs = [torch.full((cfg.T, cfg.d), float("nan"), dtype=torch.float32).pin_memory()
+            for _ in us]
+    layer.forward_host_stream(hosts, outs)
+    torch.cuda.synchronize()
+    layer.check()
+    for r, o in zip(ref, outs):
+        assert torch.equal(r.cpu(), o)
+    assert torch.equal(layer.bias, bias_ref)
