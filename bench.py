@@ -275,13 +275,21 @@ def run_gpu(args):
     layer.check()
 
     names = ["route", "quant", "permute", "gemm1", "gemm2", "combine", "bias"]
+    use_graph = world == 1 and args.graph
+    sampler = ClockSampler(local) if rank == 0 else None
+
+    def start_sampler():
+        if sampler:
+            sampler.start()
+            if sampler.proc is not None:
+                time.sleep(0.3)  # nvidia-smi needs a moment before its first sample
+
+    # headline: K eager steps with an event between every call (with --graph,
+    # K CUDA-graph replays of the step are timed as the headline instead)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
           for _ in range(args.steps)]
-    sampler = ClockSampler(local) if rank == 0 else None
-    if sampler:
-        sampler.start()
-        if sampler.proc is not None:
-            time.sleep(0.3)  # nvidia-smi needs a moment before its first sample
+    if not use_graph:
+        start_sampler()
     barrier()
     t_lo = time.perf_counter()
     lc0 = _abi.launch_count
@@ -306,14 +314,38 @@ def run_gpu(args):
     barrier()
     t_hi = time.perf_counter()
     launches = _abi.launch_count - lc0
-    if sampler:
-        sampler.window(t_lo, t_hi)
-    clocks = sampler.stop() if sampler else None
     layer.check()
     step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
     per_kernel = {n: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)) / args.steps
                   for j, n in enumerate(names)}
-    total_ms = max_over_ranks(sum(step_ms), dev, pg)
+    eager_ms = max_over_ranks(sum(step_ms), dev, pg)
+    total_ms = eager_ms
+    if use_graph:
+        # headline: the whole step replayed from a CUDA graph, one host call
+        # per step (same kernels, same order; the L2 flush stays outside)
+        graph, per_replay = layer.capture(u)
+        for i in range(args.warmup):
+            flush.fill_(i & 0xFF)
+            graph.replay()
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        start_sampler()
+        barrier()
+        t_lo = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            gev[i][0].record(st)
+            graph.replay()
+            gev[i][1].record(st)
+        barrier()
+        t_hi = time.perf_counter()
+        layer.check()
+        launches = per_replay * args.steps
+        total_ms = sum(a.elapsed_time(b) for a, b in gev)
+        del graph
+    if sampler:
+        sampler.window(t_lo, t_hi)
+    clocks = sampler.stop() if sampler else None
     tokens = cfg.T * world * args.steps
     value = tokens / (total_ms / 1e3)
 
@@ -393,6 +425,7 @@ def run_gpu(args):
                        "host->device copy of u and a device->host copy of the output, "
                        "overlapped with the neighbouring steps' compute on copy streams"},
         "gpu_launches": launches,
+        "step_launch": "one CUDA-graph replay per step" if use_graph else "eager calls",
         "roofline": roofline,
         "gemm": gemm,
         "kernel_ms": {k: round(v, 4) for k, v in per_kernel.items()},
@@ -553,6 +586,8 @@ def main():
     ap.add_argument("--config", default="v3_prefill")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time CUDA-graph replays of the step instead of eager calls (one GPU)")
     ap.add_argument("--gemm", action="store_true",
                     help="time the standalone 4096x7168x2048 block-scaled GEMM instead")
     args = ap.parse_args()

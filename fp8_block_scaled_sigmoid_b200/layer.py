@@ -176,6 +176,27 @@ class MoELayer:
         out_host.copy_(self.out, non_blocking=True)
         return out_host
 
+    def capture(self, u: torch.Tensor, update_bias: bool = True):
+        """Record one forward step on the device input ``u`` (bf16 [T][d];
+        the graph keeps its address, so refill it in place) into a CUDA
+        graph.  ``graph.replay()`` then queues the whole layer -- every
+        kernel, in order, on the current stream -- with one host call.  One
+        eager step runs first (it sets the kernels' launch attributes and
+        allocates the permutation's tables), so the bias is updated once.
+        Single GPU: the multi-rank bias update holds a collective.
+        Returns (graph, kernels per replay)."""
+        assert self.pg is None, "capture() is single-GPU"
+        side = torch.cuda.Stream(self.dev)
+        side.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(side):
+            self.forward(u, update_bias)
+        torch.cuda.current_stream(self.dev).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        n0 = _abi.launch_count
+        with torch.cuda.graph(graph):
+            self.forward(u, update_bias)
+        return graph, _abi.launch_count - n0
+
     def forward_host_stream(self, u_hosts, out_hosts, update_bias: bool = True):
         """End-to-end calls over a sequence of batches in pinned host memory
         (u_hosts[i] bf16 [T][d] -> out_hosts[i] fp32 [T][d]), with the copies

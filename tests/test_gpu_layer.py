@@ -145,3 +145,25 @@ def test_forward_host_stream_matches_forward(cuda_dev):
     for r, o in zip(ref, outs):
         assert torch.equal(r.cpu(), o)
     assert torch.equal(layer.bias, bias_ref)
+
+
+def test_captured_step_matches_forward(cuda_dev):
+    """A CUDA-graph replay of the layer step gives the bytes of the eager
+    call on the same input and bias."""
+    cfg = configs.TINY
+    layer, bias0 = _build(cfg, cuda_dev)
+    u = inputs.draw_u(cfg, cuda_dev)
+    graph, n = layer.capture(u)       # runs one eager step first
+    assert n == sum(_abi.LAUNCHES_PER_CALL[k] for k in (
+        "moe_route", "fp8_quant_1x128", "moe_permute", "moe_combine", "moe_bias_update")) + 2
+    torch.cuda.synchronize()
+    layer.bias.copy_(bias0)
+    ref = layer.forward(u).clone()
+    bias_ref = layer.bias.clone()
+    layer.bias.copy_(bias0)
+    layer.out.fill_(float("nan"))
+    graph.replay()
+    torch.cuda.synchronize()
+    layer.check()
+    assert torch.equal(layer.out, ref)
+    assert torch.equal(layer.bias, bias_ref)
