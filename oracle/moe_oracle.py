@@ -23,7 +23,9 @@ design notes):
     ordered by biased score descending, then index ascending;
   * bias update uses sign(c_i - T*K/E) with sign(0) = 0;
   * Swish beta = 1 (SiLU); shared expert has the routed experts' width and
-    gate 1; expert outputs and the layer output are fp32/fp64, not bf16.
+    gate 1; expert outputs and the layer output are fp32/fp64, not bf16;
+  * the balance loss's TopK (eq. 18) is over the raw affinities of all
+    routed experts, ties to the lower index.
 
 Parity pins: every function here is pinned by tests that do not re-type its
 formula (brute-force enumeration, exhaustive code tables, closed forms,
@@ -343,6 +345,47 @@ def bias_update(counts, T: int, K: int, gamma: float, bias) -> np.ndarray:
     b = np.asarray(bias, np.float32).astype(np.float64)
     g = np.float64(np.float32(gamma))
     return (b - g * sgn).astype(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# Complementary sequence-wise balance loss.  [ANN] "Complementary
+# Sequence-Wise Auxiliary Loss", eqs. (17)-(20), for each sequence of T
+# tokens:
+#   L_Bal = alpha * sum_i f_i P_i,
+#   f_i   = N_r / (K_r T) * #{t : s_{i,t} in TopK({s_{j,t}}_j, K_r)},
+#   s'_{i,t} = s_{i,t} / sum_j s_{j,t},   P_i = (1/T) sum_t s'_{i,t};
+# alpha = 0.0001 for DeepSeek-V3 ([ANN] training hyper-parameters; [BLOG]
+# 1.2.3).  Reading: the TopK of eq. (18) is taken over the raw affinities of
+# all N_r routed experts, as written (no bias, no group limit), ties to the
+# lower index.
+# ---------------------------------------------------------------------------
+def seq_balance_loss(z, K: int, seq_len: int, alpha: float = 1e-4):
+    """Per sequence of seq_len consecutive tokens of the logits z [T][E]:
+    (loss [n_seq], f [n_seq][E], P [n_seq][E], k_margin [T]) with k_margin the
+    per-token gap between the K-th and (K+1)-th raw affinity (for setting
+    aside near-ties when the membership counts are compared)."""
+    z = np.asarray(z, np.float64)
+    T, E = z.shape
+    assert T % seq_len == 0 and 0 < K <= E
+    s = sigmoid(z)
+    member = np.zeros((T, E), bool)
+    k_margin = np.full(T, np.inf)
+    experts = np.arange(E)
+    for t in range(T):
+        ordr = _order_desc(s[t], experts)
+        member[t, ordr[:K]] = True
+        if K < E:
+            k_margin[t] = s[t, ordr[K - 1]] - s[t, ordr[K]]
+    s_norm = s / s.sum(axis=1, keepdims=True)
+    n_seq = T // seq_len
+    f = np.zeros((n_seq, E))
+    P = np.zeros((n_seq, E))
+    for q in range(n_seq):
+        rows = slice(q * seq_len, (q + 1) * seq_len)
+        f[q] = E / (K * seq_len) * member[rows].sum(axis=0)
+        P[q] = s_norm[rows].sum(axis=0) / seq_len
+    loss = alpha * (f * P).sum(axis=1)
+    return loss, f, P, k_margin
 
 
 # ---------------------------------------------------------------------------

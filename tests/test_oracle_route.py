@@ -318,3 +318,59 @@ def test_tiny_layer_invariants():
     hq, hs = O.swiglu_quant(gu, cfg.I)
     y = O.dequant_1x128(hq, hs) @ O.dequant_128x128(w2q[e], w2s[e]).T
     assert np.allclose(y[0], Y[r["dst_of"][t, k]], rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------- sequence-wise balance loss --
+# [ANN] "Complementary Sequence-Wise Auxiliary Loss", eqs. (17)-(20).
+def test_seq_balance_loss_hand_example():
+    """Two tokens, three experts, K=1, one sequence, alpha=1.  The logits are
+    chosen so the affinities are exact: sigmoid(ln 3) = 3/4, sigmoid(0) = 1/2,
+    sigmoid(-ln 3) = 1/4.
+      token 0: s = (3/4, 1/2, 1/4), sum 3/2 -> s' = (1/2, 1/3, 1/6), top-1 = 0
+      token 1: s = (1/4, 3/4, 1/2), sum 3/2 -> s' = (1/6, 1/2, 1/3), top-1 = 1
+      f = 3/(1*2) * (1, 1, 0) = (3/2, 3/2, 0)
+      P = ((1/2+1/6)/2, (1/3+1/2)/2, (1/6+1/3)/2) = (1/3, 5/12, 1/4)
+      L = 3/2*1/3 + 3/2*5/12 = 9/8"""
+    l3 = math.log(3.0)
+    z = np.array([[l3, 0.0, -l3], [-l3, l3, 0.0]])
+    loss, f, P, _ = O.seq_balance_loss(z, K=1, seq_len=2, alpha=1.0)
+    assert np.allclose(f[0], [1.5, 1.5, 0.0], rtol=0, atol=1e-15)
+    assert np.allclose(P[0], [1 / 3, 5 / 12, 1 / 4], rtol=0, atol=1e-15)
+    assert abs(loss[0] - 9 / 8) < 1e-14
+
+
+@pytest.mark.parametrize("E,K,S", [(4, 2, 4), (16, 4, 8), (64, 8, 16)])
+def test_seq_balance_loss_uniform_affinities(E, K, S):
+    """Equal logits: every s' = 1/E, the ties go to experts 0..K-1, so
+    f = E/K on them and 0 elsewhere, and L = alpha * K * (E/K) * (1/E) = alpha."""
+    z = np.full((2 * S, E), 0.3)
+    loss, f, P, _ = O.seq_balance_loss(z, K=K, seq_len=S, alpha=1e-4)
+    assert np.allclose(loss, 1e-4, rtol=1e-14, atol=0)
+    want_f = np.zeros(E)
+    want_f[:K] = E / K
+    assert np.array_equal(f, np.stack([want_f, want_f]))
+    assert np.allclose(P, 1.0 / E, rtol=1e-14, atol=0)
+
+
+def test_seq_balance_loss_invariants_and_sequences():
+    """Random logits: sum_i f_i = N_r (each token counts K experts, scaled by
+    N_r/(K T)); sum_i P_i = 1 (each s' row sums to 1); 0 < L <= alpha*N_r/K
+    (P sums to 1, f_i <= N_r/K); sequences are independent (the loss of each
+    sequence equals the loss computed on it alone)."""
+    rng = np.random.default_rng(17)
+    E, K, S = 32, 6, 24
+    z = rng.normal(0, 1.5, (3 * S, E))
+    loss, f, P, _ = O.seq_balance_loss(z, K=K, seq_len=S, alpha=2e-4)
+    assert np.allclose(f.sum(axis=1), E, rtol=1e-13, atol=0)
+    assert np.allclose(P.sum(axis=1), 1.0, rtol=1e-13, atol=0)
+    assert (loss > 0).all() and (loss <= 2e-4 * E / K + 1e-18).all()
+    for q in range(3):
+        lq, fq, Pq, _ = O.seq_balance_loss(z[q * S:(q + 1) * S], K=K, seq_len=S, alpha=2e-4)
+        assert lq[0] == loss[q] and np.array_equal(fq[0], f[q]) and np.array_equal(Pq[0], P[q])
+    # a token whose affinity mass sits on its own top-K raises the loss it
+    # would have with flat affinities: concentrating every token on the same
+    # K experts gives f = N_r/K there and P close to 1/K, so L -> alpha*N_r/K
+    zc = np.full((S, E), -30.0)
+    zc[:, :K] = 30.0
+    lc, _, _, _ = O.seq_balance_loss(zc, K=K, seq_len=S, alpha=1.0)
+    assert abs(lc[0] - E / K) < 1e-9
