@@ -43,6 +43,8 @@ _SIGS = {
     "swiglu_quant": (_i, [_p, _i, _i, _p, _p, _p]),
     "moe_combine": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_bias_update": (_i, [_p, _i, _i64, _i, _f, _p, _p]),
+    "moe_seq_balance_loss_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
+    "moe_seq_balance_loss": (_i, [_p, _i, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
 }
 
 EP_F32 = 0
@@ -56,7 +58,8 @@ _lib = None
 LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant": 1,
                      "moe_route": 2, "moe_permute": 4, "moe_permute_noalloc": 4,
                      "moe_tile_table": 1,
-                     "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1}
+                     "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1,
+                     "moe_seq_balance_loss": 3}
 launch_count = 0
 
 
@@ -315,6 +318,31 @@ def moe_combine(Y, dst_of, topk_gate, Y_shared, u, out=None, stream=None):
     _check(lib().moe_combine(_ptr(Y), _ptr(dst_of), _ptr(topk_gate), _ptr(Y_shared), _ptr(u),
                              T, K, d, _ptr(out), _stream(stream)), "moe_combine")
     return out
+
+
+def moe_seq_balance_loss(logits, K, seq_len, alpha=1e-4, with_fp=False, ws=None, stream=None):
+    """Sequence-wise balance loss of logits fp32 [T][E] (moe_route's
+    logits_out) per sequence of seq_len tokens.  Returns loss fp32 [T/seq_len],
+    or (loss, f, P) with with_fp."""
+    T, E = logits.shape
+    dev = _dev(logits)
+    n_seq = T // seq_len if seq_len > 0 else 0
+    loss = torch.empty(max(n_seq, 1), dtype=torch.float32, device=dev)
+    f = torch.empty(max(n_seq, 1), E, dtype=torch.float32, device=dev) if with_fp else None
+    P = torch.empty(max(n_seq, 1), E, dtype=torch.float32, device=dev) if with_fp else None
+    n = _sz(0)
+    _check(lib().moe_seq_balance_loss_workspace_size(T, E, seq_len, ctypes.byref(n)),
+           "moe_seq_balance_loss_workspace_size")
+    if ws is None:
+        ws = torch.empty(max(n.value, 16), dtype=torch.uint8, device=dev)
+    _count("moe_seq_balance_loss")
+    _check(lib().moe_seq_balance_loss(_ptr(logits), T, E, K, seq_len, float(alpha), _ptr(loss),
+                                      _ptr(f), _ptr(P), _ptr(ws), ws.numel() * ws.element_size(),
+                                      _stream(stream)), "moe_seq_balance_loss")
+    loss = loss[:n_seq]
+    if with_fp:
+        return loss, f[:n_seq], P[:n_seq]
+    return loss
 
 
 def moe_bias_update(counts, T, K, gamma, bias, stream=None):

@@ -78,7 +78,8 @@ class MoELayer:
     """Device buffers and call sequence of one layer for a fixed batch size T."""
 
     def __init__(self, cfg: MoEConfig, centroids: torch.Tensor, bias: torch.Tensor,
-                 w1q, w1s, w2q, w2s, T: int | None = None, process_group=None):
+                 w1q, w1s, w2q, w2s, T: int | None = None, process_group=None,
+                 keep_logits: bool = False):
         self.cfg = cfg
         self.T = cfg.T if T is None else T
         self.dev = centroids.device
@@ -92,6 +93,8 @@ class MoELayer:
         dev = self.dev
         i32, f32, u8 = torch.int32, torch.float32, torch.uint8
         self.idx = torch.empty(T, K, dtype=i32, device=dev)
+        # router logits of the last step, kept for seq_balance_loss
+        self.logits = torch.empty(T, E, dtype=f32, device=dev) if keep_logits else None
         self.gate = torch.empty(T, K, dtype=f32, device=dev)
         self.route_ws = torch.empty(max(_abi.moe_route_workspace_size(T, d, E), 16), dtype=u8, device=dev)
         self.Xq = torch.empty(P + T, d, dtype=u8, device=dev)
@@ -117,7 +120,7 @@ class MoELayer:
     def step_route(self, u):
         c = self.cfg
         _abi.moe_route(u, self.centroids, self.bias, c.G, c.M, c.K, self.idx, self.gate,
-                       ws=self.route_ws, dev_err=self.dev_err)
+                       logits_out=self.logits, ws=self.route_ws, dev_err=self.dev_err)
 
     def step_quant(self, u):
         _abi.fp8_quant_1x128(u, self.Xq[self.pairs:], self.Xs[self.pairs:])
@@ -175,6 +178,13 @@ class MoELayer:
         self.forward(self.u_dev, update_bias)
         out_host.copy_(self.out, non_blocking=True)
         return out_host
+
+    def seq_balance_loss(self, seq_len: int, alpha: float = 1e-4, with_fp: bool = False):
+        """The complementary sequence-wise balance loss (eqs. 17-20) of the
+        last step's router logits, per sequence of seq_len tokens (the layer
+        must be built with keep_logits=True)."""
+        assert self.logits is not None, "build the layer with keep_logits=True"
+        return _abi.moe_seq_balance_loss(self.logits, self.cfg.K, seq_len, alpha, with_fp)
 
     def capture(self, u: torch.Tensor, update_bias: bool = True):
         """Record one forward step on the device input ``u`` (bf16 [T][d];

@@ -245,6 +245,26 @@ moe_status moe_combine(const float* Y, const int32_t* dst_of, const float* topk_
 moe_status moe_bias_update(const int32_t* counts, int E, int64_t T, int K, float gamma,
                            float* bias, moe_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * moe_seq_balance_loss -- the complementary sequence-wise balance loss,
+ * [ANN] "Complementary Sequence-Wise Auxiliary Loss", eqs. (17)-(20), for
+ * every sequence of seq_len consecutive tokens:
+ *   L = alpha * sum_i f_i P_i,  f_i = E / (K * seq_len) * #{t : i in TopK(s_t)},
+ *   P_i = (1/seq_len) * sum_t s_{i,t} / sum_j s_{j,t},  s = Sigmoid(logits);
+ * the TopK over the raw affinities of all E routed experts (no bias, no group
+ * limit), ties to the lower index.  DeepSeek-V3 uses alpha = 1e-4.
+ * Deterministic (fixed reduction orders, no atomics); fp32 arithmetic.
+ *   logits fp32 [T][E] (moe_route's logits_out);  T % seq_len == 0
+ *   loss fp32 [T/seq_len]; f, P fp32 [T/seq_len][E] (each may be NULL)
+ *   ws: moe_seq_balance_loss_workspace_size bytes (T*E floats plus the
+ *       per-128-token partials)
+ * Limits: K <= min(E, 32), E <= 1024.
+ */
+moe_status moe_seq_balance_loss_workspace_size(int T, int E, int seq_len, size_t* bytes);
+moe_status moe_seq_balance_loss(const float* logits, int T, int E, int K, int seq_len,
+                                float alpha, float* loss, float* f, float* P, void* ws,
+                                size_t ws_bytes, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

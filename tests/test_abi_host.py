@@ -61,6 +61,14 @@ def test_max_m_tiles_bound():
                                               None, 4, 1, 256, 128, 7, None, None, None,
                                               None), 1),                      # bad epilogue
     (lambda L: L.swiglu_quant(None, 4, 100, None, None, None), 2),
+    (lambda L: L.moe_seq_balance_loss(None, 100, 16, 4, 30, ctypes.c_float(1e-4), None, None,
+                                      None, None, 0, None), 2),              # T % seq_len
+    (lambda L: L.moe_seq_balance_loss(None, 100, 16, 40, 50, ctypes.c_float(1e-4), None, None,
+                                      None, None, 0, None), 2),              # K > 32
+    (lambda L: L.moe_seq_balance_loss(None, 100, 2048, 4, 50, ctypes.c_float(1e-4), None, None,
+                                      None, None, 0, None), 4),              # E > 1024
+    (lambda L: L.moe_seq_balance_loss(None, 100, 16, 4, 50, ctypes.c_float(1e-4), None, None,
+                                      None, None, 0, None), 1),              # NULL logits
     (lambda L: L.moe_combine(None, None, None, None, None, 4, 40, 128, None, None), 4),
     (lambda L: L.moe_bias_update(None, 4, 8, 2, ctypes.c_float(0.001), None, None), 1),
 ])
