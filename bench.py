@@ -367,6 +367,27 @@ def run_gpu(args):
     e2e_value = tokens / (e2e_ms / 1e3)
     out_host = out_hosts[0]
 
+    # the sequence-wise balance loss (eqs. 17-20) of this batch's router logits,
+    # one sequence of T tokens; off the step (a training-time reduction)
+    logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
+    _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K, logits_out=logits)
+    bl_ws = torch.empty(max(_abi.moe_seq_balance_loss_ws(cfg.T, cfg.E, cfg.T), 16),
+                        dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        _abi.moe_seq_balance_loss(logits, cfg.K, cfg.T, ws=bl_ws)
+    bl0, bl1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    bl0.record(st)
+    for _ in range(args.steps):
+        _abi.moe_seq_balance_loss(logits, cfg.K, cfg.T, ws=bl_ws)
+    bl1.record(st)
+    barrier()
+    bl_us = bl0.elapsed_time(bl1) * 1e3 / args.steps
+    # logits read twice, normalised rows written once and read once
+    bl_bytes = 4 * cfg.T * cfg.E * 4
+    balance_loss = {"us": round(bl_us, 2), "seq_len": cfg.T, "bytes": bl_bytes,
+                    "gbs": round(bl_bytes / (bl_us * 1e-6) / 1e9, 1)}
+    del logits, bl_ws
+
     # roofline of the dominant kernel (grouped GEMM 1 with the SwiGLU epilogue)
     counts = layer.perm["counts"].cpu()
     active = int((counts > 0).sum()) + cfg.n_shared
@@ -429,6 +450,7 @@ def run_gpu(args):
         "roofline": roofline,
         "gemm": gemm,
         "kernel_ms": {k: round(v, 4) for k, v in per_kernel.items()},
+        "seq_balance_loss": balance_loss,
         "loads": {"max": int(counts.max()), "mean": float(counts.float().mean()),
                   "active_experts": active - cfg.n_shared},
         "clocks": clocks,

@@ -320,6 +320,13 @@ def moe_combine(Y, dst_of, topk_gate, Y_shared, u, out=None, stream=None):
     return out
 
 
+def moe_seq_balance_loss_ws(T, E, seq_len) -> int:
+    n = _sz(0)
+    _check(lib().moe_seq_balance_loss_workspace_size(T, E, seq_len, ctypes.byref(n)),
+           "moe_seq_balance_loss_workspace_size")
+    return n.value
+
+
 def moe_seq_balance_loss(logits, K, seq_len, alpha=1e-4, with_fp=False, ws=None, stream=None):
     """Sequence-wise balance loss of logits fp32 [T][E] (moe_route's
     logits_out) per sequence of seq_len tokens.  Returns loss fp32 [T/seq_len],

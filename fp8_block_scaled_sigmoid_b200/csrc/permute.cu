@@ -9,11 +9,12 @@
 //  2. scan    -- one CTA: per expert a running sum over chunks (chunk bases),
 //                then an exclusive scan over experts -> offsets, and the
 //                128-row tile table of every segment.
-//  3. scatter -- per chunk, one warp walks its tokens in order, several
-//                tokens per step (lane = (token, k)); lanes that picked the
-//                same expert are ranked with __match_any_sync in lane order,
-//                which is token order, so each expert's rows stay in
-//                ascending token order.
+//  3. scatter -- per chunk, four warps each walk a quarter of its tokens in
+//                order, several tokens per step (lane = (token, k)), from
+//                per-warp cursors (the chunk base plus the earlier quarters'
+//                counts); lanes that picked the same expert are ranked with
+//                __match_any_sync in lane order, which is token order, so
+//                each expert's rows stay in ascending token order.
 //  4. gather  -- one warp per destination row copies the FP8 row (16-byte
 //                vectors, coalesced) and its 1x128 scales.
 #include <mutex>
@@ -144,43 +145,66 @@ __global__ void __launch_bounds__(kScanThreads) perm_scan_kernel(
   }
 }
 
-__global__ void __launch_bounds__(32) perm_scatter_kernel(const int32_t* __restrict__ idx, int T,
-                                                          int K, int E,
-                                                          const int32_t* __restrict__ cbase,
-                                                          int32_t* __restrict__ src_row,
-                                                          int32_t* __restrict__ dst_of) {
+// One CTA per chunk, kScatterWarps warps: warp j places the pairs of tokens
+// [j*kChunkT/kScatterWarps, ...) of the chunk.  Each warp's starting cursor
+// per expert is the chunk base plus the pairs of that expert in the earlier
+// warps' tokens (counted first), so the result is the one a single warp
+// walking the whole chunk would produce.
+constexpr int kScatterWarps = 4;
+constexpr int kTokPerWarp = kChunkT / kScatterWarps;
+
+__global__ void __launch_bounds__(32 * kScatterWarps) perm_scatter_kernel(
+    const int32_t* __restrict__ idx, int T, int K, int E, const int32_t* __restrict__ cbase,
+    int32_t* __restrict__ src_row, int32_t* __restrict__ dst_of) {
   extern __shared__ int32_t sm[];
-  int32_t* cursor = sm;       // [E]
-  int32_t* sidx = sm + E;     // [kChunkT * K]
-  const int lane = threadIdx.x;
+  int32_t* cursor = sm;                       // [kScatterWarps][E]
+  int32_t* hist = sm + kScatterWarps * E;     // [kScatterWarps][E]
+  int32_t* sidx = sm + 2 * kScatterWarps * E; // [kChunkT * K]
+  const int lane = threadIdx.x & 31, wj = threadIdx.x >> 5;
   const int t0 = blockIdx.x * kChunkT;
   const int nt = min(kChunkT, T - t0);
-  for (int e = lane; e < E; e += 32) cursor[e] = cbase[static_cast<int64_t>(blockIdx.x) * E + e];
-  for (int p = lane; p < nt * K; p += 32) sidx[p] = idx[static_cast<int64_t>(t0) * K + p];
-  __syncwarp();
+  for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) hist[i] = 0;
+  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) sidx[p] = idx[static_cast<int64_t>(t0) * K + p];
+  __syncthreads();
+  // pairs per expert in each warp's tokens (integer adds: order-free)
+  const int wt0 = wj * kTokPerWarp, wt1 = min(nt, wt0 + kTokPerWarp);
+  for (int p = wt0 * K + lane; p < wt1 * K; p += 32) {
+    const int e = sidx[p];
+    if (e >= 0 && e < E) atomicAdd(&hist[wj * E + e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = cbase[static_cast<int64_t>(blockIdx.x) * E + e];
+    for (int j = 0; j < kScatterWarps; ++j) {
+      cursor[j * E + e] = run;
+      run += hist[j * E + e];
+    }
+  }
+  __syncthreads();
+  int32_t* cur = cursor + wj * E;
   const int tpi = 32 / K;  // tokens per step
   const int tl = lane / K, k = lane - (lane / K) * K;
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int tb = 0; tb < nt; tb += tpi) {
+  for (int tb = wt0; tb < wt1; tb += tpi) {
     const int tt = tb + tl;
     int e = -1;
-    if (tl < tpi && tt < nt) e = sidx[tt * K + k];
+    if (tl < tpi && tt < wt1) e = sidx[tt * K + k];
     const bool active = e >= 0 && e < E;
     const unsigned amask = __ballot_sync(0xffffffffu, active);
     unsigned peers = 0;
     int pos = 0;
     if (active) {
       peers = __match_any_sync(amask, e);
-      pos = cursor[e] + __popc(peers & lt_mask);
+      pos = cur[e] + __popc(peers & lt_mask);
     }
     __syncwarp();
-    if (active && lane == __ffs(peers) - 1) cursor[e] += __popc(peers);
+    if (active && lane == __ffs(peers) - 1) cur[e] += __popc(peers);
     __syncwarp();
     if (active) {
       const int t = t0 + tt;
       src_row[pos] = t;
       dst_of[static_cast<int64_t>(t) * K + k] = pos;
-    } else if (tl < tpi && tt < nt) {
+    } else if (tl < tpi && tt < wt1) {
       dst_of[static_cast<int64_t>(t0 + tt) * K + k] = -1;  // flagged bad index: no row
     }
   }
@@ -275,8 +299,9 @@ extern "C" moe_status moe_permute(const int32_t* topk_idx, int T, int K, int E, 
                                                tile_group, tile_start, n_tiles, max_tiles, dev_err);
   MOE_CUDA_CHECK_LAUNCH();
   if (nch > 0) {
-    const size_t sm = (static_cast<size_t>(E) + kChunkT * K) * sizeof(int32_t);
-    perm_scatter_kernel<<<nch, 32, sm, st>>>(topk_idx, T, K, E, ccount, src_row, dst_of);
+    const size_t sm = (2 * kScatterWarps * static_cast<size_t>(E) + kChunkT * K) * sizeof(int32_t);
+    perm_scatter_kernel<<<nch, 32 * kScatterWarps, sm, st>>>(topk_idx, T, K, E, ccount, src_row,
+                                                             dst_of);
     MOE_CUDA_CHECK_LAUNCH();
     const int rows = T * K;
     perm_gather_kernel<<<(rows + 7) / 8, 256, 0, st>>>(src_row, rows, T, xq, xscale, d, xq_perm,
