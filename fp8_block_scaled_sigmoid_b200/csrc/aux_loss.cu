@@ -11,7 +11,7 @@
 //               normalised s' and the raw top-K; writes s' with the sign bit
 //               set on the K chosen experts (s' > 0, so the sign carries the
 //               membership) -> ws [T][E].
-//  2. chunk  -- one CTA per 128-token chunk of a sequence, one thread per
+//  2. chunk  -- one CTA per 32-token chunk of a sequence, one thread per
 //               expert: sums |s'| and the members over the chunk in token
 //               order -> partials [chunks][E] (sum, count).
 //  3. final  -- one CTA per sequence: sums its chunks in order, f_i P_i per
@@ -24,7 +24,7 @@ namespace moe {
 namespace {
 
 constexpr int kAuxTokThreads = 256;  // 8 tokens per CTA in pass 1
-constexpr int kAuxChunk = 128;       // tokens per partial in pass 2
+constexpr int kAuxChunk = 32;        // tokens per partial in pass 2
 
 template <int P>
 __global__ void __launch_bounds__(kAuxTokThreads) aux_token_kernel(const float* __restrict__ z,
@@ -102,7 +102,18 @@ __global__ void aux_chunk_kernel(const float* __restrict__ ws, int E, int seq_le
   const int t1 = q * seq_len + min(seq_len, (c + 1) * kAuxChunk);
   float acc = 0.f;
   int cnt = 0;
-  for (int t = t0; t < t1; ++t) {
+  int t = t0;
+  for (; t + 8 <= t1; t += 8) {  // eight loads in flight, summed in token order
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = __ldg(ws + static_cast<int64_t>(t + j) * E + e);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      acc = __fadd_rn(acc, fabsf(v[j]));
+      cnt += v[j] < 0.f;
+    }
+  }
+  for (; t < t1; ++t) {
     const float v = __ldg(ws + static_cast<int64_t>(t) * E + e);
     acc = __fadd_rn(acc, fabsf(v));
     cnt += v < 0.f;

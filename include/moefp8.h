@@ -257,7 +257,7 @@ moe_status moe_bias_update(const int32_t* counts, int E, int64_t T, int K, float
  *   logits fp32 [T][E] (moe_route's logits_out);  T % seq_len == 0
  *   loss fp32 [T/seq_len]; f, P fp32 [T/seq_len][E] (each may be NULL)
  *   ws: moe_seq_balance_loss_workspace_size bytes (T*E floats plus the
- *       per-128-token partials)
+ *       per-32-token partials)
  * Limits: K <= min(E, 32), E <= 1024.
  */
 moe_status moe_seq_balance_loss_workspace_size(int T, int E, int seq_len, size_t* bytes);
