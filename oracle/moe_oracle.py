@@ -25,7 +25,9 @@ design notes):
   * Swish beta = 1 (SiLU); shared expert has the routed experts' width and
     gate 1; expert outputs and the layer output are fp32/fp64, not bf16;
   * the balance loss's TopK (eq. 18) is over the raw affinities of all
-    routed experts, ties to the lower index.
+    routed experts, ties to the lower index;
+  * a power-of-two scale is the fp32 scale above rounded up to the next
+    power of two (nothing saturates; x / scale is exact).
 
 Parity pins: every function here is pinned by tests that do not re-type its
 formula (brute-force enumeration, exhaustive code tables, closed forms,
@@ -128,6 +130,53 @@ def quant_128x128(w) -> tuple[np.ndarray, np.ndarray]:
         for j in range(cols // TILE):
             b = blk[:, j * TILE:(j + 1) * TILE]
             s = _scale_of(np.abs(b).max())
+            scale[i, j] = s
+            q[i * TILE:(i + 1) * TILE, j * TILE:(j + 1) * TILE] = e4m3_encode((b / s).astype(np.float32))
+    return q, scale
+
+
+# ---------------------------------------------------------------------------
+# Power-of-two scales.  [ANN] "Low-Precision Storage and Communication": the
+# activations quantised before the dispatch to the MoE up-projection (like the
+# input of the Linear after attention) carry scaling factors that are integral
+# powers of 2.  Reading: the power of two is the fp32 scale above rounded UP
+# (the smallest 2^e >= fl32(max(amax, eps)/448)), so no element saturates and
+# x / 2^e is exact in fp32.  The block-scaled variant applies the same rounding
+# to the 128x128 weight blocks and to the SwiGLU output, so that every operand
+# scale of both expert GEMMs is a pure exponent (UE8M0).
+# ---------------------------------------------------------------------------
+def pow2_ceil(s) -> np.ndarray:
+    """Smallest power of two >= s, for positive finite s (returned in fp32)."""
+    s = np.asarray(s, np.float64)
+    if (s <= 0).any() or not np.isfinite(s).all():
+        raise ValueError("pow2_ceil: positive finite scales only")
+    m, ex = np.frexp(s)                  # s = m * 2^ex, m in [0.5, 1)
+    return np.where(m == 0.5, s, np.ldexp(1.0, ex)).astype(np.float32)
+
+
+def quant_1x128_pow2(x) -> tuple[np.ndarray, np.ndarray]:
+    """quant_1x128 with each tile's scale rounded up to a power of two."""
+    x = np.asarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    assert cols % TILE == 0
+    tiles = x.reshape(rows, cols // TILE, TILE)
+    scale = pow2_ceil(_scale_of(np.abs(tiles).max(axis=2)))
+    y = (tiles / scale[:, :, None]).astype(np.float32)
+    return e4m3_encode(y).reshape(rows, cols), scale
+
+
+def quant_128x128_pow2(w) -> tuple[np.ndarray, np.ndarray]:
+    """quant_128x128 with each block's scale rounded up to a power of two."""
+    w = np.asarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    assert cols % TILE == 0
+    rb = -(-rows // TILE)
+    q = np.empty((rows, cols), dtype=np.uint8)
+    scale = np.empty((rb, cols // TILE), dtype=np.float32)
+    for i in range(rb):
+        for j in range(cols // TILE):
+            b = w[i * TILE:(i + 1) * TILE, j * TILE:(j + 1) * TILE]
+            s = pow2_ceil(_scale_of(np.abs(b).max()))
             scale[i, j] = s
             q[i * TILE:(i + 1) * TILE, j * TILE:(j + 1) * TILE] = e4m3_encode((b / s).astype(np.float32))
     return q, scale
@@ -309,10 +358,12 @@ def swiglu(gu, I: int) -> np.ndarray:
     return h.reshape(rows, I)
 
 
-def swiglu_quant(gu, I: int):
+def swiglu_quant(gu, I: int, pow2: bool = False):
     """SwiGLU, then 1x128 online quantisation of its fp32 value (the input of
-    the down projection is FP8 like every other GEMM input)."""
-    return quant_1x128(swiglu(gu, I).astype(np.float32))
+    the down projection is FP8 like every other GEMM input); ``pow2`` rounds
+    the scales up to powers of two."""
+    h = swiglu(gu, I).astype(np.float32)
+    return quant_1x128_pow2(h) if pow2 else quant_1x128(h)
 
 
 # ---------------------------------------------------------------------------
@@ -391,27 +442,31 @@ def seq_balance_loss(z, K: int, seq_len: int, alpha: float = 1e-4):
 # ---------------------------------------------------------------------------
 # Whole layer, composed from the steps above.
 # ---------------------------------------------------------------------------
-def quantise_weights(w1, w2):
-    """Per expert 128x128 block quantisation of the stacked bf16 weights."""
+def quantise_weights(w1, w2, pow2: bool = False):
+    """Per expert 128x128 block quantisation of the stacked bf16 weights
+    (``pow2``: scales rounded up to powers of two)."""
     w1 = np.asarray(w1, np.float32)
     w2 = np.asarray(w2, np.float32)
-    q1, s1 = zip(*[quant_128x128(w) for w in w1])
-    q2, s2 = zip(*[quant_128x128(w) for w in w2])
+    qf = quant_128x128_pow2 if pow2 else quant_128x128
+    q1, s1 = zip(*[qf(w) for w in w1])
+    q2, s2 = zip(*[qf(w) for w in w2])
     return np.stack(q1), np.stack(s1), np.stack(q2), np.stack(s2)
 
 
 def moe_layer(u, centroids, bias, w1q, w1s, w2q, w2s, G, M, K, gamma,
-              h_override=None):
+              h_override=None, pow2: bool = False):
     """Forward of one layer plus the bias update.  Weights are given already
     quantised ([E+1] stacks, shared expert last).  ``h_override`` =
     (hq, hs) makes the second GEMM consume given FP8 activations (used to
-    check the second GEMM and the combine on the CUDA path's own operands)."""
+    check the second GEMM and the combine on the CUDA path's own operands).
+    ``pow2`` quantises the activations and the SwiGLU output with power-of-two
+    scales (the weights must then be quantised with ``pow2`` too)."""
     u = np.asarray(u, np.float32)
     T, d = u.shape
     E = np.asarray(centroids).shape[0]
     I = np.asarray(w1q).shape[1] // 2
     idx, gate, rinfo = route(u, centroids, bias, G, M, K)
-    xq_tok, xs_tok = quant_1x128(u)
+    xq_tok, xs_tok = quant_1x128_pow2(u) if pow2 else quant_1x128(u)
     counts, offsets, src_row, dst_of = permute(idx, E)
     pairs = T * K
     xq = np.concatenate([xq_tok[src_row], xq_tok])
@@ -419,7 +474,7 @@ def moe_layer(u, centroids, bias, w1q, w1s, w2q, w2s, G, M, K, gamma,
     offs = segment_offsets_with_shared(offsets, T)
     gu = grouped_gemm(xq, xs, w1q, w1s, offs)
     if h_override is None:
-        hq, hs = swiglu_quant(gu, I)
+        hq, hs = swiglu_quant(gu, I, pow2)
     else:
         hq, hs = h_override
     Y = grouped_gemm(hq, hs, w2q, w2s, offs)
