@@ -256,11 +256,12 @@ def run_gpu(args):
 
     cfg = configs.PRESETS[args.config]
     cfg_rank = cfg.with_(seed=cfg.seed + rank)       # each rank its own token batch
-    w1q, w1s, w2q, w2s = make_fp8_weights(cfg, dev)  # same weights on every rank
+    w1q, w1s, w2q, w2s = make_fp8_weights(cfg, dev, pow2=args.pow2)  # same on every rank
     cent = inputs.draw_centroids(cfg, dev)
     bias = inputs.draw_bias(cfg, dev)
     u = inputs.draw_u(cfg_rank, dev)
-    layer = MoELayer(cfg, cent, bias.clone(), w1q, w1s, w2q, w2s, process_group=pg)
+    layer = MoELayer(cfg, cent, bias.clone(), w1q, w1s, w2q, w2s, process_group=pg,
+                     pow2=args.pow2)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream()
 
@@ -406,19 +407,20 @@ def run_gpu(args):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     fp8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = g1_bytes / t1 / 1e9
-    traffic = read_traffic("grouped_gemm_fp8", cfg.name)
+    gemm_name = "grouped_gemm_fp8_pow2" if args.pow2 else "grouped_gemm_fp8"
+    traffic = read_traffic(gemm_name, cfg.name)
     # the dominant kernel's bound: weight streaming below the ridge point
     # (FP8 peak / HBM bandwidth, in FLOP per byte), the tensor pipe above it
     ridge = fp8_peak * 1e12 / (hbm * 1e9)
     src_note = (f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback")
     if g1_flops / g1_bytes < ridge:
-        roofline = {"kernel": "grouped_gemm_fp8 (GEMM 1, SwiGLU+quant epilogue)", "bound": "hbm",
+        roofline = {"kernel": f"{gemm_name} (GEMM 1, SwiGLU+quant epilogue)", "bound": "hbm",
                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                     "frac": round(achieved / hbm, 4), "traffic": traffic,
                     "peak_source": f"hbm_gbs, {src_note}", "algorithmic_bytes": int(g1_bytes)}
     else:
         tf1 = g1_flops / t1 / 1e12
-        roofline = {"kernel": "grouped_gemm_fp8 (GEMM 1, SwiGLU+quant epilogue)",
+        roofline = {"kernel": f"{gemm_name} (GEMM 1, SwiGLU+quant epilogue)",
                     "bound": "tensor", "achieved": round(tf1, 1), "peak": fp8_peak,
                     "unit": "TFLOP/s", "frac": round(tf1 / fp8_peak, 4), "traffic": traffic,
                     "peak_source": f"2 x bf16_tflops, {src_note} (nominal fp8:bf16 ratio)",
@@ -438,7 +440,9 @@ def run_gpu(args):
         "config": {"workload": workload_name(cfg), "tokens_per_gpu": cfg.T,
                    "parallelism": f"dp{world} (full expert set per GPU, load counts all-reduced)"
                    if world > 1 else "single GPU",
-                   "l2": "512 MB buffer written between timed steps; FP8 weights (11.3 GB) > L2"},
+                   "l2": "512 MB buffer written between timed steps; FP8 weights (11.3 GB) > L2",
+                   "scales": "powers of two; the tensor core applies them (UE8M0 block scaling)"
+                   if args.pow2 else "fp32 amax/448; promoted per 128-wide K block"},
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(u_host.numel() * u_host.element_size()),
                 "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
@@ -559,15 +563,15 @@ def run_gemm(args):
     dev = torch.device("cuda", 0)
     cfg = configs.STANDALONE_GEMM
     a, bt = inputs.draw_gemm(cfg, dev)
-    aq, sa = _abi.fp8_quant_1x128(a)
-    bq, sb = _abi.fp8_quant_128x128(bt.unsqueeze(0))
+    aq, sa = _abi.fp8_quant_1x128(a, pow2=args.pow2)
+    bq, sb = _abi.fp8_quant_128x128(bt.unsqueeze(0), pow2=args.pow2)
     offs = torch.tensor([0, cfg.M], dtype=torch.int32, device=dev)
     mt = cfg.M // 128
     tg, ts, nt = _abi.moe_tile_table(offs, mt)
     D = torch.empty(cfg.M, cfg.N, dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
-        _abi.grouped_gemm_fp8_blockscaled(aq, sa, bq, sb, offs, tg, ts, nt, mt, D=D)
+        _abi.grouped_gemm_fp8_blockscaled(aq, sa, bq, sb, offs, tg, ts, nt, mt, D=D, pow2=args.pow2)
     torch.cuda.synchronize()
     sampler = ClockSampler(0)
     sampler.start()
@@ -578,7 +582,7 @@ def run_gemm(args):
         flush.fill_(i & 0xFF)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        _abi.grouped_gemm_fp8_blockscaled(aq, sa, bq, sb, offs, tg, ts, nt, mt, D=D)
+        _abi.grouped_gemm_fp8_blockscaled(aq, sa, bq, sb, offs, tg, ts, nt, mt, D=D, pow2=args.pow2)
         e1.record()
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
@@ -592,7 +596,9 @@ def run_gemm(args):
         "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 4), "higher_is_better": True, "dtype": "fp8_e4m3",
         "config": {"workload": f"{cfg.name}: A {cfg.M}x{cfg.K} (1x128 scales, 1% outliers x50) "
-                               f"x B^T {cfg.N}x{cfg.K} (128x128 scales), fp32 out",
+                               f"x B^T {cfg.N}x{cfg.K} (128x128 scales), fp32 out"
+                               + (", power-of-two scales applied by the tensor core"
+                                  if args.pow2 else ""),
                    "l2": "512 MB buffer written between timed launches"},
         "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4),
@@ -610,6 +616,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true",
                     help="time CUDA-graph replays of the step instead of eager calls (one GPU)")
+    ap.add_argument("--pow2", action="store_true",
+                    help="power-of-two scale variant (tensor-core UE8M0 block scaling)")
     ap.add_argument("--gemm", action="store_true",
                     help="time the standalone 4096x7168x2048 block-scaled GEMM instead")
     args = ap.parse_args()

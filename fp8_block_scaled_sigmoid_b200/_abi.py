@@ -29,6 +29,8 @@ _SIGS = {
     "moe_abi_version": (_i, []),
     "fp8_quant_1x128": (_i, [_p, _i64, _i, _i, _p, _p, _p]),
     "fp8_quant_128x128": (_i, [_p, _i64, _i, _i, _p, _p, _p]),
+    "fp8_quant_1x128_pow2": (_i, [_p, _i64, _i, _i, _p, _p, _p]),
+    "fp8_quant_128x128_pow2": (_i, [_p, _i64, _i, _i, _p, _p, _p]),
     "moe_route_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
     "moe_route": (_i, [_p, _i64, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _sz, _p, _p]),
     "moe_max_m_tiles": (_i, [_i, _i, _i, _i]),
@@ -40,6 +42,8 @@ _SIGS = {
     "moe_tile_table": (_i, [_p, _i, _i, _p, _p, _p, _p, _p]),
     "grouped_gemm_fp8_blockscaled": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
                                           _i, _p, _p, _p, _p]),
+    "grouped_gemm_fp8_pow2": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
+                                   _i, _p, _p, _p, _p]),
     "swiglu_quant": (_i, [_p, _i, _i, _p, _p, _p]),
     "moe_combine": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_bias_update": (_i, [_p, _i, _i64, _i, _f, _p, _p]),
@@ -50,12 +54,14 @@ _SIGS = {
 EP_F32 = 0
 EP_SWIGLU_QUANT = 1
 DEVERR = {0: "none", 1: "bounded wait timed out", 2: "inconsistent segment table",
-          3: "expert index out of range"}
+          3: "expert index out of range", 4: "a scale is not a power of two"}
 
 _lib = None
 
 # Kernels each entry point launches (for the benchmark's launch count).
 LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant": 1,
+                     "fp8_quant_1x128_pow2": 1, "fp8_quant_128x128_pow2": 1,
+                     "grouped_gemm_fp8_pow2": 1,
                      "moe_route": 2, "moe_permute": 4, "moe_permute_noalloc": 4,
                      "moe_tile_table": 1,
                      "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1,
@@ -116,21 +122,24 @@ def _dev(t):
 
 
 # ----------------------------------------------------------------- quant ---
-def fp8_quant_1x128(x, q=None, scale=None, stream=None):
-    """x bf16 [rows][cols] (row stride may exceed cols) -> (q uint8, scale fp32)."""
+def fp8_quant_1x128(x, q=None, scale=None, stream=None, pow2=False):
+    """x bf16 [rows][cols] (row stride may exceed cols) -> (q uint8, scale fp32);
+    pow2 rounds every scale up to a power of two."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     rows, cols = x.shape
     q = torch.empty(rows, cols, dtype=torch.uint8, device=_dev(x)) if q is None else q
     scale = torch.empty(rows, cols // 128, dtype=torch.float32, device=_dev(x)) if scale is None else scale
-    _count("fp8_quant_1x128")
-    _check(lib().fp8_quant_1x128(_ptr(x), x.stride(0), rows, cols, _ptr(q), _ptr(scale),
-                                 _stream(stream)), "fp8_quant_1x128")
+    name = "fp8_quant_1x128_pow2" if pow2 else "fp8_quant_1x128"
+    _count(name)
+    _check(getattr(lib(), name)(_ptr(x), x.stride(0), rows, cols, _ptr(q), _ptr(scale),
+                                _stream(stream)), name)
     return q, scale
 
 
-def fp8_quant_128x128(w, q=None, scale=None, stream=None):
+def fp8_quant_128x128(w, q=None, scale=None, stream=None, pow2=False):
     """w bf16 [rows][cols] or a stack [G][N][K] (N % 128 == 0) -> (q, scale)
-    with scale [ceil(rows/128)][cols/128] (stack: [G][N/128][K/128])."""
+    with scale [ceil(rows/128)][cols/128] (stack: [G][N/128][K/128]); pow2
+    rounds every scale up to a power of two."""
     assert w.dtype == torch.bfloat16 and w.stride(-1) == 1
     shape = w.shape
     w2 = w.reshape(-1, shape[-1])
@@ -142,9 +151,10 @@ def fp8_quant_128x128(w, q=None, scale=None, stream=None):
         sshape = ((rows + 127) // 128, cols // 128)
     q = torch.empty(shape, dtype=torch.uint8, device=_dev(w)) if q is None else q
     scale = torch.empty(sshape, dtype=torch.float32, device=_dev(w)) if scale is None else scale
-    _count("fp8_quant_128x128")
-    _check(lib().fp8_quant_128x128(_ptr(w2), w2.stride(0), rows, cols, _ptr(q), _ptr(scale),
-                                   _stream(stream)), "fp8_quant_128x128")
+    name = "fp8_quant_128x128_pow2" if pow2 else "fp8_quant_128x128"
+    _count(name)
+    _check(getattr(lib(), name)(_ptr(w2), w2.stride(0), rows, cols, _ptr(q), _ptr(scale),
+                                _stream(stream)), name)
     return q, scale
 
 
@@ -288,10 +298,12 @@ def moe_tile_table(offsets, max_tiles, tile_group=None, tile_start=None, n_tiles
 # ------------------------------------------------------------------ GEMM ---
 def grouped_gemm_fp8_blockscaled(A, sa, B, sb, offsets, tile_group, tile_start, n_tiles,
                                  max_tiles, ep=EP_F32, D=None, d_scale=None, dev_err=None,
-                                 stream=None):
+                                 stream=None, pow2=False):
     """A uint8 [rows][K], sa fp32 [rows][K/128], B uint8 [G][N][K], sb fp32
     [G][N/128][K/128].  ep=EP_F32 -> D fp32 [rows][N]; ep=EP_SWIGLU_QUANT ->
-    (h uint8 [rows][N/2], h_scale fp32 [rows][N/256])."""
+    (h uint8 [rows][N/2], h_scale fp32 [rows][N/256]).  pow2 calls
+    grouped_gemm_fp8_pow2 (every scale a power of two; the tensor core
+    applies them)."""
     rows, K = A.shape
     G, N, _ = B.shape
     dev = _dev(A)
@@ -300,12 +312,12 @@ def grouped_gemm_fp8_blockscaled(A, sa, B, sb, offsets, tile_group, tile_start, 
     else:
         D = torch.empty(rows, N // 2, dtype=torch.uint8, device=dev) if D is None else D
         d_scale = torch.empty(rows, N // 256, dtype=torch.float32, device=dev) if d_scale is None else d_scale
-    _count("grouped_gemm_fp8_blockscaled")
-    _check(lib().grouped_gemm_fp8_blockscaled(_ptr(A), _ptr(sa), rows, _ptr(B), _ptr(sb),
-                                              _ptr(offsets), _ptr(tile_group), _ptr(tile_start),
-                                              _ptr(n_tiles), max_tiles, G, N, K, ep, _ptr(D),
-                                              _ptr(d_scale), _ptr(dev_err), _stream(stream)),
-           "grouped_gemm_fp8_blockscaled")
+    name = "grouped_gemm_fp8_pow2" if pow2 else "grouped_gemm_fp8_blockscaled"
+    _count(name)
+    _check(getattr(lib(), name)(_ptr(A), _ptr(sa), rows, _ptr(B), _ptr(sb), _ptr(offsets),
+                                _ptr(tile_group), _ptr(tile_start), _ptr(n_tiles), max_tiles, G,
+                                N, K, ep, _ptr(D), _ptr(d_scale), _ptr(dev_err), _stream(stream)),
+           name)
     return D if ep == EP_F32 else (D, d_scale)
 
 

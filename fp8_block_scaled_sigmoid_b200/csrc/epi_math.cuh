@@ -18,6 +18,14 @@ __device__ __forceinline__ float quant_scale(float amax) {
   return __fdiv_rn(fmaxf(amax, kQuantEps), kE4M3Max);
 }
 
+// Smallest power of two >= s for a positive normal fp32 s: a non-zero
+// mantissa moves the exponent up by one and is cleared.
+__device__ __forceinline__ float pow2_ceil(float s) {
+  uint32_t b = __float_as_uint(s);
+  if (b & 0x007FFFFFu) b = (b & 0x7F800000u) + 0x00800000u;
+  return __uint_as_float(b);
+}
+
 // x / s rounded to nearest even, given r = RN(1/s): Markstein's correction
 // step (P. W. Markstein, "Computation of elementary functions on the IBM
 // RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): y = RN(x r),

@@ -143,6 +143,100 @@ __device__ __forceinline__ Work decode_work(int w, int nN, const int* rstart, co
 }
 
 // ------------------------------------------------------------------ epilogue
+// Writes one finished tile from this thread's fp32 accumulators: row r_in of
+// the tile, columns c_lo..c_lo+63 and c_hi..c_hi+63 as 64 packed pairs.  POW2
+// rounds the requantisation scale of h up to a power of two.  Returns false
+// if a bounded wait gave up.
+template <int EP, bool POW2>
+__device__ __forceinline__ bool write_tile(const GemmArgs& args, const Work& t, float2 (&acc)[64],
+                                           int warp, int lane, int N, int& xtile, uint64_t* xbar,
+                                           float* amax_x, volatile int* abort_v) {
+  const int g = (warp - 4) >> 2;
+  const int r_in = (warp & 3) * 32 + lane;
+  const int64_t arow = static_cast<int64_t>(t.row0) + r_in;
+  const bool row_ok = r_in < t.rows;
+  if (EP == MOE_EP_F32) {
+    // Each lane holds one row (128 columns).  Per 32-column chunk, the 8
+    // lanes of each group (rows rb..rb+7) transpose their 8 x 8 block of
+    // float4 with three xor-butterfly exchange rounds: afterwards lane rb+i
+    // holds columns 4i..4i+3 of every row of the group, so one store
+    // instruction writes 4 rows x 128 contiguous bytes (whole lines).
+    const int li = lane & 7;
+    const int rb = r_in - li;  // first row of this lane's group inside the tile
+    float* base = static_cast<float*>(args.D) + (static_cast<int64_t>(t.row0) + rb) * N +
+                  t.n_idx * kBN + 128 * g + 4 * li;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      float4 e[8];  // e[j] = columns 32b + 4j .. 32b + 4j + 3 of this lane's row
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float2 x0 = acc[16 * b + 2 * j], x1 = acc[16 * b + 2 * j + 1];
+        e[j] = make_float4(x0.x, x0.y, x1.x, x1.y);
+      }
+      // round s: for each pair (j0, j0 | s), a lane with bit s set sends e[j0]
+      // and receives its partner's e[j0 | s] into e[j0]; the other sends
+      // e[j0 | s] and receives into it
+#pragma unroll
+      for (int sft = 1; sft < 8; sft <<= 1) {
+        const bool hi = (lane & sft) != 0;
+#pragma unroll
+        for (int j0 = 0; j0 < 8; ++j0) {
+          if (j0 & sft) continue;
+          const int j1 = j0 | sft;
+          const float4 x = hi ? e[j0] : e[j1];
+          float4 y;
+          y.x = __shfl_xor_sync(0xffffffffu, x.x, sft);
+          y.y = __shfl_xor_sync(0xffffffffu, x.y, sft);
+          y.z = __shfl_xor_sync(0xffffffffu, x.z, sft);
+          y.w = __shfl_xor_sync(0xffffffffu, x.w, sft);
+          if (hi) e[j0] = y;
+          else e[j1] = y;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (rb + j < t.rows)
+          *reinterpret_cast<float4*>(base + static_cast<int64_t>(j) * N + 32 * b) = e[j];
+    }
+  } else {
+    // h = SiLU(gate) * up overwrites the gate accumulators: h[2i], h[2i+1]
+    // are acc[i].x, acc[i].y; the up channels are acc[32..63]
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      acc[i].x = silu_mul(acc[i].x, acc[32 + i].x);
+      acc[i].y = silu_mul(acc[i].y, acc[32 + i].y);
+      amax = fmaxf(amax, fmaxf(fabsf(acc[i].x), fabsf(acc[i].y)));
+    }
+    // the 1x128 tile amax is shared with the partner thread of the other half
+    const int xb = xtile & 1;
+    amax_x[(xb * 2 + g) * 128 + r_in] = amax;
+    mbar_arrive(&xbar[xb]);
+    if (!__all_sync(0xffffffffu, mbar_wait(&xbar[xb], (xtile >> 1) & 1, abort_v, args.dev_err)))
+      return false;
+    amax = fmaxf(amax_x[(xb * 2 + 0) * 128 + r_in], amax_x[(xb * 2 + 1) * 128 + r_in]);
+    ++xtile;
+    const float sq = POW2 ? pow2_ceil(quant_scale(amax)) : quant_scale(amax);
+    const float rq = __frcp_rn(sq);
+    if (row_ok) {
+      const int I = N / 2;
+      uint8_t* dst = static_cast<uint8_t*>(args.D) + arow * I + t.n_idx * 128 + 64 * g;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2* hp = acc + 8 * i;  // h[16i .. 16i+15]
+        uint32_t w4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          w4[j] = e4m3x4(div_by_scale(hp[2 * j].x, sq, rq), div_by_scale(hp[2 * j].y, sq, rq),
+                         div_by_scale(hp[2 * j + 1].x, sq, rq), div_by_scale(hp[2 * j + 1].y, sq, rq));
+        reinterpret_cast<uint4*>(dst)[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+      if (g == 0) args.d_scale[arow * (I / 128) + t.n_idx] = sq;
+    }
+  }
+  return true;
+}
+
 // Promotes every K block of one tile into fp32 registers and writes the
 // tile.  Returns false if a bounded wait gave up.
 template <int EP>
@@ -219,87 +313,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs& args, const Work& 
       acc[48 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), fhi, acc[48 + i]);
     }
   }
-  const bool row_ok = r_in < t.rows;
-  if (EP == MOE_EP_F32) {
-    // Each lane holds one row (128 columns).  Per 32-column chunk, the 8
-    // lanes of each group (rows rb..rb+7) transpose their 8 x 8 block of
-    // float4 with three xor-butterfly exchange rounds: afterwards lane rb+i
-    // holds columns 4i..4i+3 of every row of the group, so one store
-    // instruction writes 4 rows x 128 contiguous bytes (whole lines).
-    const int li = lane & 7;
-    const int rb = r_in - li;  // first row of this lane's group inside the tile
-    float* base = static_cast<float*>(args.D) + (static_cast<int64_t>(t.row0) + rb) * N +
-                  t.n_idx * kBN + 128 * g + 4 * li;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      float4 e[8];  // e[j] = columns 32b + 4j .. 32b + 4j + 3 of this lane's row
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float2 x0 = acc[16 * b + 2 * j], x1 = acc[16 * b + 2 * j + 1];
-        e[j] = make_float4(x0.x, x0.y, x1.x, x1.y);
-      }
-      // round s: for each pair (j0, j0 | s), a lane with bit s set sends e[j0]
-      // and receives its partner's e[j0 | s] into e[j0]; the other sends
-      // e[j0 | s] and receives into it
-#pragma unroll
-      for (int sft = 1; sft < 8; sft <<= 1) {
-        const bool hi = (lane & sft) != 0;
-#pragma unroll
-        for (int j0 = 0; j0 < 8; ++j0) {
-          if (j0 & sft) continue;
-          const int j1 = j0 | sft;
-          const float4 x = hi ? e[j0] : e[j1];
-          float4 y;
-          y.x = __shfl_xor_sync(0xffffffffu, x.x, sft);
-          y.y = __shfl_xor_sync(0xffffffffu, x.y, sft);
-          y.z = __shfl_xor_sync(0xffffffffu, x.z, sft);
-          y.w = __shfl_xor_sync(0xffffffffu, x.w, sft);
-          if (hi) e[j0] = y;
-          else e[j1] = y;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (rb + j < t.rows)
-          *reinterpret_cast<float4*>(base + static_cast<int64_t>(j) * N + 32 * b) = e[j];
-    }
-  } else {
-    // h = SiLU(gate) * up overwrites the gate accumulators: h[2i], h[2i+1]
-    // are acc[i].x, acc[i].y; the up channels are acc[32..63]
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      acc[i].x = silu_mul(acc[i].x, acc[32 + i].x);
-      acc[i].y = silu_mul(acc[i].y, acc[32 + i].y);
-      amax = fmaxf(amax, fmaxf(fabsf(acc[i].x), fabsf(acc[i].y)));
-    }
-    // the 1x128 tile amax is shared with the partner thread of the other half
-    const int xb = xtile & 1;
-    amax_x[(xb * 2 + g) * 128 + r_in] = amax;
-    mbar_arrive(&xbar[xb]);
-    if (!__all_sync(0xffffffffu, mbar_wait(&xbar[xb], (xtile >> 1) & 1, abort_v, args.dev_err)))
-      return false;
-    amax = fmaxf(amax_x[(xb * 2 + 0) * 128 + r_in], amax_x[(xb * 2 + 1) * 128 + r_in]);
-    ++xtile;
-    const float sq = quant_scale(amax);
-    const float rq = __frcp_rn(sq);
-    if (row_ok) {
-      const int I = N / 2;
-      uint8_t* dst = static_cast<uint8_t*>(args.D) + arow * I + t.n_idx * 128 + 64 * g;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2* hp = acc + 8 * i;  // h[16i .. 16i+15]
-        uint32_t w4[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          w4[j] = e4m3x4(div_by_scale(hp[2 * j].x, sq, rq), div_by_scale(hp[2 * j].y, sq, rq),
-                         div_by_scale(hp[2 * j + 1].x, sq, rq), div_by_scale(hp[2 * j + 1].y, sq, rq));
-        reinterpret_cast<uint4*>(dst)[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
-      if (g == 0) args.d_scale[arow * (I / 128) + t.n_idx] = sq;
-    }
-  }
-  return true;
+  return write_tile<EP, false>(args, t, acc, warp, lane, N, xtile, xbar, amax_x, abort_v);
 }
 
 // Shared-memory layout after the 1024-aligned ring.
@@ -317,9 +331,9 @@ struct Ctl {
 };
 
 template <int STAGES>
-__device__ __forceinline__ Ctl carve(uint8_t* base) {
+__device__ __forceinline__ Ctl carve(uint8_t* base, int ctl_off = kRingBytes) {
   Ctl c;
-  c.full = reinterpret_cast<uint64_t*>(base + kRingBytes);
+  c.full = reinterpret_cast<uint64_t*>(base + ctl_off);
   c.empty = c.full + STAGES;
   c.tfull = c.empty + STAGES;
   c.tempty = c.tfull + 2;
@@ -327,9 +341,47 @@ __device__ __forceinline__ Ctl carve(uint8_t* base) {
   c.xbar = c.done + 1;
   c.tmem_slot = reinterpret_cast<uint32_t*>(c.xbar + 2);
   c.abort_flag = reinterpret_cast<int*>(c.tmem_slot + 1);
-  c.rstart = reinterpret_cast<int*>(base + kRingBytes + 512);
+  c.rstart = reinterpret_cast<int*>(base + ctl_off + 512);
   c.amax_x = reinterpret_cast<float*>(c.rstart + kMaxGroups + 1);
   return c;
+}
+
+// TMA producer (one thread): every K slice of every work item of this CTA,
+// A rows and the weight tile into the stage ring; waits for its own copies
+// before returning.
+template <int STAGES, int SK>
+__device__ __forceinline__ void tma_producer(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                             const GemmArgs& args, const Ctl& c, uint8_t* base,
+                                             int total, int nN, int KB, volatile int* abort_v) {
+  constexpr int kSub = kBK / SK;
+  constexpr int kA = kBM * SK, kStage = kA + kBN * SK;
+  const int N = args.N;
+  int it = 0;
+  bool live = true;
+  for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
+    const Work t = decode_work<128>(w, nN, c.rstart, args);
+    if (!t.ok) {
+      set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
+      continue;
+    }
+    const int brow = t.e * N + t.n_idx * kBN;
+    for (int kk = 0; kk < KB * kSub; ++kk, ++it) {
+      const int s = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
+      if (!mbar_wait(&c.empty[s], ph ^ 1, abort_v, args.dev_err)) {
+        live = false;
+        break;
+      }
+      uint8_t* sA = base + s * kStage;
+      mbar_arrive_expect_tx(&c.full[s], kStage);
+      tma_load_2d(sA, &tmA, &c.full[s], kk * SK, t.row0);
+      tma_load_2d(sA + kA, &tmB, &c.full[s], kk * SK, brow);
+    }
+  }
+  // every issued copy lands before the CTA can exit
+  const int first = it > STAGES ? it - STAGES : 0;
+  for (int i = first; i < it; ++i)
+    mbar_wait(&c.full[i % STAGES], (i / STAGES) & 1, nullptr, args.dev_err);
 }
 
 // =========================================================== 1-SM mainloop
@@ -381,33 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
     if (warp == 0 && lane == 0) {
-      // ------------------------------------------------------ TMA producer
-      int it = 0;
-      bool live = true;
-      for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
-        const Work t = decode_work<128>(w, nN, c.rstart, args);
-        if (!t.ok) {
-          set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
-          continue;
-        }
-        const int brow = t.e * N + t.n_idx * kBN;
-        for (int kk = 0; kk < KB * kSub; ++kk, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!mbar_wait(&c.empty[s], ph ^ 1, abort_v, args.dev_err)) {
-            live = false;
-            break;
-          }
-          uint8_t* sA = base + s * kStage;
-          mbar_arrive_expect_tx(&c.full[s], kStage);
-          tma_load_2d(sA, &tmA, &c.full[s], kk * SK, t.row0);
-          tma_load_2d(sA + kA, &tmB, &c.full[s], kk * SK, brow);
-        }
-      }
-      // every issued copy lands before the CTA can exit
-      const int first = it > kStages ? it - kStages : 0;
-      for (int i = first; i < it; ++i)
-        mbar_wait(&c.full[i % kStages], (i / kStages) & 1, nullptr, args.dev_err);
+      tma_producer<kStages, SK>(tmA, tmB, args, c, base, total, nN, KB, abort_v);
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------- MMA issuer
       const uint32_t idesc = instr_desc(kFmtE4M3, kFmtE4M3, kBM, kBN);
@@ -461,6 +487,264 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+
+// ================================================ power-of-two scale mainloop
+// When every scale is a power of two (UE8M0), the tensor core applies them
+// itself: tcgen05.mma kind::mxf8f6f4.block_scale multiplies each 32-element K
+// slice of row m of A by 2^SFA[m] and of row n of B by 2^SFB[n] and keeps
+// accumulating the whole K extent in TMEM, so no partial sum is promoted and
+// no scale touches the epilogue.  A 1x128 (or 128x128) scale covers four
+// consecutive 32-element slices, which all read the same exponent.
+//
+// Per ring stage (one 128-wide K block) the scale-factor warps write three
+// 512-byte atoms into shared memory: A's 128 row exponents and B's two 128-row
+// blocks.  Atom byte 16 r + 4 j + b holds the exponent of row 32 j + r for the
+// K block (4 g + b) of the group g the stage belongs to, so the MMAs of K block
+// kb read byte kb % 4.  The MMA thread moves the atoms into TMEM with
+// tcgen05.cp (replicated over the four lane quarters) right before the stage's
+// MMAs; the tensor core runs a thread's tcgen05 operations in issue order, so
+// one TMEM scale region serves every stage.  TMEM: the 256-column accumulator
+// at 0, A's exponents at 256..259, B's at 264..271; with one accumulator the
+// epilogue releases it as soon as it has loaded the tile into registers.
+constexpr int kSfSlot = 1536;       // per stage: A atom + two B atoms
+constexpr uint32_t kTmemSfa = 256, kTmemSfb = 264;
+constexpr int kStagesMx = kRingBytes / ((kBM + kBN) * kBK);
+constexpr size_t kSmemMxBytes = kSmemBytes + kStagesMx * kSfSlot;
+
+// Exponent bytes (UE8M0 = the fp32 biased exponent) of four power-of-two
+// scales, byte i from v[i]; anything that is not a positive normal power of
+// two sets `bad`.
+__device__ __forceinline__ uint32_t ue8m0x4(const float (&v)[4], uint32_t& bad) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t b = __float_as_uint(v[i]);
+    const uint32_t e = b >> 23;  // sign bit included: a negative scale fails below
+    bad |= (b & 0x007FFFFFu) | static_cast<uint32_t>(e == 0u || e >= 255u);
+    w |= (e & 0xFFu) << (8 * i);
+  }
+  return w;
+}
+
+// The scales of K-block group g (blocks 4g..4g+3) for this lane: A rows
+// row0 + lane + 32 j (clamped into the buffer), or the tile's two B blocks.
+template <bool IS_A>
+__device__ __forceinline__ void sf_load_group(const GemmArgs& a, const Work& t, const float* sb0,
+                                              int KB, int g, int lane, float (&v)[4][4]) {
+  if (IS_A) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int64_t r = static_cast<int64_t>(t.row0) + lane + 32 * j;
+      r = r < a.a_rows ? r : a.a_rows - 1;
+      const float* p = a.sa + r * KB;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[j][i] = (4 * g + i < KB) ? __ldg(p + 4 * g + i) : 1.0f;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool in = 4 * g + i < KB;
+      v[0][i] = in ? __ldg(sb0 + 4 * g + i) : 1.0f;
+      v[1][i] = in ? __ldg(sb0 + KB + 4 * g + i) : 1.0f;
+    }
+  }
+}
+
+// Scale-factor producers (warp 2 for A's atom, warp 3 for B's two atoms):
+// per stage, the exponent atoms.  The next group's scales are loaded while
+// the current group's four stages are written.
+template <int STAGES, bool IS_A>
+__device__ __forceinline__ void sf_producer(const GemmArgs& args, const Ctl& c, uint8_t* sf,
+                                            int total, int nN, int KB, int lane,
+                                            volatile int* abort_v) {
+  const int N = args.N;
+  int it = 0;
+  uint32_t bad = 0;
+  bool live = true;
+  for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
+    const Work t = decode_work<128>(w, nN, c.rstart, args);
+    if (!t.ok) continue;
+    const float* sb0 = args.sb + (static_cast<int64_t>(t.e) * (N / 128) + t.n_idx * 2) * KB;
+    float v[4][4];
+    sf_load_group<IS_A>(args, t, sb0, KB, 0, lane, v);
+    for (int g = 0; 4 * g < KB && live; ++g) {
+      const uint32_t p0 = ue8m0x4(v[0], bad), p1 = ue8m0x4(v[1], bad);
+      const uint32_t p2 = IS_A ? ue8m0x4(v[2], bad) : 0u, p3 = IS_A ? ue8m0x4(v[3], bad) : 0u;
+      if (4 * (g + 1) < KB) sf_load_group<IS_A>(args, t, sb0, KB, g + 1, lane, v);
+      for (int j = 0; j < 4 && 4 * g + j < KB; ++j, ++it) {
+        const int s = it % STAGES;
+        if (!__all_sync(0xffffffffu, mbar_wait(&c.empty[s], ((it / STAGES) & 1) ^ 1, abort_v,
+                                                args.dev_err))) {
+          live = false;
+          break;
+        }
+        uint4* slot = reinterpret_cast<uint4*>(sf + s * kSfSlot);
+        if (IS_A) {
+          slot[lane] = make_uint4(p0, p1, p2, p3);
+        } else {
+          slot[32 + lane] = make_uint4(p0, p0, p0, p0);
+          slot[64 + lane] = make_uint4(p1, p1, p1, p1);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.full[s]);
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, bad != 0) && lane == 0) set_dev_err(args.dev_err, MOE_DEVERR_BAD_SCALE);
+}
+
+// Epilogue of one tile: load the accumulator into registers, release it to
+// the MMA thread, then write the tile.
+template <int EP>
+__device__ __forceinline__ bool epilogue_mx_tile(const GemmArgs& args, const Work& t, uint32_t tmem,
+                                                 int warp, int lane, int N, int& tit, int& xtile,
+                                                 uint64_t* tfull, uint64_t* tempty,
+                                                 uint64_t* xbar, float* amax_x,
+                                                 volatile int* abort_v) {
+  const int g = (warp - 4) >> 2;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const int c_lo = (EP == MOE_EP_F32) ? 128 * g : 64 * g;
+  const int c_hi = (EP == MOE_EP_F32) ? 128 * g + 64 : 128 + 64 * g;
+  if (!__all_sync(0xffffffffu, mbar_wait(tfull, tit & 1, abort_v, args.dev_err))) return false;
+  ++tit;
+  tc_fence_after();
+  float2 acc[64];
+  {
+    const uint32_t ta = tmem + lane_base;
+    float v0[32], v1[32], v2[32], v3[32];
+    tmem_ld32(ta + c_lo, v0);
+    tmem_ld32(ta + c_lo + 32, v1);
+    tmem_ld32(ta + c_hi, v2);
+    tmem_ld32(ta + c_hi + 32, v3);
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tempty);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      acc[i] = make_float2(v0[2 * i], v0[2 * i + 1]);
+      acc[16 + i] = make_float2(v1[2 * i], v1[2 * i + 1]);
+      acc[32 + i] = make_float2(v2[2 * i], v2[2 * i + 1]);
+      acc[48 + i] = make_float2(v3[2 * i], v3[2 * i + 1]);
+    }
+  }
+  return write_tile<EP, true>(args, t, acc, warp, lane, N, xtile, xbar, amax_x, abort_v);
+}
+
+// Warp roles as in gemm1sm_kernel, plus warps 2 and 3 = scale-factor
+// producers (A's and B's exponents; warp 2 first builds the work list).
+// Stages are whole 128-wide K blocks.
+template <int EP>
+__global__ void __launch_bounds__(kThreads, 1) gemm_pow2_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const GemmArgs args) {
+  constexpr int kA = kBM * kBK, kB = kBN * kBK;
+  constexpr int kStage = kA + kB;
+  constexpr int kStages = kStagesMx;
+  constexpr int kSfBytes = kStages * kSfSlot;
+  static_assert((2 * kStages + 8) * 8 + 8 <= 512, "barrier area");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sf = base + kRingBytes;
+  const Ctl c = carve<kStages>(base, kRingBytes + kSfBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KB = args.K / kBK, nN = args.N / kBN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&c.full[s], 3);  // TMA bytes + the two scale-factor warps
+      mbar_init(&c.empty[s], 1);
+    }
+    mbar_init(&c.tfull[0], 1);
+    mbar_init(&c.tempty[0], kEpiThreads / 32);
+    mbar_init(c.done, 1);
+    mbar_init(&c.xbar[0], kEpiThreads);
+    mbar_init(&c.xbar[1], kEpiThreads);
+    *c.abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 2) build_tile_prefix<128>(args, c.rstart, lane);
+  if (warp == 1) {
+    tmem_alloc(c.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *c.tmem_slot;
+  volatile int* abort_v = c.abort_flag;
+  const int total = c.rstart[args.groups] * nN;
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+    if (warp == 0 && lane == 0) {
+      tma_producer<kStages, kBK>(tmA, tmB, args, c, base, total, nN, KB, abort_v);
+    } else if (warp == 2) {
+      sf_producer<kStages, true>(args, c, sf, total, nN, KB, lane, abort_v);
+    } else if (warp == 3) {
+      sf_producer<kStages, false>(args, c, sf, total, nN, KB, lane, abort_v);
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------- MMA issuer
+      const uint32_t t_sfa = tmem + kTmemSfa, t_sfb = tmem + kTmemSfb;
+      const uint32_t sf0 = smem_u32(sf);
+      int it = 0, tit = 0;
+      bool live = true;
+      for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
+        const Work t = decode_work<128>(w, nN, c.rstart, args);
+        if (!t.ok) continue;
+        // the accumulator is free once the epilogue has loaded the last tile
+        if (!mbar_wait(&c.tempty[0], (tit & 1) ^ 1, abort_v, args.dev_err)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&c.full[s], (it / kStages) & 1, abort_v, args.dev_err)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfs = sf0 + s * kSfSlot;
+          tmem_cp_32x128b_x4(t_sfa, smem_desc_interleave(sfs, 128));
+          tmem_cp_32x128b_x4(t_sfb, smem_desc_interleave(sfs + 512, 128));
+          tmem_cp_32x128b_x4(t_sfb + 4, smem_desc_interleave(sfs + 1024, 128));
+          const uint32_t sA = smem_u32(base + s * kStage);
+          const uint64_t ad = smem_desc_sw128(sA);
+          const uint64_t bd = smem_desc_sw128(sA + kA);
+          const uint32_t sid = static_cast<uint32_t>(kb & 3);
+          const uint32_t idesc = instr_desc_mx(kBM, kBN, sid);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_mxf8f6f4(tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u,
+                         t_sfa | (sid << 30), t_sfb | (sid << 30));
+          mma_commit(&c.empty[s]);
+        }
+        if (!live) break;
+        mma_commit(&c.tfull[0]);
+        ++tit;
+      }
+      mma_commit(c.done);
+      mbar_wait(c.done, 0, nullptr, args.dev_err);
+    }
+    __syncwarp();
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
+    int tit = 0, xtile = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      const Work t = decode_work<128>(w, nN, c.rstart, args);
+      if (!t.ok) continue;
+      if (!epilogue_mx_tile<EP>(args, t, tmem, warp, lane, args.N, tit, xtile, &c.tfull[0],
+                                &c.tempty[0], c.xbar, c.amax_x, abort_v))
+        break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
 template <int EP>
 const void* kernel_ptr() {
   return reinterpret_cast<const void*>(gemm1sm_kernel<EP, MOE_GEMM_SK>);
@@ -471,11 +755,14 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 }  // namespace moe
 
-extern "C" moe_status grouped_gemm_fp8_blockscaled(
-    const uint8_t* A, const float* sa, int64_t a_rows, const uint8_t* B, const float* sb,
-    const int32_t* offsets, const int32_t* tile_group, const int32_t* tile_start,
-    const int32_t* n_tiles, int max_tiles, int groups, int N, int K, moe_epilogue ep, void* D,
-    float* d_scale, int32_t* dev_err, moe_stream_t stream) {
+namespace {
+
+moe_status gemm_launch(bool pow2, const uint8_t* A, const float* sa, int64_t a_rows,
+                       const uint8_t* B, const float* sb, const int32_t* offsets,
+                       const int32_t* tile_group, const int32_t* tile_start,
+                       const int32_t* n_tiles, int max_tiles, int groups, int N, int K,
+                       moe_epilogue ep, void* D, float* d_scale, int32_t* dev_err,
+                       moe_stream_t stream) {
   using namespace moe;
   if (a_rows < 0 || groups <= 0 || N <= 0 || K <= 0 || max_tiles < 0) return MOE_ERR_INVALID_ARG;
   if (K % kBK != 0 || N % kBN != 0) return MOE_ERR_SHAPE;
@@ -488,7 +775,8 @@ extern "C" moe_status grouped_gemm_fp8_blockscaled(
   if (a_rows > 0x7FFFFFFF || static_cast<int64_t>(groups) * N > 0x7FFFFFFF)
     return MOE_ERR_UNSUPPORTED;
   if (groups > kMaxGroups) return MOE_ERR_UNSUPPORTED;
-  constexpr int SK = MOE_GEMM_SK;
+  // the block-scaled mainloop stages whole 128-byte K blocks
+  const int SK = pow2 ? kBK : MOE_GEMM_SK;
   // A: 128-row boxes; B: the 256 weight rows of a tile; boxes are SK bytes
   // wide with an SK-byte swizzle
   CUtensorMap tmA, tmB;
@@ -513,10 +801,13 @@ extern "C" moe_status grouped_gemm_fp8_blockscaled(
   a.dev_err = dev_err;
   static int configured = 0;
   if (!configured) {
-    for (int i = 0; i < 2; ++i) {
-      const void* f = i == 0 ? kernel_ptr<MOE_EP_F32>() : kernel_ptr<MOE_EP_SWIGLU_QUANT>();
-      if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmemBytes)) != cudaSuccess)
+    const void* fs[4] = {kernel_ptr<MOE_EP_F32>(), kernel_ptr<MOE_EP_SWIGLU_QUANT>(),
+                         reinterpret_cast<const void*>(gemm_pow2_kernel<MOE_EP_F32>),
+                         reinterpret_cast<const void*>(gemm_pow2_kernel<MOE_EP_SWIGLU_QUANT>)};
+    for (int i = 0; i < 4; ++i) {
+      const int bytes = static_cast<int>(i < 2 ? kSmemBytes : kSmemMxBytes);
+      if (cudaFuncSetAttribute(fs[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+          cudaSuccess)
         return MOE_ERR_CUDA;
     }
     configured = 1;
@@ -524,10 +815,35 @@ extern "C" moe_status grouped_gemm_fp8_blockscaled(
   // persistent: one CTA per SM, no more CTAs than work items
   const int64_t work_max = static_cast<int64_t>(max_tiles) * (N / kBN);
   const int ctas = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(moe_num_sms(), work_max)));
-  const void* fn = ep == MOE_EP_F32 ? kernel_ptr<MOE_EP_F32>() : kernel_ptr<MOE_EP_SWIGLU_QUANT>();
+  const void* fn;
+  if (pow2)
+    fn = ep == MOE_EP_F32 ? reinterpret_cast<const void*>(gemm_pow2_kernel<MOE_EP_F32>)
+                          : reinterpret_cast<const void*>(gemm_pow2_kernel<MOE_EP_SWIGLU_QUANT>);
+  else
+    fn = ep == MOE_EP_F32 ? kernel_ptr<MOE_EP_F32>() : kernel_ptr<MOE_EP_SWIGLU_QUANT>();
   void* kargs[3] = {&tmA, &tmB, &a};
-  if (cudaLaunchKernel(fn, dim3(ctas), dim3(kThreads), kargs, kSmemBytes,
+  if (cudaLaunchKernel(fn, dim3(ctas), dim3(kThreads), kargs, pow2 ? kSmemMxBytes : kSmemBytes,
                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status grouped_gemm_fp8_blockscaled(
+    const uint8_t* A, const float* sa, int64_t a_rows, const uint8_t* B, const float* sb,
+    const int32_t* offsets, const int32_t* tile_group, const int32_t* tile_start,
+    const int32_t* n_tiles, int max_tiles, int groups, int N, int K, moe_epilogue ep, void* D,
+    float* d_scale, int32_t* dev_err, moe_stream_t stream) {
+  return gemm_launch(false, A, sa, a_rows, B, sb, offsets, tile_group, tile_start, n_tiles,
+                     max_tiles, groups, N, K, ep, D, d_scale, dev_err, stream);
+}
+
+extern "C" moe_status grouped_gemm_fp8_pow2(
+    const uint8_t* A, const float* sa, int64_t a_rows, const uint8_t* B, const float* sb,
+    const int32_t* offsets, const int32_t* tile_group, const int32_t* tile_start,
+    const int32_t* n_tiles, int max_tiles, int groups, int N, int K, moe_epilogue ep, void* D,
+    float* d_scale, int32_t* dev_err, moe_stream_t stream) {
+  return gemm_launch(true, A, sa, a_rows, B, sb, offsets, tile_group, tile_start, n_tiles,
+                     max_tiles, groups, N, K, ep, D, d_scale, dev_err, stream);
 }

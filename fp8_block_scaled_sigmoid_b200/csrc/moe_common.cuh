@@ -252,6 +252,59 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t a_fmt, uint32_t b_fmt
 constexpr uint32_t kFmtE4M3 = 0;  // kind::f8f6f4
 constexpr uint32_t kFmtBF16 = 1;  // kind::f16
 
+// ------------------------------------------- block-scaled MMA (UE8M0 scales)
+// Instruction descriptor of kind::mxf8f6f4 with E4M3 A and B, both K-major,
+// fp32 accumulator, scale factors in UE8M0 (bit 23 set); sf_id picks which
+// byte of each 32-bit TMEM scale word the MMA reads (B's at bits 4-5, A's at
+// bits 29-30), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+__host__ __device__ constexpr uint32_t instr_desc_mx(uint32_t M, uint32_t N, uint32_t sf_id) {
+  return (sf_id << 4) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) | (sf_id << 29);
+}
+
+// D[tmem] (+)= (A x 2^SFA) (B x 2^SFB)^T over one K = 32 slice: E4M3 operands
+// in shared memory, one UE8M0 exponent per row of A and per row of B read from
+// TMEM at sfa / sfb (the byte chosen by the descriptor's sf ids, which the
+// scale addresses also carry in bits 30-31).  For M = 128 the exponent of row
+// m = 32 j + r sits in TMEM lane r (of every 32-lane quarter), column
+// (sfa + j); for N = 256, row n = 32 j + r of B in lane r, column (sfb + j).
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+      "r"(sfb_tmem)
+      : "memory");
+}
+
+// Shared -> TMEM copy of 32 rows x 16 bytes, replicated into all four 32-lane
+// quarters: lane 32 q + r, columns c..c+3 receive bytes 16 r .. 16 r + 15 of
+// the source (tcgen05.cp 32x128b with warpx4).  Ordered before the tcgen05
+// MMAs this thread issues after it.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+               : "memory");
+}
+
+// Shared-memory descriptor of an unswizzled K-major block of 16-byte rows:
+// 8-row core matrices of 128 contiguous bytes, `sbo` bytes apart (layout 0).
+__device__ __forceinline__ uint64_t smem_desc_interleave(uint32_t smem_addr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(16u >> 4) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+// Make generic-proxy shared-memory writes visible to the async proxy (TMA,
+// tcgen05.cp) before a barrier hands them over.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

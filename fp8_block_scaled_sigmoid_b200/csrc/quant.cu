@@ -15,6 +15,15 @@
 namespace moe {
 namespace {
 
+// The scale of a tile: amax/448 in fp32, or (POW2) that value rounded up to a
+// power of two ("Low-Precision Storage and Communication": scaling factors
+// that are integral powers of 2).  Dividing by a power of two is exact, so
+// div_by_scale returns the plain product x * 2^-e there.
+template <bool POW2>
+__device__ __forceinline__ float tile_scale(float amax) {
+  return POW2 ? pow2_ceil(quant_scale(amax)) : quant_scale(amax);
+}
+
 // ----------------------------------------------------------- 1x128 tiles --
 // A half-warp owns one tile (16 lanes x 8 bf16 = 256 bytes); each half-warp
 // takes kTilesPerHW consecutive tiles, loading all of them before reducing.
@@ -22,6 +31,7 @@ constexpr int kQ1Threads = 256;
 constexpr int kTilesPerHW = 4;
 constexpr int kQ1TilesPerBlock = (kQ1Threads / 16) * kTilesPerHW;
 
+template <bool POW2>
 __global__ void __launch_bounds__(kQ1Threads) quant_1x128_kernel(
     const uint16_t* __restrict__ x, int64_t ldx, int rows, int tiles_per_row,
     uint8_t* __restrict__ q, float* __restrict__ scale) {
@@ -69,7 +79,7 @@ __global__ void __launch_bounds__(kQ1Threads) quant_1x128_kernel(
     for (int off = 8; off > 0; off >>= 1)
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     if (t < total) {
-      const float s = quant_scale(amax);
+      const float s = tile_scale<POW2>(amax);
       const float rs = __frcp_rn(s);
       uint2 out;
       out.x = e4m3x4(div_by_scale(f[0], s, rs), div_by_scale(f[1], s, rs),
@@ -90,6 +100,7 @@ __global__ void __launch_bounds__(kQ1Threads) quant_1x128_kernel(
 // One CTA per block: 256 threads x 8 chunks of 8 bf16 = 128 x 128.
 constexpr int kQ2Threads = 256;
 
+template <bool POW2>
 __global__ void __launch_bounds__(kQ2Threads) quant_128x128_kernel(
     const uint16_t* __restrict__ w, int64_t ldw, int rows, int cols, uint8_t* __restrict__ q,
     float* __restrict__ scale) {
@@ -120,7 +131,7 @@ __global__ void __launch_bounds__(kQ2Threads) quant_128x128_kernel(
   amax = red[0];
 #pragma unroll
   for (int k = 1; k < kQ2Threads / 32; ++k) amax = fmaxf(amax, red[k]);
-  const float s = quant_scale(amax);
+  const float s = tile_scale<POW2>(amax);
   const float rs = __frcp_rn(s);
   if (tid == 0) scale[static_cast<int64_t>(bi) * (cols / 128) + bj] = s;
 #pragma unroll
@@ -176,8 +187,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 }  // namespace moe
 
-extern "C" moe_status fp8_quant_1x128(const uint16_t* x, int64_t ldx, int rows, int cols,
-                                      uint8_t* q, float* scale, moe_stream_t stream) {
+namespace {
+
+moe_status quant_1x128_launch(bool pow2, const uint16_t* x, int64_t ldx, int rows, int cols,
+                              uint8_t* q, float* scale, moe_stream_t stream) {
   using namespace moe;
   if (rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
   if (cols % 128 != 0 || ldx < cols) return MOE_ERR_SHAPE;
@@ -188,14 +201,15 @@ extern "C" moe_status fp8_quant_1x128(const uint16_t* x, int64_t ldx, int rows, 
   const int64_t tiles = static_cast<int64_t>(rows) * (cols / 128);
   const int64_t blocks = (tiles + kQ1TilesPerBlock - 1) / kQ1TilesPerBlock;
   if (blocks > 0x7FFFFFFF) return MOE_ERR_UNSUPPORTED;
-  quant_1x128_kernel<<<static_cast<unsigned>(blocks), kQ1Threads, 0,
-                       static_cast<cudaStream_t>(stream)>>>(x, ldx, rows, cols / 128, q, scale);
+  auto kern = pow2 ? quant_1x128_kernel<true> : quant_1x128_kernel<false>;
+  kern<<<static_cast<unsigned>(blocks), kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, ldx, rows, cols / 128, q, scale);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }
 
-extern "C" moe_status fp8_quant_128x128(const uint16_t* w, int64_t ldw, int rows, int cols,
-                                        uint8_t* q, float* scale, moe_stream_t stream) {
+moe_status quant_128x128_launch(bool pow2, const uint16_t* w, int64_t ldw, int rows, int cols,
+                                uint8_t* q, float* scale, moe_stream_t stream) {
   using namespace moe;
   if (rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
   if (cols % 128 != 0 || ldw < cols) return MOE_ERR_SHAPE;
@@ -206,10 +220,32 @@ extern "C" moe_status fp8_quant_128x128(const uint16_t* w, int64_t ldw, int rows
   const int rb = (rows + 127) / 128;
   if (rb > 65535) return MOE_ERR_UNSUPPORTED;
   dim3 grid(cols / 128, rb);
-  quant_128x128_kernel<<<grid, kQ2Threads, 0, static_cast<cudaStream_t>(stream)>>>(w, ldw, rows,
-                                                                                   cols, q, scale);
+  auto kern = pow2 ? quant_128x128_kernel<true> : quant_128x128_kernel<false>;
+  kern<<<grid, kQ2Threads, 0, static_cast<cudaStream_t>(stream)>>>(w, ldw, rows, cols, q, scale);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status fp8_quant_1x128(const uint16_t* x, int64_t ldx, int rows, int cols,
+                                      uint8_t* q, float* scale, moe_stream_t stream) {
+  return quant_1x128_launch(false, x, ldx, rows, cols, q, scale, stream);
+}
+
+extern "C" moe_status fp8_quant_1x128_pow2(const uint16_t* x, int64_t ldx, int rows, int cols,
+                                           uint8_t* q, float* scale, moe_stream_t stream) {
+  return quant_1x128_launch(true, x, ldx, rows, cols, q, scale, stream);
+}
+
+extern "C" moe_status fp8_quant_128x128(const uint16_t* w, int64_t ldw, int rows, int cols,
+                                        uint8_t* q, float* scale, moe_stream_t stream) {
+  return quant_128x128_launch(false, w, ldw, rows, cols, q, scale, stream);
+}
+
+extern "C" moe_status fp8_quant_128x128_pow2(const uint16_t* w, int64_t ldw, int rows, int cols,
+                                             uint8_t* q, float* scale, moe_stream_t stream) {
+  return quant_128x128_launch(true, w, ldw, rows, cols, q, scale, stream);
 }
 
 extern "C" moe_status swiglu_quant(const float* gu, int rows, int I, uint8_t* h, float* h_scale,

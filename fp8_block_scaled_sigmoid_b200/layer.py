@@ -51,14 +51,16 @@ def max_over_ranks(value: float, device, process_group=None) -> float:
     return float(t.item())
 
 
-def quantise_weight_stack(w_bf16: torch.Tensor, q=None, s=None):
+def quantise_weight_stack(w_bf16: torch.Tensor, q=None, s=None, pow2: bool = False):
     """128x128 block quantisation of a [G][N][K] bf16 stack on the device."""
-    return _abi.fp8_quant_128x128(w_bf16, q, s)
+    return _abi.fp8_quant_128x128(w_bf16, q, s, pow2=pow2)
 
 
-def make_fp8_weights(cfg: MoEConfig, device, chunk: int = 16):
+def make_fp8_weights(cfg: MoEConfig, device, chunk: int = 16, pow2: bool = False):
     """Draw the bf16 expert weights (seeded, per expert) and quantise them on
-    the device a few experts at a time; only the FP8 stacks stay resident."""
+    the device a few experts at a time; only the FP8 stacks stay resident.
+    ``pow2`` rounds the block scales up to powers of two (for a layer built
+    with pow2=True)."""
     G = cfg.E + cfg.n_shared
     w1q = torch.empty(G, 2 * cfg.I, cfg.d, dtype=torch.uint8, device=device)
     w1s = torch.empty(G, 2 * cfg.I // 128, cfg.d // 128, dtype=torch.float32, device=device)
@@ -68,19 +70,25 @@ def make_fp8_weights(cfg: MoEConfig, device, chunk: int = 16):
         e1 = min(G, e0 + chunk)
         w1 = torch.stack([_inputs.draw_w1(cfg, e, device) for e in range(e0, e1)])
         w2 = torch.stack([_inputs.draw_w2(cfg, e, device) for e in range(e0, e1)])
-        _abi.fp8_quant_128x128(w1, w1q[e0:e1], w1s[e0:e1])
-        _abi.fp8_quant_128x128(w2, w2q[e0:e1], w2s[e0:e1])
+        _abi.fp8_quant_128x128(w1, w1q[e0:e1], w1s[e0:e1], pow2=pow2)
+        _abi.fp8_quant_128x128(w2, w2q[e0:e1], w2s[e0:e1], pow2=pow2)
         del w1, w2
     return w1q, w1s, w2q, w2s
 
 
 class MoELayer:
-    """Device buffers and call sequence of one layer for a fixed batch size T."""
+    """Device buffers and call sequence of one layer for a fixed batch size T.
+
+    ``pow2`` selects the power-of-two scale variant: the activations and h are
+    quantised with scales rounded up to powers of two and both expert GEMMs
+    hand the scales to the tensor core (grouped_gemm_fp8_pow2); the weights
+    must come from make_fp8_weights(..., pow2=True)."""
 
     def __init__(self, cfg: MoEConfig, centroids: torch.Tensor, bias: torch.Tensor,
                  w1q, w1s, w2q, w2s, T: int | None = None, process_group=None,
-                 keep_logits: bool = False):
+                 keep_logits: bool = False, pow2: bool = False):
         self.cfg = cfg
+        self.pow2 = pow2
         self.T = cfg.T if T is None else T
         self.dev = centroids.device
         self.centroids = centroids
@@ -123,7 +131,7 @@ class MoELayer:
                        logits_out=self.logits, ws=self.route_ws, dev_err=self.dev_err)
 
     def step_quant(self, u):
-        _abi.fp8_quant_1x128(u, self.Xq[self.pairs:], self.Xs[self.pairs:])
+        _abi.fp8_quant_1x128(u, self.Xq[self.pairs:], self.Xs[self.pairs:], pow2=self.pow2)
 
     def step_permute(self):
         c = self.cfg
@@ -135,14 +143,14 @@ class MoELayer:
         _abi.grouped_gemm_fp8_blockscaled(self.Xq, self.Xs, self.w1q, self.w1s, p["offsets"],
                                           p["tile_group"], p["tile_start"], p["n_tiles"],
                                           self.max_tiles, _abi.EP_SWIGLU_QUANT, self.H, self.Hs,
-                                          dev_err=self.dev_err)
+                                          dev_err=self.dev_err, pow2=self.pow2)
 
     def step_gemm2(self):
         p = self.perm
         _abi.grouped_gemm_fp8_blockscaled(self.H, self.Hs, self.w2q, self.w2s, p["offsets"],
                                           p["tile_group"], p["tile_start"], p["n_tiles"],
                                           self.max_tiles, _abi.EP_F32, self.Y,
-                                          dev_err=self.dev_err)
+                                          dev_err=self.dev_err, pow2=self.pow2)
 
     def step_combine(self, u, out=None):
         P = self.pairs

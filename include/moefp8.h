@@ -63,6 +63,8 @@ typedef enum {
 #define MOE_DEVERR_TIMEOUT 1   /* a bounded wait gave up; results are invalid */
 #define MOE_DEVERR_BAD_TABLE 2 /* segment offsets / tile table inconsistent */
 #define MOE_DEVERR_BAD_INDEX 3 /* an expert index outside [0, E) */
+#define MOE_DEVERR_BAD_SCALE 4 /* a scale that is not a positive power of two reached the
+                                  power-of-two GEMM */
 
 typedef void* moe_stream_t; /* cudaStream_t */
 
@@ -97,6 +99,22 @@ moe_status fp8_quant_1x128(const uint16_t* x, int64_t ldx, int rows, int cols, u
  */
 moe_status fp8_quant_128x128(const uint16_t* w, int64_t ldw, int rows, int cols, uint8_t* q,
                              float* scale, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * fp8_quant_1x128_pow2 / fp8_quant_128x128_pow2 -- the same quantisers with
+ * power-of-two scales.  [ANN] "Low-Precision Storage and Communication": the
+ * activations quantised before the dispatch carry scaling factors that are
+ * integral powers of 2.  Each tile's or block's scale max(amax, 1e-4)/448 is
+ * rounded UP to the next power of two (so nothing saturates and the tile
+ * maximum lands in [224, 448]); x / scale is then exact and q is its E4M3
+ * rounding.  Arguments, layouts, limits and errors as above; the scales are
+ * still written as fp32 values (each an exact power of two, i.e. a UE8M0
+ * exponent), ready for grouped_gemm_fp8_pow2.
+ */
+moe_status fp8_quant_1x128_pow2(const uint16_t* x, int64_t ldx, int rows, int cols, uint8_t* q,
+                                float* scale, moe_stream_t stream);
+moe_status fp8_quant_128x128_pow2(const uint16_t* w, int64_t ldw, int rows, int cols,
+                                  uint8_t* q, float* scale, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * moe_route -- sigmoid router with bias-based, group-limited top-K selection.
@@ -214,6 +232,30 @@ moe_status grouped_gemm_fp8_blockscaled(const uint8_t* A, const float* sa, int64
                                         int max_tiles, int groups, int N, int K,
                                         moe_epilogue ep, void* D, float* d_scale,
                                         int32_t* dev_err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * grouped_gemm_fp8_pow2 -- grouped_gemm_fp8_blockscaled for operands whose
+ * every scale is a power of two (from the _pow2 quantisers).  [ANN] "Low-
+ * Precision Storage and Communication" (power-of-two scaling factors) and
+ * "Suggestions on Hardware Design" / "Support for Tile- and Block-Wise
+ * Quantization" (tensor cores that apply the group scales themselves, with
+ * no copy of partial results to the CUDA cores): each scale's exponent is handed to the tensor core as a
+ * UE8M0 scale factor (tcgen05 kind::mxf8f6f4 block scaling, one exponent
+ * per row per 32-element K slice, the 1x128 / 128x128 scale repeated over
+ * its four slices), and the whole K extent accumulates in the tensor core's
+ * fp32 TMEM accumulator with no promotion step.
+ * Arguments, layouts and limits as in grouped_gemm_fp8_blockscaled; with
+ * MOE_EP_SWIGLU_QUANT the scales of h are rounded up to powers of two as in
+ * fp8_quant_1x128_pow2.  A scale that is not a positive normal power of two
+ * records MOE_DEVERR_BAD_SCALE (its exponent is used as if the mantissa were
+ * zero).
+ */
+moe_status grouped_gemm_fp8_pow2(const uint8_t* A, const float* sa, int64_t a_rows,
+                                 const uint8_t* B, const float* sb, const int32_t* offsets,
+                                 const int32_t* tile_group, const int32_t* tile_start,
+                                 const int32_t* n_tiles, int max_tiles, int groups, int N, int K,
+                                 moe_epilogue ep, void* D, float* d_scale, int32_t* dev_err,
+                                 moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * swiglu_quant -- standalone SwiGLU + 1x128 quantisation of fp32 GEMM output
