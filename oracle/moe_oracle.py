@@ -473,6 +473,8 @@ def moe_layer(u, centroids, bias, w1q, w1s, w2q, w2s, G, M, K, gamma,
     xs = np.concatenate([xs_tok[src_row], xs_tok])
     offs = segment_offsets_with_shared(offsets, T)
     gu = grouped_gemm(xq, xs, w1q, w1s, offs)
+    # the SwiGLU input, cached in FP8 for the backward pass ([ANN] "Low-Precision Activation")
+    guq, gus = quant_1x128_pow2(gu.astype(np.float32)) if pow2 else quant_1x128(gu.astype(np.float32))
     if h_override is None:
         hq, hs = swiglu_quant(gu, I, pow2)
     else:
@@ -482,4 +484,175 @@ def moe_layer(u, centroids, bias, w1q, w1s, w2q, w2s, G, M, K, gamma,
     new_bias = bias_update(counts, T, K, gamma, bias)
     return {"idx": idx, "gate": gate, "route": rinfo, "xq_tok": xq_tok, "xs_tok": xs_tok,
             "counts": counts, "offsets": offs, "src_row": src_row, "dst_of": dst_of,
-            "gu": gu, "hq": hq, "hs": hs, "Y": Y, "out": out, "bias": new_bias}
+            "xq": xq, "xs": xs, "gu": gu, "guq": guq, "gus": gus, "hq": hq, "hs": hs, "Y": Y,
+            "out": out, "bias": new_bias}
+
+
+# ---------------------------------------------------------------------------
+# Backward of the expert FFNs.  [ANN] "Mixed Precision Framework": the three
+# GEMMs of a linear operator -- Fprop, Dgrad (activation gradient) and Wgrad
+# (weight gradient) -- take FP8 inputs and give high-precision outputs; the
+# weight gradients stay in high precision.  "Low-Precision Activation": the
+# SwiGLU input is cached in FP8 and the SwiGLU output is recomputed in the
+# backward pass.  "Low-Precision Communication": the activation gradient
+# before the MoE down-projection is quantised to FP8 with power-of-two
+# scales.  "Support for Transposed GEMM Operations": an operand whose
+# reduction runs over tokens is re-quantised in 128x1 tiles (128 tokens of one
+# channel).
+# Readings (also in the design notes): every gradient quantisation is 1x128
+# along the channels with power-of-two scales (activation gradients are never
+# block-quantised: [INFRA] "V3 FP8" reports divergence for 128x128 Dgrad
+# gradients); a
+# 128x1 operand is quantised from the fp32 value where the backward pass
+# computes it (dy, dgu, the recomputed h) and from the dequantised FP8 cache
+# for x; each expert's token segment is zero-padded to a multiple of 128
+# tokens for its Wgrad; the router's gradient (not an FP8 GEMM) is not part
+# of this path.
+# ---------------------------------------------------------------------------
+def transpose_weights(q, s):
+    """FP8 weight stack [G][N][K] with 128x128 block scales [G][N/128][K/128]
+    -> the transposed stack [G][K][N] and scales [G][K/128][N/128].  Exact:
+    every 128x128 block keeps its own scale."""
+    return (np.ascontiguousarray(np.swapaxes(np.asarray(q), 1, 2)),
+            np.ascontiguousarray(np.swapaxes(np.asarray(s), 1, 2)))
+
+
+def wgrad_segments(offsets):
+    """Column offsets koff [groups+1] of the token-major (transposed) Wgrad
+    operands: segment g's rows, zero-padded to a multiple of 128."""
+    offsets = np.asarray(offsets, np.int64)
+    kpad = [-(-(int(offsets[g + 1]) - int(offsets[g])) // TILE) * TILE
+            for g in range(len(offsets) - 1)]
+    return np.concatenate([[0], np.cumsum(kpad)]).astype(np.int64)
+
+
+def quant_128x1_pow2(m, offsets):
+    """m [rows][C] (fp32 values) in token segments [offsets[g], offsets[g+1]).
+    Each column of each segment is quantised in blocks of 128 tokens (the
+    segment zero-padded to a multiple of 128) with a power-of-two scale.
+    Returns the transposed codes qt uint8 [C][Ktot], scales st fp32
+    [C][Ktot/128] and koff [groups+1] (segment g = columns koff[g]..koff[g+1])."""
+    m = np.asarray(m, np.float32)
+    C = m.shape[1]
+    offsets = np.asarray(offsets, np.int64)
+    koff = wgrad_segments(offsets)
+    qt = np.zeros((C, int(koff[-1])), np.uint8)
+    st = np.zeros((C, int(koff[-1]) // TILE), np.float32)
+    for g in range(len(offsets) - 1):
+        r0, r1 = int(offsets[g]), int(offsets[g + 1])
+        for b in range(0, r1 - r0, TILE):
+            blk = m[r0 + b:min(r1, r0 + b + TILE)]          # up to 128 tokens x C
+            scale = pow2_ceil(_scale_of(np.abs(blk).max(axis=0)))
+            col = int(koff[g]) + b
+            st[:, col // TILE] = scale
+            qt[:, col:col + blk.shape[0]] = e4m3_encode((blk / scale[None, :]).astype(np.float32)).T
+    return qt, st, koff
+
+
+def dequant_rows(qt, st) -> np.ndarray:
+    """Codes [C][Ktot] with one scale per row per 128 columns."""
+    return e4m3_decode(qt) * np.repeat(np.asarray(st, np.float64), TILE, axis=1)
+
+
+def wgrad(at, bt, koff) -> np.ndarray:
+    """Per segment g: dW[g] = At[:, seg g] . Bt[:, seg g]^T (fp64), from two
+    dequantised token-major operands At [Ca][Ktot], Bt [Cb][Ktot]."""
+    G = len(koff) - 1
+    out = np.zeros((G, at.shape[0], bt.shape[0]), np.float64)
+    for g in range(G):
+        k0, k1 = int(koff[g]), int(koff[g + 1])
+        if k1 > k0:
+            out[g] = at[:, k0:k1] @ bt[:, k0:k1].T
+    return out
+
+
+def expert_backward(dout, fwd, w1q, w1s, w2q, w2s, quantize: bool = True):
+    """Gradients of the expert FFNs for the upstream gradient dout [T][d] of
+    the layer output, with the routing of the forward pass ``fwd`` (a
+    moe_layer result).  ``quantize=False`` replaces every FP8 quantisation
+    of the backward pass by the exact value (and uses the exact SwiGLU input
+    and x) -- the plain chain rule, for checking against finite differences.
+    Returns dy, dh, dgu, h, dx (per permuted row), du [T][d] (gradient of the
+    layer input through the experts and the residual), dW1 [G][2I][d],
+    dW2 [G][d][I] (fp64) and the FP8 operands of each GEMM."""
+    dout = np.asarray(dout, np.float32)
+    T, d = dout.shape
+    dst_of, gate, offs = fwd["dst_of"], np.asarray(fwd["gate"], np.float32), fwd["offsets"]
+    K = dst_of.shape[1]
+    P = T * K
+    rows = P + T
+    I = np.asarray(w2q).shape[2]
+    w1 = np.stack([dequant_128x128(q, s) for q, s in zip(w1q, w1s)])
+    w2 = np.stack([dequant_128x128(q, s) for q, s in zip(w2q, w2s)])
+    r = {}
+
+    def seg_gemm(a, w):   # rows of segment g times w[g]^T
+        o = np.zeros((a.shape[0], w.shape[1]), np.float64)
+        for g in range(len(offs) - 1):
+            r0, r1 = int(offs[g]), int(offs[g + 1])
+            if r1 > r0:
+                o[r0:r1] = a[r0:r1] @ w[g].T
+        return o
+
+    # 1. the gradient at every expert output row: gate * dout for a routed
+    #    pair (one fp32 product), dout itself for the shared expert's row
+    dy = np.empty((rows, d), np.float32)
+    for k in range(K):
+        dy[dst_of[:, k]] = gate[:, k:k + 1] * dout
+    dy[P:] = dout
+    r["dy"] = dy
+    if quantize:
+        r["dyq"], r["dys"] = quant_1x128_pow2(dy)
+        dy_in = dequant_1x128(r["dyq"], r["dys"])
+    else:
+        dy_in = dy.astype(np.float64)
+    # 2. Dgrad of the down projection: dh = dy . W2 (the GEMM's B is W2^T)
+    dh = seg_gemm(dy_in, np.swapaxes(w2, 1, 2))
+    r["dh"] = dh
+    # 3. SwiGLU backward on its cached input (gate/up blocks interleaved)
+    gu = dequant_1x128(fwd["guq"], fwd["gus"]) if quantize else np.asarray(fwd["gu"], np.float64)
+    gu = gu.reshape(rows, I // TILE, 2, TILE)
+    g, u = gu[:, :, 0, :], gu[:, :, 1, :]
+    with np.errstate(over="ignore"):
+        sg = 1.0 / (1.0 + np.exp(-g))
+    silu_g = g * sg
+    dsilu = sg * (1.0 + g * (1.0 - sg))
+    dh4 = dh.reshape(rows, I // TILE, TILE)
+    dgu = np.stack([dh4 * u * dsilu, dh4 * silu_g], axis=2).reshape(rows, 2 * I)
+    h = (silu_g * u).reshape(rows, I)
+    r["dgu"], r["h"] = dgu, h
+    dgu32 = dgu.astype(np.float32)
+    if quantize:
+        r["dguq"], r["dgus"] = quant_1x128_pow2(dgu32)
+        dgu_in = dequant_1x128(r["dguq"], r["dgus"])
+    else:
+        dgu_in = dgu
+    # 4. Dgrad of the up projection: dx = dgu . W1
+    dx = seg_gemm(dgu_in, np.swapaxes(w1, 1, 2))
+    r["dx"] = dx
+    # 5. back to the tokens: the residual plus every expert row of the token
+    du = dout.astype(np.float64) + dx[P:]
+    for k in range(K):
+        du += dx[dst_of[:, k]]
+    r["du"] = du
+    # 6. Wgrad: token-major operands, 128x1 tiles
+    x = dequant_1x128(fwd["xq"], fwd["xs"])
+    koff = wgrad_segments(offs)
+    r["koff"] = koff
+    if quantize:
+        r["dyt"] = quant_128x1_pow2(dy, offs)[:2]
+        r["ht"] = quant_128x1_pow2(h.astype(np.float32), offs)[:2]
+        r["dgut"] = quant_128x1_pow2(dgu32, offs)[:2]
+        r["xt"] = quant_128x1_pow2(x.astype(np.float32), offs)[:2]
+        ops = {k: dequant_rows(*r[k]) for k in ("dyt", "ht", "dgut", "xt")}
+    else:
+        def tm(m):   # token-major, zero-padded segments, exact
+            out = np.zeros((m.shape[1], int(koff[-1])), np.float64)
+            for gi in range(len(offs) - 1):
+                r0, r1 = int(offs[gi]), int(offs[gi + 1])
+                out[:, int(koff[gi]):int(koff[gi]) + r1 - r0] = m[r0:r1].T
+            return out
+        ops = {"dyt": tm(dy.astype(np.float64)), "ht": tm(h), "dgut": tm(dgu), "xt": tm(x)}
+    r["dW2"] = wgrad(ops["dyt"], ops["ht"], koff)
+    r["dW1"] = wgrad(ops["dgut"], ops["xt"], koff)
+    return r
