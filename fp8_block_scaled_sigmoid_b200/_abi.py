@@ -45,6 +45,15 @@ _SIGS = {
     "grouped_gemm_fp8_pow2": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
                                    _i, _p, _p, _p, _p]),
     "swiglu_quant": (_i, [_p, _i, _i, _p, _p, _p]),
+    "swiglu_quant_pow2": (_i, [_p, _i, _i, _p, _p, _p]),
+    "fp8_quant_1x128_f32": (_i, [_p, _i64, _i, _i, _i, _p, _p, _p]),
+    "moe_combine_backward": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _p, _p]),
+    "swiglu_backward": (_i, [_p, _p, _p, _i, _i, _p, _p, _p, _p, _p]),
+    "fp8_quant_128x1_pow2": (_i, [_p, _i64, _p, _p, _p, _p, _i, _i, _p, _i64, _p, _p, _p]),
+    "fp8_requant_128x1_pow2": (_i, [_p, _p, _i64, _p, _p, _p, _p, _i, _i, _p, _i64, _p, _p, _p]),
+    "fp8_transpose_128x128": (_i, [_p, _p, _i, _i, _i, _p, _p, _p]),
+    "moe_unpermute_add": (_i, [_p, _p, _p, _i, _i, _i, _p, _p]),
+    "grouped_gemm_fp8_wgrad": (_i, [_p, _p, _p, _p, _i64, _i, _i, _p, _i, _p, _p, _p]),
     "moe_combine": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_bias_update": (_i, [_p, _i, _i64, _i, _f, _p, _p]),
     "moe_seq_balance_loss_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
@@ -60,8 +69,12 @@ _lib = None
 
 # Kernels each entry point launches (for the benchmark's launch count).
 LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant": 1,
+                     "swiglu_quant_pow2": 1,
                      "fp8_quant_1x128_pow2": 1, "fp8_quant_128x128_pow2": 1,
-                     "grouped_gemm_fp8_pow2": 1,
+                     "grouped_gemm_fp8_pow2": 1, "fp8_quant_1x128_f32": 1,
+                     "moe_combine_backward": 1, "swiglu_backward": 1, "fp8_quant_128x1_pow2": 1,
+                     "fp8_requant_128x1_pow2": 1, "fp8_transpose_128x128": 1,
+                     "moe_unpermute_add": 1, "grouped_gemm_fp8_wgrad": 1,
                      "moe_route": 2, "moe_permute": 4, "moe_permute_noalloc": 4,
                      "moe_tile_table": 1,
                      "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1,
@@ -158,13 +171,13 @@ def fp8_quant_128x128(w, q=None, scale=None, stream=None, pow2=False):
     return q, scale
 
 
-def swiglu_quant(gu, I, h=None, h_scale=None, stream=None):
+def swiglu_quant(gu, I, h=None, h_scale=None, stream=None, pow2=False):
     rows = gu.shape[0]
     h = torch.empty(rows, I, dtype=torch.uint8, device=_dev(gu)) if h is None else h
     h_scale = torch.empty(rows, I // 128, dtype=torch.float32, device=_dev(gu)) if h_scale is None else h_scale
-    _count("swiglu_quant")
-    _check(lib().swiglu_quant(_ptr(gu), rows, I, _ptr(h), _ptr(h_scale), _stream(stream)),
-           "swiglu_quant")
+    name = "swiglu_quant_pow2" if pow2 else "swiglu_quant"
+    _count(name)
+    _check(getattr(lib(), name)(_ptr(gu), rows, I, _ptr(h), _ptr(h_scale), _stream(stream)), name)
     return h, h_scale
 
 
@@ -381,3 +394,122 @@ def raise_dev_err(dev_err) -> None:
     v = read_dev_err(dev_err)
     if v != 0:
         raise MoEError(f"device-side error {v}: {DEVERR.get(v, 'unknown')}")
+
+
+# ------------------------------------------------------ backward (experts) ---
+def fp8_quant_1x128_f32(x, pow2=False, q=None, scale=None, stream=None):
+    """x fp32 [rows][cols] -> (q uint8, scale fp32 [rows][cols/128])."""
+    assert x.dtype == torch.float32 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    q = torch.empty(rows, cols, dtype=torch.uint8, device=_dev(x)) if q is None else q
+    scale = torch.empty(rows, cols // 128, dtype=torch.float32, device=_dev(x)) if scale is None else scale
+    _count("fp8_quant_1x128_f32")
+    _check(lib().fp8_quant_1x128_f32(_ptr(x), x.stride(0), rows, cols, int(bool(pow2)), _ptr(q),
+                                     _ptr(scale), _stream(stream)), "fp8_quant_1x128_f32")
+    return q, scale
+
+
+def moe_combine_backward(dout, dst_of, topk_gate, dyq=None, dys=None, dy=None, want_dy=False,
+                         stream=None):
+    """dout fp32 [T][d] -> (dyq uint8 [T*K+T][d], dys [T*K+T][d/128], dy fp32 or None)."""
+    T, d = dout.shape
+    K = dst_of.shape[1]
+    rows = T * K + T
+    dev = _dev(dout)
+    dyq = torch.empty(rows, d, dtype=torch.uint8, device=dev) if dyq is None else dyq
+    dys = torch.empty(rows, d // 128, dtype=torch.float32, device=dev) if dys is None else dys
+    if want_dy and dy is None:
+        dy = torch.empty(rows, d, dtype=torch.float32, device=dev)
+    _count("moe_combine_backward")
+    _check(lib().moe_combine_backward(_ptr(dout), _ptr(dst_of), _ptr(topk_gate), T, K, d,
+                                      _ptr(dyq), _ptr(dys), _ptr(dy), _stream(stream)),
+           "moe_combine_backward")
+    return dyq, dys, dy
+
+
+def swiglu_backward(dh, guq, gus, dguq=None, dgus=None, dgu=None, h=None, want_fp32=False,
+                    stream=None):
+    """dh fp32 [rows][I], cached gu (uint8 [rows][2I], scales [rows][2I/128]) ->
+    (dguq, dgus, dgu fp32 or None, h fp32 or None)."""
+    rows, I = dh.shape
+    dev = _dev(dh)
+    dguq = torch.empty(rows, 2 * I, dtype=torch.uint8, device=dev) if dguq is None else dguq
+    dgus = torch.empty(rows, 2 * I // 128, dtype=torch.float32, device=dev) if dgus is None else dgus
+    if want_fp32:
+        dgu = torch.empty(rows, 2 * I, dtype=torch.float32, device=dev) if dgu is None else dgu
+        h = torch.empty(rows, I, dtype=torch.float32, device=dev) if h is None else h
+    _count("swiglu_backward")
+    _check(lib().swiglu_backward(_ptr(dh), _ptr(guq), _ptr(gus), rows, I, _ptr(dguq), _ptr(dgus),
+                                 _ptr(dgu), _ptr(h), _stream(stream)), "swiglu_backward")
+    return dguq, dgus, dgu, h
+
+
+def wgrad_ld(max_tiles: int) -> int:
+    """Row length (bytes) of a token-major Wgrad operand: 128 per tile, a
+    multiple of 512."""
+    return (128 * max_tiles + 511) // 512 * 512
+
+
+def fp8_quant_128x1_pow2(src, offsets, tile_group, tile_start, n_tiles, max_tiles, src_scale=None,
+                         qt=None, st=None, atoms=None, stream=None):
+    """Token-major 128x1 re-quantisation.  src fp32 [rows][C] (or uint8 with
+    src_scale [rows][C/128], the _requant form) -> (qt uint8 [C][ldt], st fp32
+    [C][ldt/128], atoms uint8 [C/128][ldt/512][512])."""
+    rows, C = src.shape
+    ldt = wgrad_ld(max_tiles)
+    dev = _dev(src)
+    qt = torch.zeros(C, ldt, dtype=torch.uint8, device=dev) if qt is None else qt
+    st = torch.zeros(C, ldt // 128, dtype=torch.float32, device=dev) if st is None else st
+    atoms = torch.zeros(C // 128, ldt // 512, 512, dtype=torch.uint8, device=dev) if atoms is None else atoms
+    if src_scale is None:
+        assert src.dtype == torch.float32
+        _count("fp8_quant_128x1_pow2")
+        _check(lib().fp8_quant_128x1_pow2(_ptr(src), src.stride(0), _ptr(offsets), _ptr(tile_group),
+                                          _ptr(tile_start), _ptr(n_tiles), max_tiles, C, _ptr(qt),
+                                          ldt, _ptr(st), _ptr(atoms), _stream(stream)),
+               "fp8_quant_128x1_pow2")
+    else:
+        assert src.dtype == torch.uint8
+        _count("fp8_requant_128x1_pow2")
+        _check(lib().fp8_requant_128x1_pow2(_ptr(src), _ptr(src_scale), src.stride(0),
+                                            _ptr(offsets), _ptr(tile_group), _ptr(tile_start),
+                                            _ptr(n_tiles), max_tiles, C, _ptr(qt), ldt, _ptr(st),
+                                            _ptr(atoms), _stream(stream)),
+               "fp8_requant_128x1_pow2")
+    return qt, st, atoms
+
+
+def fp8_transpose_128x128(q, scale, qt=None, scale_t=None, stream=None):
+    """[G][N][K] FP8 weights and [G][N/128][K/128] scales -> [G][K][N], [G][K/128][N/128]."""
+    G, N, K = q.shape
+    dev = _dev(q)
+    qt = torch.empty(G, K, N, dtype=torch.uint8, device=dev) if qt is None else qt
+    scale_t = torch.empty(G, K // 128, N // 128, dtype=torch.float32, device=dev) if scale_t is None else scale_t
+    _count("fp8_transpose_128x128")
+    _check(lib().fp8_transpose_128x128(_ptr(q), _ptr(scale), G, N, K, _ptr(qt), _ptr(scale_t),
+                                       _stream(stream)), "fp8_transpose_128x128")
+    return qt, scale_t
+
+
+def moe_unpermute_add(dx, dst_of, dout, du=None, stream=None):
+    """du[t] = dout[t] + dx[T*K + t] + sum_k dx[dst_of[t][k]]."""
+    T, d = dout.shape
+    K = dst_of.shape[1]
+    du = torch.empty(T, d, dtype=torch.float32, device=_dev(dout)) if du is None else du
+    _count("moe_unpermute_add")
+    _check(lib().moe_unpermute_add(_ptr(dx), _ptr(dst_of), _ptr(dout), T, K, d, _ptr(du),
+                                   _stream(stream)), "moe_unpermute_add")
+    return du
+
+
+def grouped_gemm_fp8_wgrad(At, a_atoms, Bt, b_atoms, tile_start, groups, dW=None, dev_err=None,
+                           stream=None):
+    """At uint8 [Ma][ldt], Bt uint8 [Nb][ldt] (token-major) -> dW fp32 [groups][Ma][Nb]."""
+    Ma, ldt = At.shape
+    Nb = Bt.shape[0]
+    dW = torch.empty(groups, Ma, Nb, dtype=torch.float32, device=_dev(At)) if dW is None else dW
+    _count("grouped_gemm_fp8_wgrad")
+    _check(lib().grouped_gemm_fp8_wgrad(_ptr(At), _ptr(a_atoms), _ptr(Bt), _ptr(b_atoms), ldt, Ma,
+                                        Nb, _ptr(tile_start), groups, _ptr(dW), _ptr(dev_err),
+                                        _stream(stream)), "grouped_gemm_fp8_wgrad")
+    return dW

@@ -745,6 +745,192 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pow2_kernel(
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+
+// ====================================================== Wgrad (K-grouped) GEMM
+// dW[g] = At[:, segment g] . Bt[:, segment g]^T for the token-major operands
+// of the weight gradients ("Support for Transposed GEMM Operations": 128x1
+// tiles, one power-of-two scale per channel row per 128 tokens).  Here the
+// groups split K, not M: group g owns the 128-token blocks
+// tile_start[g] .. tile_start[g+1] of both operands and a full Ma x Nb
+// output.  Both operands carry per-row exponents, which the block-scaled MMA
+// takes as they are (B's 256 rows per tile have 256 exponents).  The
+// exponents come pre-arranged in 512-byte atoms (channel block cb, token
+// blocks 4a..4a+3: byte 16 r + 4 j + b = row 32 j + r, block 4a + b), so the
+// producer thread moves them with three bulk copies per stage and no
+// scale-factor warps run.  A group without tokens writes a zero gradient.
+struct WgradArgs {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const int32_t* tile_start;
+  int64_t atoms_per_row;  // ldt / 512
+  int groups, Ma, Nb;
+  float* D;
+  int32_t* dev_err;
+};
+
+struct WItem {
+  int e, m, n, k0, kb;
+};
+
+__device__ __forceinline__ WItem decode_wgrad(int w, const WgradArgs& a) {
+  const int mT = a.Ma / kBM, nN = a.Nb / kBN;
+  WItem it;
+  it.e = w / (mT * nN);
+  const int rem = w - it.e * mT * nN;
+  it.n = rem / mT;
+  it.m = rem - it.n * mT;
+  it.k0 = __ldg(a.tile_start + it.e);
+  it.kb = __ldg(a.tile_start + it.e + 1) - it.k0;
+  if (it.kb < 0) {
+    set_dev_err(a.dev_err, MOE_DEVERR_BAD_TABLE);
+    it.kb = 0;
+  }
+  return it;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_wgrad_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const WgradArgs args) {
+  constexpr int kA = kBM * kBK, kB = kBN * kBK;
+  constexpr int kStage = kA + kB;
+  constexpr int kStages = kStagesMx;
+  constexpr int kSfBytes = kStages * kSfSlot;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sf = base + kRingBytes;
+  const Ctl c = carve<kStages>(base, kRingBytes + kSfBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = args.groups * (args.Ma / kBM) * (args.Nb / kBN);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], 1);
+    }
+    mbar_init(&c.tfull[0], 1);
+    mbar_init(&c.tempty[0], kEpiThreads / 32);
+    mbar_init(c.done, 1);
+    mbar_init(&c.xbar[0], kEpiThreads);
+    mbar_init(&c.xbar[1], kEpiThreads);
+    *c.abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(c.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *c.tmem_slot;
+  volatile int* abort_v = c.abort_flag;
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------- TMA + exponent atoms
+      int it = 0;
+      bool live = true;
+      for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
+        const WItem t = decode_wgrad(w, args);
+        for (int kb = 0; kb < t.kb; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&c.empty[s], ((it / kStages) & 1) ^ 1, abort_v, args.dev_err)) {
+            live = false;
+            break;
+          }
+          uint8_t* sA = base + s * kStage;
+          uint8_t* sfs = sf + s * kSfSlot;
+          const int kk = t.k0 + kb;
+          const int64_t atom = kk >> 2;
+          mbar_arrive_expect_tx(&c.full[s], kStage + 3 * 512);
+          tma_load_2d(sA, &tmA, &c.full[s], kk * kBK, t.m * kBM);
+          tma_load_2d(sA + kA, &tmB, &c.full[s], kk * kBK, t.n * kBN);
+          bulk_load(sfs, args.sfa + (t.m * args.atoms_per_row + atom) * 512, 512, &c.full[s]);
+          bulk_load(sfs + 512, args.sfb + ((2 * t.n) * args.atoms_per_row + atom) * 512, 512,
+                    &c.full[s]);
+          bulk_load(sfs + 1024, args.sfb + ((2 * t.n + 1) * args.atoms_per_row + atom) * 512, 512,
+                    &c.full[s]);
+        }
+      }
+      const int first = it > kStages ? it - kStages : 0;
+      for (int i = first; i < it; ++i)
+        mbar_wait(&c.full[i % kStages], (i / kStages) & 1, nullptr, args.dev_err);
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------- MMA issuer
+      const uint32_t t_sfa = tmem + kTmemSfa, t_sfb = tmem + kTmemSfb;
+      const uint32_t sf0 = smem_u32(sf);
+      int it = 0, tit = 0;
+      bool live = true;
+      for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
+        const WItem t = decode_wgrad(w, args);
+        if (t.kb == 0) continue;
+        if (!mbar_wait(&c.tempty[0], (tit & 1) ^ 1, abort_v, args.dev_err)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < t.kb; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&c.full[s], (it / kStages) & 1, abort_v, args.dev_err)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfs = sf0 + s * kSfSlot;
+          tmem_cp_32x128b_x4(t_sfa, smem_desc_interleave(sfs, 128));
+          tmem_cp_32x128b_x4(t_sfb, smem_desc_interleave(sfs + 512, 128));
+          tmem_cp_32x128b_x4(t_sfb + 4, smem_desc_interleave(sfs + 1024, 128));
+          const uint32_t sA = smem_u32(base + s * kStage);
+          const uint64_t ad = smem_desc_sw128(sA);
+          const uint64_t bd = smem_desc_sw128(sA + kA);
+          const uint32_t sid = static_cast<uint32_t>((t.k0 + kb) & 3);
+          const uint32_t idesc = instr_desc_mx(kBM, kBN, sid);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_mxf8f6f4(tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u,
+                         t_sfa | (sid << 30), t_sfb | (sid << 30));
+          mma_commit(&c.empty[s]);
+        }
+        if (!live) break;
+        mma_commit(&c.tfull[0]);
+        ++tit;
+      }
+      mma_commit(c.done);
+      mbar_wait(c.done, 0, nullptr, args.dev_err);
+    }
+    __syncwarp();
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
+    GemmArgs ga{};
+    ga.D = args.D;
+    int tit = 0, xtile = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      const WItem it = decode_wgrad(w, args);
+      Work t;
+      t.e = it.e;
+      t.n_idx = it.n;
+      t.row0 = it.e * args.Ma + it.m * kBM;  // row of dW viewed as [groups * Ma][Nb]
+      t.rows = kBM;
+      t.ok = true;
+      if (it.kb == 0) {
+        float2 acc[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
+        write_tile<MOE_EP_F32, true>(ga, t, acc, warp, lane, args.Nb, xtile, c.xbar, c.amax_x,
+                                     abort_v);
+        continue;
+      }
+      if (!epilogue_mx_tile<MOE_EP_F32>(ga, t, tmem, warp, lane, args.Nb, tit, xtile,
+                                        &c.tfull[0], &c.tempty[0], c.xbar, c.amax_x, abort_v))
+        break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
 template <int EP>
 const void* kernel_ptr() {
   return reinterpret_cast<const void*>(gemm1sm_kernel<EP, MOE_GEMM_SK>);
@@ -846,4 +1032,52 @@ extern "C" moe_status grouped_gemm_fp8_pow2(
     float* d_scale, int32_t* dev_err, moe_stream_t stream) {
   return gemm_launch(true, A, sa, a_rows, B, sb, offsets, tile_group, tile_start, n_tiles,
                      max_tiles, groups, N, K, ep, D, d_scale, dev_err, stream);
+}
+
+extern "C" moe_status grouped_gemm_fp8_wgrad(const uint8_t* At, const uint8_t* sfa_atoms,
+                                             const uint8_t* Bt, const uint8_t* sfb_atoms,
+                                             int64_t ldt, int Ma, int Nb,
+                                             const int32_t* tile_start, int groups, float* dW,
+                                             int32_t* dev_err, moe_stream_t stream) {
+  using namespace moe;
+  if (ldt < 0 || Ma < 0 || Nb < 0 || groups < 0) return MOE_ERR_INVALID_ARG;
+  if (Ma % kBM != 0 || Nb % kBN != 0 || ldt % 512 != 0) return MOE_ERR_SHAPE;
+  if (groups == 0 || Ma == 0 || Nb == 0) return MOE_OK;
+  if (!At || !sfa_atoms || !Bt || !sfb_atoms || !tile_start || !dW) return MOE_ERR_INVALID_ARG;
+  if (ldt == 0) return MOE_ERR_SHAPE;
+  if (!aligned16(At) || !aligned16(Bt) || !aligned16(sfa_atoms) || !aligned16(sfb_atoms) ||
+      !aligned16(dW))
+    return MOE_ERR_ALIGN;
+  if (static_cast<int64_t>(groups) * Ma > 0x7FFFFFFF || ldt / kBK > 0x7FFFFFFF / kBK)
+    return MOE_ERR_UNSUPPORTED;
+  const int64_t items = static_cast<int64_t>(groups) * (Ma / kBM) * (Nb / kBN);
+  if (items > 0x7FFFFFFF) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap tmA, tmB;
+  if (!moe_make_tmap_2d(&tmA, At, CU_TENSOR_MAP_DATA_TYPE_UINT8, ldt, Ma, ldt, kBK, kBM, kBK) ||
+      !moe_make_tmap_2d(&tmB, Bt, CU_TENSOR_MAP_DATA_TYPE_UINT8, ldt, Nb, ldt, kBK, kBN, kBK))
+    return MOE_ERR_CUDA;
+  WgradArgs a;
+  a.sfa = sfa_atoms;
+  a.sfb = sfb_atoms;
+  a.tile_start = tile_start;
+  a.atoms_per_row = ldt / 512;
+  a.groups = groups;
+  a.Ma = Ma;
+  a.Nb = Nb;
+  a.D = dW;
+  a.dev_err = dev_err;
+  static int configured = 0;
+  if (!configured) {
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(gemm_wgrad_kernel),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemMxBytes)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    configured = 1;
+  }
+  const int ctas = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(moe_num_sms(), items)));
+  void* kargs[3] = {&tmA, &tmB, &a};
+  if (cudaLaunchKernel(reinterpret_cast<const void*>(gemm_wgrad_kernel), dim3(ctas), dim3(kThreads),
+                       kargs, kSmemMxBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
 }

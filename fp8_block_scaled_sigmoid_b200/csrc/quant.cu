@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kQ2Threads) quant_128x128_kernel(
 // One warp per 128-wide output tile: lane l takes gate/up elements 4l..4l+3.
 constexpr int kSwThreads = 256;
 
+template <bool POW2>
 __global__ void __launch_bounds__(kSwThreads) swiglu_quant_kernel(
     const float* __restrict__ gu, int rows, int I, uint8_t* __restrict__ h,
     float* __restrict__ h_scale) {
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(kSwThreads) swiglu_quant_kernel(
   float amax = fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3])));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float s = quant_scale(amax);
+  const float s = tile_scale<POW2>(amax);
   const float rs = __frcp_rn(s);
   const uint32_t packed = e4m3x4(div_by_scale(hv[0], s, rs), div_by_scale(hv[1], s, rs),
                                  div_by_scale(hv[2], s, rs), div_by_scale(hv[3], s, rs));
@@ -248,8 +249,9 @@ extern "C" moe_status fp8_quant_128x128_pow2(const uint16_t* w, int64_t ldw, int
   return quant_128x128_launch(true, w, ldw, rows, cols, q, scale, stream);
 }
 
-extern "C" moe_status swiglu_quant(const float* gu, int rows, int I, uint8_t* h, float* h_scale,
-                                   moe_stream_t stream) {
+namespace {
+moe_status swiglu_quant_launch(bool pow2, const float* gu, int rows, int I, uint8_t* h,
+                               float* h_scale, moe_stream_t stream) {
   using namespace moe;
   if (rows < 0 || I < 0) return MOE_ERR_INVALID_ARG;
   if (I % 128 != 0) return MOE_ERR_SHAPE;
@@ -261,8 +263,20 @@ extern "C" moe_status swiglu_quant(const float* gu, int rows, int I, uint8_t* h,
   const int64_t tiles = static_cast<int64_t>(rows) * (I / 128);
   const int64_t blocks = (tiles + (kSwThreads / 32) - 1) / (kSwThreads / 32);
   if (blocks > 0x7FFFFFFF) return MOE_ERR_UNSUPPORTED;
-  swiglu_quant_kernel<<<static_cast<unsigned>(blocks), kSwThreads, 0,
-                        static_cast<cudaStream_t>(stream)>>>(gu, rows, I, h, h_scale);
+  auto kern = pow2 ? swiglu_quant_kernel<true> : swiglu_quant_kernel<false>;
+  kern<<<static_cast<unsigned>(blocks), kSwThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      gu, rows, I, h, h_scale);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
+}
+}  // namespace
+
+extern "C" moe_status swiglu_quant(const float* gu, int rows, int I, uint8_t* h, float* h_scale,
+                                   moe_stream_t stream) {
+  return swiglu_quant_launch(false, gu, rows, I, h, h_scale, stream);
+}
+
+extern "C" moe_status swiglu_quant_pow2(const float* gu, int rows, int I, uint8_t* h,
+                                        float* h_scale, moe_stream_t stream) {
+  return swiglu_quant_launch(true, gu, rows, I, h, h_scale, stream);
 }

@@ -178,6 +178,83 @@ class MoELayer:
             self.step_bias_update()
         return out
 
+    # -- training: forward with the SwiGLU input cached, and the backward ---
+    def forward_train(self, u: torch.Tensor, update_bias: bool = True) -> torch.Tensor:
+        """forward() that also caches what the backward needs: the SwiGLU
+        input gu in FP8 (1x128 tiles; "Low-Precision Activation"), besides the
+        FP8 expert inputs Xq and the routing that forward() keeps anyway.
+        GEMM 1 writes gu in fp32, which is quantised for the cache and
+        through SwiGLU for h."""
+        assert u.shape == (self.T, self.cfg.d) and u.dtype == torch.bfloat16
+        c = self.cfg
+        rows = self.pairs + self.T
+        if getattr(self, "GU", None) is None:
+            dev = self.dev
+            self.GU = torch.empty(rows, 2 * c.I, dtype=torch.float32, device=dev)
+            self.GUq = torch.empty(rows, 2 * c.I, dtype=torch.uint8, device=dev)
+            self.GUs = torch.empty(rows, 2 * c.I // 128, dtype=torch.float32, device=dev)
+        self.step_route(u)
+        self.step_quant(u)
+        self.step_permute()
+        p = self.perm
+        _abi.grouped_gemm_fp8_blockscaled(self.Xq, self.Xs, self.w1q, self.w1s, p["offsets"],
+                                          p["tile_group"], p["tile_start"], p["n_tiles"],
+                                          self.max_tiles, _abi.EP_F32, self.GU,
+                                          dev_err=self.dev_err, pow2=self.pow2)
+        _abi.fp8_quant_1x128_f32(self.GU, self.pow2, self.GUq, self.GUs)
+        _abi.swiglu_quant(self.GU, c.I, self.H, self.Hs, pow2=self.pow2)
+        self.step_gemm2()
+        self.step_combine(u, self.out)
+        if update_bias:
+            self.step_bias_update()
+        return self.out
+
+    def transposed_weights(self):
+        """The Dgrad GEMMs' B operands: W1^T [G][d][2I] and W2^T [G][I][d]
+        with their block scales (made once per weight version)."""
+        if getattr(self, "_wt", None) is None:
+            w1t, w1ts = _abi.fp8_transpose_128x128(self.w1q, self.w1s)
+            w2t, w2ts = _abi.fp8_transpose_128x128(self.w2q, self.w2s)
+            self._wt = (w1t, w1ts, w2t, w2ts)
+        return self._wt
+
+    def backward(self, dout: torch.Tensor, weight_grads: bool = True) -> dict:
+        """Gradients of the expert FFNs for the upstream gradient dout (fp32
+        [T][d]) of the last forward_train: du (the layer input's gradient
+        through the residual and the experts; the router's share is not
+        included), and with weight_grads dW1 [G][2I][d], dW2 [G][d][I].
+        Dgrad: dy (1x128 FP8) . W2 -> dh; SwiGLU backward on the cached FP8
+        gu -> dgu (1x128 FP8); dgu . W1 -> dx; un-permute.  Wgrad: the
+        token-major 128x1 operands dy^T, h^T (recomputed), dgu^T, x^T through
+        grouped_gemm_fp8_wgrad."""
+        c = self.cfg
+        p = self.perm
+        d, I = c.d, c.I
+        w1t, w1ts, w2t, w2ts = self.transposed_weights()
+        dyq, dys, dy = _abi.moe_combine_backward(dout, p["dst_of"], self.gate, want_dy=weight_grads)
+        dh = _abi.grouped_gemm_fp8_blockscaled(dyq, dys, w2t, w2ts, p["offsets"], p["tile_group"],
+                                               p["tile_start"], p["n_tiles"], self.max_tiles,
+                                               _abi.EP_F32, dev_err=self.dev_err, pow2=self.pow2)
+        dguq, dgus, dgu, h = _abi.swiglu_backward(dh, self.GUq, self.GUs, want_fp32=weight_grads)
+        dx = _abi.grouped_gemm_fp8_blockscaled(dguq, dgus, w1t, w1ts, p["offsets"], p["tile_group"],
+                                               p["tile_start"], p["n_tiles"], self.max_tiles,
+                                               _abi.EP_F32, dev_err=self.dev_err, pow2=self.pow2)
+        du = _abi.moe_unpermute_add(dx, p["dst_of"], dout)
+        r = {"du": du, "dyq": dyq, "dys": dys, "dh": dh, "dguq": dguq, "dgus": dgus, "dx": dx}
+        if weight_grads:
+            G = c.E + c.n_shared
+            tabs = (p["offsets"], p["tile_group"], p["tile_start"], p["n_tiles"], self.max_tiles)
+            dyt = _abi.fp8_quant_128x1_pow2(dy, *tabs)
+            ht = _abi.fp8_quant_128x1_pow2(h, *tabs)
+            dgut = _abi.fp8_quant_128x1_pow2(dgu, *tabs)
+            xt = _abi.fp8_quant_128x1_pow2(self.Xq, *tabs, src_scale=self.Xs)
+            r["dW2"] = _abi.grouped_gemm_fp8_wgrad(dyt[0], dyt[2], ht[0], ht[2], p["tile_start"], G,
+                                                   dev_err=self.dev_err)
+            r["dW1"] = _abi.grouped_gemm_fp8_wgrad(dgut[0], dgut[2], xt[0], xt[2], p["tile_start"], G,
+                                                   dev_err=self.dev_err)
+            r.update({"dy": dy, "dgu": dgu, "h": h, "dyt": dyt, "ht": ht, "dgut": dgut, "xt": xt})
+        return r
+
     def forward_host(self, u_host: torch.Tensor, out_host: torch.Tensor,
                      update_bias: bool = True) -> torch.Tensor:
         """End-to-end call with host buffers: copy u in (pinned host ->

@@ -257,6 +257,101 @@ moe_status grouped_gemm_fp8_pow2(const uint8_t* A, const float* sa, int64_t a_ro
                                  moe_epilogue ep, void* D, float* d_scale, int32_t* dev_err,
                                  moe_stream_t stream);
 
+/* ===========================================================================
+ * Backward of the expert FFNs.  [ANN] "Mixed Precision Framework": Fprop,
+ * Dgrad (activation gradient) and Wgrad (weight gradient) GEMMs all take FP8
+ * inputs; weight gradients stay fp32.  "Low-Precision Activation": the
+ * SwiGLU input is cached in FP8 and the SwiGLU output recomputed.  "Low-
+ * Precision Communication": the gradient before the down projection is
+ * quantised to FP8 with power-of-two scales.  "Support for Transposed GEMM
+ * Operations": an operand reduced over tokens is re-quantised in 128x1 tiles.
+ * Every gradient quantisation here is 1x128 along channels (or 128x1 along
+ * tokens for Wgrad) with power-of-two scales.  The Dgrad GEMMs are
+ * grouped_gemm_fp8_blockscaled / grouped_gemm_fp8_pow2 with A = the
+ * quantised gradient and B = the transposed weights (fp8_transpose_128x128).
+ * =========================================================================== */
+
+/* fp8_quant_1x128_f32 -- 1x128 quantisation of fp32 rows (the SwiGLU input
+ * cache); pow2 != 0 rounds each scale up to a power of two.
+ *   x fp32 [rows][ldx];  q E4M3 [rows][cols];  scale fp32 [rows][cols/128]
+ * Limits: cols % 128 == 0, ldx % 4 == 0. */
+moe_status fp8_quant_1x128_f32(const float* x, int64_t ldx, int rows, int cols, int pow2,
+                               uint8_t* q, float* scale, moe_stream_t stream);
+
+/* moe_combine_backward -- the gradient at every expert output row of the
+ * permuted layout (the backward of eq. (12)): dy[dst_of[t][k]] = fl32(gate
+ * [t][k] * dout[t]), dy[T*K + t] = dout[t], quantised 1x128 with power-of-two
+ * scales.  Rows with dst_of < 0 are skipped.
+ *   dout fp32 [T][d];  dyq E4M3 [T*K+T][d];  dys fp32 [T*K+T][d/128]
+ *   dy fp32 [T*K+T][d] or NULL (the unquantised values, for the Wgrad operand)
+ * Limits: d % 128 == 0, K <= 32. */
+moe_status moe_combine_backward(const float* dout, const int32_t* dst_of, const float* topk_gate,
+                                int T, int K, int d, uint8_t* dyq, float* dys, float* dy,
+                                moe_stream_t stream);
+
+/* swiglu_backward -- from dh [rows][I] (Dgrad of the down projection) and the
+ * cached SwiGLU input gu (E4M3 [rows][2I], 1x128 scales [rows][2I/128], gate/
+ * up blocks interleaved as in the forward): sigma = 1/(1+e^-g), dg = dh * u *
+ * sigma (1 + g (1 - sigma)), du = dh * g sigma, in fp32; dgu (same
+ * interleaving) quantised 1x128 with power-of-two scales.
+ *   dguq E4M3 [rows][2I], dgus fp32 [rows][2I/128]
+ *   dgu fp32 [rows][2I] or NULL;  h fp32 [rows][I] or NULL (the recomputed
+ *   SwiGLU output g sigma u, for the Wgrad of the down projection)
+ * Limits: I % 128 == 0. */
+moe_status swiglu_backward(const float* dh, const uint8_t* guq, const float* gus, int rows, int I,
+                           uint8_t* dguq, float* dgus, float* dgu, float* h, moe_stream_t stream);
+
+/* fp8_quant_128x1_pow2 / fp8_requant_128x1_pow2 -- token-major (transposed)
+ * re-quantisation for Wgrad.  For every 128-token tile i of the segment table
+ * (tile_group, tile_start, n_tiles as written by moe_permute or
+ * moe_tile_table), rows offsets[g] + 128 (i - tile_start[g]) .. (zero past
+ * the segment's end): qt[c][128 i + r] = E4M3(src[row r][c] / st[c][i]), st
+ * = the power-of-two scale of the 128 tokens of channel c.  The _requant form
+ * reads an FP8 source with 1x128 scales (the cached x) and dequantises it
+ * first.
+ *   src fp32 [rows][ld_src]  (or q E4M3 [rows][ld_src], scale [rows][ld_src/128])
+ *   qt E4M3 [C][ldt], st fp32 [C][ldt/128], ldt >= 128 * max_tiles
+ *   sf_atoms NULL or [C/128][ldt/512][512] bytes (ldt % 512 == 0): the
+ *   exponents (UE8M0) of st arranged for grouped_gemm_fp8_wgrad (byte
+ *   16 r + 4 j + b of atom (cb, a) = channel 128 cb + 32 j + r, tile 4a + b)
+ * Limits: C % 128 == 0. */
+moe_status fp8_quant_128x1_pow2(const float* src, int64_t ld_src, const int32_t* offsets,
+                                const int32_t* tile_group, const int32_t* tile_start,
+                                const int32_t* n_tiles, int max_tiles, int C, uint8_t* qt,
+                                int64_t ldt, float* st, uint8_t* sf_atoms, moe_stream_t stream);
+moe_status fp8_requant_128x1_pow2(const uint8_t* q, const float* scale, int64_t ld_src,
+                                  const int32_t* offsets, const int32_t* tile_group,
+                                  const int32_t* tile_start, const int32_t* n_tiles,
+                                  int max_tiles, int C, uint8_t* qt, int64_t ldt, float* st,
+                                  uint8_t* sf_atoms, moe_stream_t stream);
+
+/* fp8_transpose_128x128 -- FP8 weight stack [groups][N][K] with 128x128
+ * scales [groups][N/128][K/128] -> [groups][K][N] and [groups][K/128][N/128]
+ * (exact: every block keeps its scale); the B operand of a Dgrad GEMM.
+ * Limits: N % 128 == 0, K % 128 == 0. */
+moe_status fp8_transpose_128x128(const uint8_t* q, const float* scale, int groups, int N, int K,
+                                 uint8_t* qt, float* scale_t, moe_stream_t stream);
+
+/* moe_unpermute_add -- du[t] = dout[t] + dx[T*K + t] + sum_k dx[dst_of[t][k]]
+ * (fp32, added in that order): the gradient of the layer input through the
+ * residual and the experts (the router's share is not included).
+ *   dx fp32 [T*K+T][d] (Dgrad of the up projection by permuted row) */
+moe_status moe_unpermute_add(const float* dx, const int32_t* dst_of, const float* dout, int T,
+                             int K, int d, float* du, moe_stream_t stream);
+
+/* grouped_gemm_fp8_wgrad -- dW[g] = At[:, tiles of g] . Bt[:, tiles of g]^T,
+ * fp32 [groups][Ma][Nb], for every group g with tiles tile_start[g] ..
+ * tile_start[g+1] (128 tokens each) of both token-major operands; a group
+ * without tiles gets a zero gradient.  The exponents of both operands (one
+ * per row per 128 tokens, from fp8_quant_128x1_pow2's sf_atoms) are applied
+ * by the tensor core (block-scaled tcgen05 MMA), fp32 accumulation in TMEM.
+ *   At E4M3 [Ma][ldt], Bt E4M3 [Nb][ldt]; sfa_atoms / sfb_atoms as above
+ * Limits: Ma % 128 == 0, Nb % 256 == 0, ldt % 512 == 0. */
+moe_status grouped_gemm_fp8_wgrad(const uint8_t* At, const uint8_t* sfa_atoms, const uint8_t* Bt,
+                                  const uint8_t* sfb_atoms, int64_t ldt, int Ma, int Nb,
+                                  const int32_t* tile_start, int groups, float* dW,
+                                  int32_t* dev_err, moe_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * swiglu_quant -- standalone SwiGLU + 1x128 quantisation of fp32 GEMM output
  * in the block-interleaved layout above; bit-identical to the fused epilogue
@@ -265,6 +360,11 @@ moe_status grouped_gemm_fp8_pow2(const uint8_t* A, const float* sa, int64_t a_ro
  */
 moe_status swiglu_quant(const float* gu, int rows, int I, uint8_t* h, float* h_scale,
                         moe_stream_t stream);
+/* swiglu_quant_pow2 -- the same with the scales of h rounded up to powers of
+ * two (bit-identical to grouped_gemm_fp8_pow2's fused epilogue on identical
+ * input). */
+moe_status swiglu_quant_pow2(const float* gu, int rows, int I, uint8_t* h, float* h_scale,
+                             moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * moe_combine -- [ANN] eq. (12): out_t = u_t + FFN_shared(u_t)

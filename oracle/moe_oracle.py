@@ -566,6 +566,36 @@ def wgrad(at, bt, koff) -> np.ndarray:
     return out
 
 
+def swiglu_backward(dh, gu, I: int):
+    """SwiGLU backward ([ANN] SwiGLU operator notes, Swish beta = 1): for the
+    block-interleaved input gu [rows][2I] (gate blocks, then the matching up
+    blocks) and dh = dL/dh [rows][I]: sigma = 1/(1+e^-g), dg = dh u sigma
+    (1 + g (1 - sigma)), du = dh g sigma.  Returns dgu [rows][2I] (same
+    interleaving) and the recomputed h = g sigma u [rows][I], fp64."""
+    gu = np.asarray(gu, np.float64)
+    rows = gu.shape[0]
+    blk = gu.reshape(rows, I // TILE, 2, TILE)
+    g, u = blk[:, :, 0, :], blk[:, :, 1, :]
+    with np.errstate(over="ignore"):
+        sg = 1.0 / (1.0 + np.exp(-g))
+    silu_g = g * sg
+    dsilu = sg * (1.0 + g * (1.0 - sg))
+    dh4 = np.asarray(dh, np.float64).reshape(rows, I // TILE, TILE)
+    dgu = np.stack([dh4 * u * dsilu, dh4 * silu_g], axis=2).reshape(rows, 2 * I)
+    return dgu, (silu_g * u).reshape(rows, I)
+
+
+def unpermute_add(dx, dst_of, dout) -> np.ndarray:
+    """du_t = dout_t + dx[T*K + t] + sum_k dx[dst_of[t][k]] (fp64)."""
+    dst_of = np.asarray(dst_of)
+    T, K = dst_of.shape
+    dx = np.asarray(dx, np.float64)
+    du = np.asarray(dout, np.float64) + dx[T * K:T * K + T]
+    for k in range(K):
+        du = du + dx[dst_of[:, k]]
+    return du
+
+
 def expert_backward(dout, fwd, w1q, w1s, w2q, w2s, quantize: bool = True):
     """Gradients of the expert FFNs for the upstream gradient dout [T][d] of
     the layer output, with the routing of the forward pass ``fwd`` (a
@@ -611,15 +641,7 @@ def expert_backward(dout, fwd, w1q, w1s, w2q, w2s, quantize: bool = True):
     r["dh"] = dh
     # 3. SwiGLU backward on its cached input (gate/up blocks interleaved)
     gu = dequant_1x128(fwd["guq"], fwd["gus"]) if quantize else np.asarray(fwd["gu"], np.float64)
-    gu = gu.reshape(rows, I // TILE, 2, TILE)
-    g, u = gu[:, :, 0, :], gu[:, :, 1, :]
-    with np.errstate(over="ignore"):
-        sg = 1.0 / (1.0 + np.exp(-g))
-    silu_g = g * sg
-    dsilu = sg * (1.0 + g * (1.0 - sg))
-    dh4 = dh.reshape(rows, I // TILE, TILE)
-    dgu = np.stack([dh4 * u * dsilu, dh4 * silu_g], axis=2).reshape(rows, 2 * I)
-    h = (silu_g * u).reshape(rows, I)
+    dgu, h = swiglu_backward(dh, gu, I)
     r["dgu"], r["h"] = dgu, h
     dgu32 = dgu.astype(np.float32)
     if quantize:
@@ -631,10 +653,7 @@ def expert_backward(dout, fwd, w1q, w1s, w2q, w2s, quantize: bool = True):
     dx = seg_gemm(dgu_in, np.swapaxes(w1, 1, 2))
     r["dx"] = dx
     # 5. back to the tokens: the residual plus every expert row of the token
-    du = dout.astype(np.float64) + dx[P:]
-    for k in range(K):
-        du += dx[dst_of[:, k]]
-    r["du"] = du
+    r["du"] = unpermute_add(dx, dst_of, dout)
     # 6. Wgrad: token-major operands, 128x1 tiles
     x = dequant_1x128(fwd["xq"], fwd["xs"])
     koff = wgrad_segments(offs)
