@@ -606,6 +606,104 @@ def run_gemm(args):
         "clocks": clocks}), flush=True)
 
 
+def run_backward(args):
+    """Backward of the expert FFNs at the configured layer size (one GPU):
+    forward_train once per step (untimed), then the timed backward with the
+    weight gradients.  Tokens/s = T / backward time."""
+    import torch
+
+    from fp8_block_scaled_sigmoid_b200 import _abi, configs, inputs
+    from fp8_block_scaled_sigmoid_b200.layer import MoELayer, make_fp8_weights
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = configs.PRESETS[args.config]
+    w1q, w1s, w2q, w2s = make_fp8_weights(cfg, dev, pow2=args.pow2)
+    layer = MoELayer(cfg, inputs.draw_centroids(cfg, dev), inputs.draw_bias(cfg, dev), w1q, w1s,
+                     w2q, w2s, pow2=args.pow2)
+    u = inputs.draw_u(cfg, dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed + 77)
+    dout = torch.randn(cfg.T, cfg.d, generator=g, device=dev) * 0.01
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+    layer.forward_train(u, update_bias=False)
+    layer.transposed_weights()
+    for _ in range(args.warmup):
+        layer.backward(dout)
+    torch.cuda.synchronize()
+    layer.check()
+    names = ["combine_backward", "dgrad2", "swiglu_backward", "dgrad1", "unpermute", "quant_128x1",
+             "wgrad2", "wgrad1"]
+    per = {n: 0.0 for n in names}
+    total = 0.0
+    sampler = ClockSampler(0)
+    sampler.start()
+    if sampler.proc is not None:
+        time.sleep(0.3)
+    launches = 0
+    t_lo = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev = [torch.cuda.Event(enable_timing=True)]
+        ev[0].record(st)
+
+        def mark(name, ev=ev):
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(st)
+            ev.append(e)
+        lc0 = _abi.launch_count
+        layer.backward(dout, mark=mark)
+        launches += _abi.launch_count - lc0
+        torch.cuda.synchronize()
+        for j, n in enumerate(names):
+            per[n] += ev[j].elapsed_time(ev[j + 1])
+        total += ev[0].elapsed_time(ev[-1])
+    t_hi = time.perf_counter()
+    layer.check()
+    sampler.window(t_lo, t_hi)
+    clocks = sampler.stop()
+    per = {n: round(v / args.steps, 4) for n, v in per.items()}
+    ms = total / args.steps
+    rows = cfg.pairs + cfg.T
+    counts = layer.perm["counts"].cpu()
+    G = cfg.E + cfg.n_shared
+    ldt = _abi.wgrad_ld(layer.max_tiles)
+    peaks, src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fp8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # Wgrad of W1: both token-major operands once, the fp32 gradient of every expert written
+    ktot = 128 * int(layer.perm["n_tiles"].item())
+    w1_bytes = (2 * cfg.I + cfg.d) * ktot * (1 + 1.0 / 128) + G * 2 * cfg.I * cfg.d * 4
+    w1_flops = 2.0 * rows * 2 * cfg.I * cfg.d
+    t_w1 = per["wgrad1"] / 1e3
+    dg_flops = 2.0 * rows * cfg.I * cfg.d
+    result = {
+        "metric": "MoE expert-FFN backward tokens/s on 1 B200 (Dgrad + Wgrad, FP8)",
+        "value": round(cfg.T / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "dtype": "fp8_e4m3", "data": "synthetic (seeded)",
+        "config": {"workload": workload_name(cfg) + "; backward of the expert FFNs for a seeded "
+                   "fp32 output gradient, weight gradients fp32 [G][N][K]",
+                   "scales": "powers of two" if args.pow2 else "fp32 weights/activations, "
+                   "power-of-two gradients", "l2": "512 MB buffer written between steps"},
+        "gpu_launches": launches // args.steps,
+        "kernel_ms": per,
+        "roofline": {"kernel": "grouped_gemm_fp8_wgrad (dW1)", "bound": "hbm",
+                     "achieved": round(w1_bytes / t_w1 / 1e9, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(w1_bytes / t_w1 / 1e9 / hbm, 4),
+                     "algorithmic_bytes": int(w1_bytes), "traffic": None,
+                     "peak_source": f"hbm_gbs, {src}"},
+        "gemm_tflops": {"dgrad2": round(dg_flops / (per["dgrad2"] / 1e3) / 1e12, 1),
+                        "dgrad1": round(dg_flops * 2 / (per["dgrad1"] / 1e3) / 1e12, 1),
+                        "wgrad2": round(dg_flops / (per["wgrad2"] / 1e3) / 1e12, 1),
+                        "wgrad1": round(w1_flops / t_w1 / 1e12, 1), "fp8_peak": fp8_peak},
+        "loads": {"max": int(counts.max()), "active_experts": int((counts > 0).sum())},
+        "clocks": clocks,
+    }
+    print(json.dumps(result), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -618,6 +716,8 @@ def main():
                     help="time CUDA-graph replays of the step instead of eager calls (one GPU)")
     ap.add_argument("--pow2", action="store_true",
                     help="power-of-two scale variant (tensor-core UE8M0 block scaling)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward of the expert FFNs (Dgrad + Wgrad) instead")
     ap.add_argument("--gemm", action="store_true",
                     help="time the standalone 4096x7168x2048 block-scaled GEMM instead")
     args = ap.parse_args()
@@ -627,6 +727,8 @@ def main():
         run_reference(args)
     elif args.gemm:
         run_gemm(args)
+    elif args.backward:
+        run_backward(args)
     else:
         run_gpu(args)
 

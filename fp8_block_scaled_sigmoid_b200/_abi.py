@@ -458,9 +458,10 @@ def fp8_quant_128x1_pow2(src, offsets, tile_group, tile_start, n_tiles, max_tile
     rows, C = src.shape
     ldt = wgrad_ld(max_tiles)
     dev = _dev(src)
-    qt = torch.zeros(C, ldt, dtype=torch.uint8, device=dev) if qt is None else qt
-    st = torch.zeros(C, ldt // 128, dtype=torch.float32, device=dev) if st is None else st
-    atoms = torch.zeros(C // 128, ldt // 512, 512, dtype=torch.uint8, device=dev) if atoms is None else atoms
+    # columns past the last tile are never read (left unwritten)
+    qt = torch.empty(C, ldt, dtype=torch.uint8, device=dev) if qt is None else qt
+    st = torch.empty(C, ldt // 128, dtype=torch.float32, device=dev) if st is None else st
+    atoms = torch.empty(C // 128, ldt // 512, 512, dtype=torch.uint8, device=dev) if atoms is None else atoms
     if src_scale is None:
         assert src.dtype == torch.float32
         _count("fp8_quant_128x1_pow2")

@@ -170,10 +170,13 @@ __global__ void __launch_bounds__(256) swiglu_backward_kernel(
 // ------------------------------------------------- 128x1 re-quantisation --
 // CTA (tile i, channel block cb): the segment's 128-token tile i (rows
 // offsets[g] + 128 (i - tile_start[g]) .., zero past the segment's end) of
-// channels 128 cb .. 128 cb + 127.  Warp w loads rows w, w + 8, ...; a
-// channel's 128-token amax gives its power-of-two scale; the codes are
-// transposed through shared memory and written as 128-byte rows of qt.
-// FP8 sources (x) are dequantised first with their 1x128 scale.
+// channels 128 cb .. 128 cb + 127.  Warp w loads rows 16w .. 16w + 15 (lane l:
+// channels 4l .. 4l + 3, one coalesced 512-byte row per load), so a thread
+// holds 16 consecutive tokens of its 4 channels.  A channel's 128-token amax
+// (shared-memory reduction over the 8 warps) gives its power-of-two scale;
+// each thread then writes its 16 codes per channel as one 16-byte store into
+// the channel's row of qt.  FP8 sources (x) are dequantised first with their
+// 1x128 scale.
 template <bool FP8_SRC>
 __global__ void __launch_bounds__(256) quant_128x1_kernel(
     const float* __restrict__ src, const uint8_t* __restrict__ src_q,
@@ -183,7 +186,6 @@ __global__ void __launch_bounds__(256) quant_128x1_kernel(
     float* __restrict__ st, uint8_t* __restrict__ atoms) {
   __shared__ float red[8][128];
   __shared__ float scl[128];
-  __shared__ uint8_t tr[128][128 + 16];  // [channel][token], padded rows
   const int i = blockIdx.x;
   if (i >= __ldg(n_tiles)) return;
   const int cb = blockIdx.y;
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(256) quant_128x1_kernel(
   float am[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int m = 0; m < 16; ++m) {
-    const int r = warp + 8 * m;
+    const int r = 16 * warp + m;
 #pragma unroll
     for (int q = 0; q < 4; ++q) v[m][q] = 0.f;
     if (r < nr) {
@@ -237,36 +239,18 @@ __global__ void __launch_bounds__(256) quant_128x1_kernel(
     }
   }
   __syncthreads();
-  float s4[4], rs4[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    s4[q] = scl[c + q];
-    rs4[q] = __frcp_rn(s4[q]);
-  }
+    const float s = scl[c + q];
+    const float rs = __frcp_rn(s);
+    uint32_t w4[4];
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const int r = warp + 8 * m;
-    const uint32_t w = e4m3x4(div_by_scale(v[m][0], s4[0], rs4[0]), div_by_scale(v[m][1], s4[1], rs4[1]),
-                              div_by_scale(v[m][2], s4[2], rs4[2]), div_by_scale(v[m][3], s4[3], rs4[3]));
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tr[c + q][r] = static_cast<uint8_t>((w >> (8 * q)) & 0xFFu);
-  }
-  __syncthreads();
-  // 128 channel rows x 128 bytes: 8 threads per row, 16 bytes each
-#pragma unroll
-  for (int pass = 0; pass < 4; ++pass) {
-    const int row = (threadIdx.x >> 3) + 32 * pass;
-    const int chunk = threadIdx.x & 7;
-    uint32_t wv[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      wv[q] = static_cast<uint32_t>(tr[row][16 * chunk + 4 * q]) |
-              (static_cast<uint32_t>(tr[row][16 * chunk + 4 * q + 1]) << 8) |
-              (static_cast<uint32_t>(tr[row][16 * chunk + 4 * q + 2]) << 16) |
-              (static_cast<uint32_t>(tr[row][16 * chunk + 4 * q + 3]) << 24);
-    *reinterpret_cast<uint4*>(qt + (static_cast<int64_t>(128) * cb + row) * ldt +
-                              static_cast<int64_t>(128) * i + 16 * chunk) =
-        make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    for (int k = 0; k < 4; ++k)
+      w4[k] = e4m3x4(div_by_scale(v[4 * k][q], s, rs), div_by_scale(v[4 * k + 1][q], s, rs),
+                     div_by_scale(v[4 * k + 2][q], s, rs), div_by_scale(v[4 * k + 3][q], s, rs));
+    *reinterpret_cast<uint4*>(qt + (static_cast<int64_t>(128) * cb + c + q) * ldt +
+                              static_cast<int64_t>(128) * i + 16 * warp) =
+        make_uint4(w4[0], w4[1], w4[2], w4[3]);
   }
 }
 

@@ -218,7 +218,7 @@ class MoELayer:
             self._wt = (w1t, w1ts, w2t, w2ts)
         return self._wt
 
-    def backward(self, dout: torch.Tensor, weight_grads: bool = True) -> dict:
+    def backward(self, dout: torch.Tensor, weight_grads: bool = True, mark=None) -> dict:
         """Gradients of the expert FFNs for the upstream gradient dout (fp32
         [T][d]) of the last forward_train: du (the layer input's gradient
         through the residual and the experts; the router's share is not
@@ -229,17 +229,22 @@ class MoELayer:
         grouped_gemm_fp8_wgrad."""
         c = self.cfg
         p = self.perm
-        d, I = c.d, c.I
+        mark = mark or (lambda name: None)
         w1t, w1ts, w2t, w2ts = self.transposed_weights()
         dyq, dys, dy = _abi.moe_combine_backward(dout, p["dst_of"], self.gate, want_dy=weight_grads)
+        mark("combine_backward")
         dh = _abi.grouped_gemm_fp8_blockscaled(dyq, dys, w2t, w2ts, p["offsets"], p["tile_group"],
                                                p["tile_start"], p["n_tiles"], self.max_tiles,
                                                _abi.EP_F32, dev_err=self.dev_err, pow2=self.pow2)
+        mark("dgrad2")
         dguq, dgus, dgu, h = _abi.swiglu_backward(dh, self.GUq, self.GUs, want_fp32=weight_grads)
+        mark("swiglu_backward")
         dx = _abi.grouped_gemm_fp8_blockscaled(dguq, dgus, w1t, w1ts, p["offsets"], p["tile_group"],
                                                p["tile_start"], p["n_tiles"], self.max_tiles,
                                                _abi.EP_F32, dev_err=self.dev_err, pow2=self.pow2)
+        mark("dgrad1")
         du = _abi.moe_unpermute_add(dx, p["dst_of"], dout)
+        mark("unpermute")
         r = {"du": du, "dyq": dyq, "dys": dys, "dh": dh, "dguq": dguq, "dgus": dgus, "dx": dx}
         if weight_grads:
             G = c.E + c.n_shared
@@ -248,10 +253,13 @@ class MoELayer:
             ht = _abi.fp8_quant_128x1_pow2(h, *tabs)
             dgut = _abi.fp8_quant_128x1_pow2(dgu, *tabs)
             xt = _abi.fp8_quant_128x1_pow2(self.Xq, *tabs, src_scale=self.Xs)
+            mark("quant_128x1")
             r["dW2"] = _abi.grouped_gemm_fp8_wgrad(dyt[0], dyt[2], ht[0], ht[2], p["tile_start"], G,
                                                    dev_err=self.dev_err)
+            mark("wgrad2")
             r["dW1"] = _abi.grouped_gemm_fp8_wgrad(dgut[0], dgut[2], xt[0], xt[2], p["tile_start"], G,
                                                    dev_err=self.dev_err)
+            mark("wgrad1")
             r.update({"dy": dy, "dgu": dgu, "h": h, "dyt": dyt, "ht": ht, "dgut": dgut, "xt": xt})
         return r
 
