@@ -41,6 +41,18 @@ def reduce_load_counts(counts: torch.Tensor, tokens_per_rank: int, process_group
     return total, tokens_per_rank * dist.get_world_size(process_group)
 
 
+def reduce_weight_grads(grads: dict, process_group=None) -> dict:
+    """Data parallelism: sum the fp32 expert weight gradients (dW1, dW2) over
+    the ranks in place, so every rank holds the gradient of the whole batch."""
+    if process_group is None:
+        return grads
+    import torch.distributed as dist
+    for k in ("dW1", "dW2"):
+        if k in grads:
+            dist.all_reduce(grads[k], op=dist.ReduceOp.SUM, group=process_group)
+    return grads
+
+
 def max_over_ranks(value: float, device, process_group=None) -> float:
     """Largest value over the ranks (a time: the job finishes with its slowest rank)."""
     if process_group is None:
@@ -261,6 +273,7 @@ class MoELayer:
                                                    dev_err=self.dev_err)
             mark("wgrad1")
             r.update({"dy": dy, "dgu": dgu, "h": h, "dyt": dyt, "ht": ht, "dgut": dgut, "xt": xt})
+            reduce_weight_grads(r, self.pg)
         return r
 
     def forward_host(self, u_host: torch.Tensor, out_host: torch.Tensor,

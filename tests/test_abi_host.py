@@ -71,6 +71,36 @@ def test_max_m_tiles_bound():
                                       None, None, 0, None), 1),              # NULL logits
     (lambda L: L.moe_combine(None, None, None, None, None, 4, 40, 128, None, None), 4),
     (lambda L: L.moe_bias_update(None, 4, 8, 2, ctypes.c_float(0.001), None, None), 1),
+    # power-of-two variant
+    (lambda L: L.fp8_quant_1x128_pow2(None, 200, 4, 200, None, None, None), 2),
+    (lambda L: L.fp8_quant_128x128_pow2(None, 64, 4, 128, None, None, None), 2),
+    (lambda L: L.grouped_gemm_fp8_pow2(None, None, 10, None, None, None, None, None, None, 4, 1,
+                                       384, 128, 0, None, None, None, None), 2),  # N % 256
+    (lambda L: L.swiglu_quant_pow2(None, 4, 100, None, None, None), 2),
+    # backward
+    (lambda L: L.fp8_quant_1x128_f32(None, 200, 4, 200, 0, None, None, None), 2),
+    (lambda L: L.fp8_quant_1x128_f32(None, 128, 4, 128, 1, None, None, None), 1),
+    (lambda L: L.moe_combine_backward(None, None, None, 4, 4, 200, None, None, None, None), 2),
+    (lambda L: L.moe_combine_backward(None, None, None, 4, 40, 128, None, None, None, None), 4),
+    (lambda L: L.swiglu_backward(None, None, None, 4, 100, None, None, None, None, None), 2),
+    (lambda L: L.fp8_quant_128x1_pow2(None, 128, None, None, None, None, 4, 128, None, 512, None,
+                                      None, None), 1),                        # NULL source
+    (lambda L: L.fp8_quant_128x1_pow2(16, 128, None, None, None, None, 4, 100, None, 512, None,
+                                      None, None), 2),                        # C % 128
+    (lambda L: L.fp8_quant_128x1_pow2(16, 256, None, None, None, None, 4, 256, None, 256, None,
+                                      None, None), 2),                        # ldt < 128 * tiles
+    (lambda L: L.fp8_quant_128x1_pow2(16, 256, None, None, None, None, 2, 256, None, 384, None,
+                                      32, None), 2),                          # atoms need ldt % 512
+    (lambda L: L.fp8_requant_128x1_pow2(None, None, 128, None, None, None, None, 4, 128, None, 512,
+                                        None, None, None), 1),
+    (lambda L: L.fp8_transpose_128x128(None, None, 2, 100, 128, None, None, None), 2),
+    (lambda L: L.moe_unpermute_add(None, None, None, 4, 40, 128, None, None), 4),
+    (lambda L: L.grouped_gemm_fp8_wgrad(None, None, None, None, 512, 100, 256, None, 2, None,
+                                        None, None), 2),                      # Ma % 128
+    (lambda L: L.grouped_gemm_fp8_wgrad(None, None, None, None, 500, 128, 256, None, 2, None,
+                                        None, None), 2),                      # ldt % 512
+    (lambda L: L.grouped_gemm_fp8_wgrad(None, None, None, None, 512, 128, 256, None, 2, None,
+                                        None, None), 1),                      # NULL buffers
 ])
 def test_host_validation(call, code):
     assert call(_abi.lib()) == code
@@ -81,3 +111,9 @@ def test_empty_batches_are_no_ops():
     assert L.fp8_quant_1x128(None, 128, 0, 128, None, None, None) == 0
     assert L.moe_combine(None, None, None, None, None, 0, 8, 128, None, None) == 0
     assert L.swiglu_quant(None, 0, 128, None, None, None) == 0
+    assert L.moe_combine_backward(None, None, None, 0, 4, 128, None, None, None, None) == 0
+    assert L.swiglu_backward(None, None, None, 0, 128, None, None, None, None, None) == 0
+    assert L.fp8_quant_128x1_pow2(16, 128, None, None, None, None, 0, 128, None, 0, None, None,
+                                  None) == 0
+    assert L.grouped_gemm_fp8_wgrad(None, None, None, None, 512, 128, 256, None, 0, None, None,
+                                    None) == 0

@@ -67,3 +67,38 @@ def test_bias_update_over_two_ranks():
         assert np.array_equal(total, counts_all) and t_all == 2 * T
         assert np.array_equal(nb, want)
         assert slowest == 2.0
+
+
+def _grad_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from fp8_block_scaled_sigmoid_b200.layer import reduce_weight_grads
+    rng = np.random.default_rng(200 + rank)
+    g = {"dW1": torch.from_numpy(rng.normal(0, 1, (3, 8, 4)).astype(np.float32)),
+         "dW2": torch.from_numpy(rng.normal(0, 1, (3, 4, 8)).astype(np.float32))}
+    local = {k: v.clone() for k, v in g.items()}
+    reduce_weight_grads(g, dist.group.WORLD)
+    q.put((rank, {k: v.numpy() for k, v in local.items()}, {k: v.numpy() for k, v in g.items()}))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_weight_grads_sum_over_two_ranks():
+    """Data-parallel training: each rank's expert weight gradients (fp32,
+    "Mixed Precision Framework") are summed over the ranks, so both hold the
+    gradient of the whole batch."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_grad_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=120) for _ in procs], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for k in ("dW1", "dW2"):
+        want = res[0][1][k] + res[1][1][k]
+        for _, _, reduced in res:
+            assert np.array_equal(reduced[k], want)
