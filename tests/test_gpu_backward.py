@@ -222,3 +222,81 @@ def test_layer_backward(cuda_dev, pow2):
     for k in ("dx", "du", "dW1", "dW2"):
         rel = np.linalg.norm(npraw(r[k]) - ro[k]) / np.linalg.norm(ro[k])
         assert rel < 1e-2, (k, rel)
+
+
+@pytest.mark.slow
+def test_layer_backward_v3_prefill_sampled(cuda_dev):
+    """The benchmark's backward workload (V3 prefill, 257 experts, fp32-scale
+    weights), checked on sampled tokens, rows and weight-gradient rows, each
+    recomputed by the oracle one by one from the operands the GPU consumed."""
+    cfg = configs.V3_PREFILL
+    w1q, w1s, w2q, w2s = make_fp8_weights(cfg, cuda_dev)
+    layer = MoELayer(cfg, inputs.draw_centroids(cfg, cuda_dev), inputs.draw_bias(cfg, cuda_dev),
+                     w1q, w1s, w2q, w2s)
+    u = inputs.draw_u(cfg, cuda_dev)
+    layer.forward_train(u, update_bias=False)
+    g = torch.Generator(device=cuda_dev)
+    g.manual_seed(cfg.seed + 77)
+    dout = torch.randn(cfg.T, cfg.d, generator=g, device=cuda_dev) * 0.01
+    r = layer.backward(dout)
+    torch.cuda.synchronize()
+    layer.check()
+    T, K, P, I, d, E = cfg.T, cfg.K, cfg.T * cfg.K, cfg.I, cfg.d, cfg.E
+    dst, gate = npraw(layer.perm["dst_of"]), npraw(layer.gate)
+    idx = npraw(layer.idx)
+    offs, ts = npraw(layer.perm["offsets"]), npraw(layer.perm["tile_start"])
+    dout_h = npraw(dout)
+    rng = np.random.default_rng(1)
+    toks = sorted(rng.choice(T, 2, replace=False).tolist()) + [T - 1]
+    w = {}
+
+    def W(e):
+        if e not in w:
+            w[e] = (O.dequant_128x128(npraw(w1q[e]), npraw(w1s[e])),
+                    O.dequant_128x128(npraw(w2q[e]), npraw(w2s[e])))
+        return w[e]
+
+    for t in toks:
+        du_ref = dout_h[t].astype(np.float64)
+        for e, row, gt in [(E, P + t, np.float32(1.0))] + [(idx[t, k], dst[t, k], gate[t, k])
+                                                           for k in range(K)]:
+            W1, W2 = W(int(e))
+            dy = (gt * dout_h[t]).astype(np.float32)[None]
+            qy, sy = O.quant_1x128_pow2(dy)
+            assert np.array_equal(npraw(r["dyq"][row:row + 1]), qy)
+            assert np.array_equal(npraw(r["dys"][row:row + 1]), sy)
+            dh = O.dequant_1x128(qy, sy) @ W2                   # dy . W2 -> [1][I]
+            dh_g = npraw(r["dh"][row:row + 1])
+            assert_within_rms(dh_g, dh, what=f"dh row {row}")
+            gu = O.dequant_1x128(npraw(layer.GUq[row:row + 1]), npraw(layer.GUs[row:row + 1]))
+            dgu, h = O.swiglu_backward(dh_g, gu, I)
+            bound = 4e-6 * np.abs(dgu) + 2e-6 * np.sqrt(np.mean(dgu * dgu))
+            assert np.all(np.abs(npraw(r["dgu"][row:row + 1]) - dgu) <= bound)
+            qg, sg = O.quant_1x128_pow2(npraw(r["dgu"][row:row + 1]))
+            assert np.array_equal(npraw(r["dguq"][row:row + 1]), qg)
+            dx = O.dequant_1x128(qg, sg) @ W1                   # dgu . W1 -> [1][d]
+            dx_g = npraw(r["dx"][row:row + 1])
+            assert_within_rms(dx_g, dx, what=f"dx row {row}")
+            du_ref = du_ref + dx_g[0].astype(np.float64)
+        assert_within_rms(npraw(r["du"][t]), du_ref, what=f"du token {t}")
+    # weight-gradient rows of a routed expert and of the shared expert
+    for e in (int(np.argmax(offs[1:E + 1] - offs[:E])), E):
+        r0, r1 = int(offs[e]), int(offs[e + 1])
+        c0, c1 = 128 * int(ts[e]), 128 * int(ts[e + 1])
+        seg = [0, r1 - r0]
+        # the token-major operands of this expert are the oracle's 128x1 quantisation
+        # of the GPU's fp32 dy, h, dgu and cached x
+        xf = O.dequant_1x128(npraw(layer.Xq[r0:r1]), npraw(layer.Xs[r0:r1])).astype(np.float32)
+        ops = {}
+        for key, src in (("dyt", npraw(r["dy"][r0:r1])), ("ht", npraw(r["h"][r0:r1])),
+                         ("dgut", npraw(r["dgu"][r0:r1])), ("xt", xf)):
+            qo, so, _ = O.quant_128x1_pow2(src, seg)
+            assert np.array_equal(npraw(r[key][0][:, c0:c1]), qo), (key, e)
+            assert np.array_equal(npraw(r[key][1][:, c0 // 128:c1 // 128]), so), (key, e)
+            ops[key] = O.dequant_rows(qo, so)
+        for n in (0, 1000, d - 1):
+            ref = ops["dyt"][n] @ ops["ht"].T                   # dW2[e][n][:]
+            assert_within_rms(npraw(r["dW2"][e, n]), ref, what=f"dW2[{e}][{n}]")
+        for n in (0, 2 * I - 1):
+            ref = ops["dgut"][n] @ ops["xt"].T                  # dW1[e][n][:]
+            assert_within_rms(npraw(r["dW1"][e, n]), ref, what=f"dW1[{e}][{n}]")
