@@ -25,10 +25,17 @@ namespace {
 
 constexpr int kMaxKb = 32;
 
-// E4M3 byte -> fp32 (exact: every E4M3 value is a half value).
-__device__ __forceinline__ float e4m3_to_float(uint32_t byte) {
-  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(byte), __NV_E4M3);
-  return __half2float(__half(h));
+// Four E4M3 bytes (byte i -> f[i]) through two paired conversions (exact:
+// every E4M3 value is a half value).
+__device__ __forceinline__ void e4m3x4_to_float(uint32_t w, float (&f)[4]) {
+  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+  const float2 a = __half22float2(__half2(lo));
+  const float2 b = __half22float2(__half2(hi));
+  f[0] = a.x;
+  f[1] = a.y;
+  f[2] = b.x;
+  f[3] = b.y;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -139,10 +146,13 @@ __global__ void __launch_bounds__(256) swiglu_backward_kernel(
   const float4 dv = __ldg(reinterpret_cast<const float4*>(dh + r * I + 128 * j) + lane);
   const float dhv[4] = {dv.x, dv.y, dv.z, dv.w};
   float dg[4], du[4], hv[4];
+  float gf[4], uf[4];
+  e4m3x4_to_float(gc, gf);
+  e4m3x4_to_float(uc, uf);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float g = __fmul_rn(e4m3_to_float((gc >> (8 * i)) & 0xFFu), sg);
-    const float u = __fmul_rn(e4m3_to_float((uc >> (8 * i)) & 0xFFu), su);
+    const float g = __fmul_rn(gf[i], sg);
+    const float u = __fmul_rn(uf[i], su);
     const float sig = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-g)));
     const float silu = __fmul_rn(g, sig);
     const float dsilu = __fmul_rn(sig, __fadd_rn(1.0f, __fmul_rn(g, __fsub_rn(1.0f, sig))));
@@ -207,8 +217,10 @@ __global__ void __launch_bounds__(256) quant_128x1_kernel(
       if (FP8_SRC) {
         const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(src_q + (r0 + r) * ld_src + 128 * cb) + lane);
         const float s = __ldg(src_s + (r0 + r) * (ld_src / 128) + cb);
+        float f[4];
+        e4m3x4_to_float(w, f);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[m][q] = __fmul_rn(e4m3_to_float((w >> (8 * q)) & 0xFFu), s);
+        for (int q = 0; q < 4; ++q) v[m][q] = __fmul_rn(f[q], s);
       } else {
         const float4 a = __ldg(reinterpret_cast<const float4*>(src + (r0 + r) * ld_src + 128 * cb) + lane);
         v[m][0] = a.x;

@@ -89,8 +89,12 @@ def test_layer_full_parity(cuda_dev, cfg):
 
 
 @pytest.mark.slow
-def test_layer_v3_prefill_sampled(cuda_dev):
-    cfg = configs.V3_PREFILL
+@pytest.mark.parametrize("cfg", [configs.V3_PREFILL, configs.V3_DECODE, configs.V4_PRO],
+                         ids=lambda c: c.name)
+def test_layer_full_size_sampled(cuda_dev, cfg):
+    """The benchmark's workload and the other full-size configs (V3 decode with
+    Zipf-hot experts, V4-Pro with no group limit), checked on sampled tokens:
+    the oracle recomputes each sampled token's experts one by one."""
     layer, bias0 = _build(cfg, cuda_dev)
     u = inputs.draw_u(cfg, cuda_dev)
     out = layer.forward(u)
