@@ -70,7 +70,14 @@ V3_PREFILL_E32 = MoEConfig("v3_prefill_e32", T=512, d=7168, E=32, G=8, M=4, K=8,
 V3_TOKENS_E32 = MoEConfig("v3_tokens_e32", T=4096, d=7168, E=32, G=8, M=4, K=8, I=2048,
                           bias_lo=-0.05, bias_hi=0.05)
 
-PRESETS = {c.name: c for c in (TINY, V3_PREFILL, V3_DECODE, V4_PRO, V3_PREFILL_E32, V3_TOKENS_E32)}
+# Profiling case for the backward: V3's d and I with ~128 tokens per expert
+# (16 routed experts, top-8 within 4 of 8 groups), so its fp32 weight
+# gradients (17 experts) take ~3 GB and a multi-pass capture stays small.
+V3_BWD_E16 = MoEConfig("v3_bwd_e16", T=256, d=7168, E=16, G=8, M=4, K=8, I=2048,
+                       bias_lo=-0.05, bias_hi=0.05)
+
+PRESETS = {c.name: c for c in (TINY, V3_PREFILL, V3_DECODE, V4_PRO, V3_PREFILL_E32, V3_TOKENS_E32,
+                               V3_BWD_E16)}
 
 
 @dataclass(frozen=True)
