@@ -15,9 +15,10 @@
 //     sb[nblk,kb]) * partial (packed fp32x2 FMA), while the tensor core fills
 //     the other buffer;
 //   * a persistent grid walks the (expert, n-tile, m-tile) work list derived
-//     on the device from the segment offsets, so the ragged expert segments
-//     need no host synchronisation; the m-tiles of one expert that share a
-//     weight tile run next to each other for L2 reuse.
+//     on the device from the segment offsets and the tile table's per-expert
+//     tile prefix, so the ragged expert segments need no host
+//     synchronisation; the m-tiles of one expert that share a weight tile run
+//     next to each other for L2 reuse.
 //
 // The shared-memory ring is staged in K slices of SK bytes (128, or 64 with
 // the 64-byte swizzle): a stage is released as soon as the MMAs of its slice
@@ -31,7 +32,7 @@
 // handshakes cost more than the halved shared-memory ingress saves.
 //
 // Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
-// TMEM owner, warp 2 builds the work list then idles with warp 3 (the first
+// TMEM owner, warp 2 stages the tile prefix then idles with warp 3 (the first
 // warpgroup gives registers to the other two), warps 4..11 = epilogue (warp w
 // reads TMEM lanes 32*(w%4)..).  Epilogues: fp32 rows, or SwiGLU + 1x128 E4M3
 // requantisation of h (the W1 rows are gate/up block-interleaved so one
@@ -87,31 +88,11 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
   return SK == 128 ? smem_desc_sw128(addr) : smem_desc_sw64(addr);
 }
 
-// rstart[g] = number of RT-row tiles of the groups before g (one warp).
-template <int RT>
-__device__ void build_tile_prefix(const GemmArgs& a, int* rstart, int lane) {
-  const int G = a.groups;
-  const int per = (G + 31) / 32;
-  const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
-  int mine = 0;
-  for (int g = g0; g < g1; ++g) {
-    const int c = __ldg(a.offsets + g + 1) - __ldg(a.offsets + g);
-    if (c < 0) set_dev_err(a.dev_err, MOE_DEVERR_BAD_TABLE);
-    mine += c > 0 ? (c + RT - 1) / RT : 0;
-  }
-  int incl = mine;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += n;
-  }
-  int run = incl - mine;
-  for (int g = g0; g < g1; ++g) {
-    rstart[g] = run;
-    const int c = __ldg(a.offsets + g + 1) - __ldg(a.offsets + g);
-    run += c > 0 ? (c + RT - 1) / RT : 0;
-  }
-  if (lane == 31) rstart[G] = incl;
+// rstart[g] = number of 128-row tiles of the groups before g: the tile
+// table's tile_start (written by moe_permute / moe_tile_table), staged in
+// shared memory by one warp.
+__device__ __forceinline__ void load_tile_prefix(const GemmArgs& a, int* rstart, int lane) {
+  for (int g = lane; g <= a.groups; g += 32) rstart[g] = __ldg(a.tile_start + g);
 }
 
 // Work item w -> (expert, n-tile, RT-row tile); the items of expert e occupy
@@ -418,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  if (warp == 2) build_tile_prefix<128>(args, c.rstart, lane);
+  if (warp == 2) load_tile_prefix(args, c.rstart, lane);
   if (warp == 1) {
     tmem_alloc(c.tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -633,7 +614,7 @@ __device__ __forceinline__ bool epilogue_mx_tile(const GemmArgs& args, const Wor
 }
 
 // Warp roles as in gemm1sm_kernel, plus warps 2 and 3 = scale-factor
-// producers (A's and B's exponents; warp 2 first builds the work list).
+// producers (A's and B's exponents; warp 2 first stages the tile prefix).
 // Stages are whole 128-wide K blocks.
 template <int EP>
 __global__ void __launch_bounds__(kThreads, 1) gemm_pow2_kernel(
@@ -667,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pow2_kernel(
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  if (warp == 2) build_tile_prefix<128>(args, c.rstart, lane);
+  if (warp == 2) load_tile_prefix(args, c.rstart, lane);
   if (warp == 1) {
     tmem_alloc(c.tmem_slot, kTmemCols);
     tmem_relinquish();
