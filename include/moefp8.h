@@ -215,7 +215,9 @@ moe_status moe_tile_table(const int32_t* offsets, int groups, int max_tiles,
  *   B  E4M3 [groups][N][K], sb fp32 [groups][N/128][K/128] (128x128 blocks)
  *   offsets int32 [groups+1] (segment g = rows [offsets[g], offsets[g+1]))
  *   tile_group / tile_start / n_tiles: as written by moe_permute or
- *   moe_tile_table; max_tiles = capacity of tile_group.
+ *   moe_tile_table; max_tiles = capacity of tile_group.  The kernel walks
+ *   (group, n-tile, m-tile) work items from tile_start (the per-group tile
+ *   prefix) and offsets; max_tiles bounds its grid.
  *   ep == MOE_EP_F32:  D fp32 [a_rows][N] (rows outside every segment are
  *                      left untouched); d_scale unused.
  *   ep == MOE_EP_SWIGLU_QUANT: B rows are gate/up block-interleaved (rows
