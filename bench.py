@@ -1,7 +1,8 @@
 """Benchmark: MoE-layer tokens/s of the V3-shaped prefill layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config v3_prefill]
-                    [--impl reference] [--no-cpu-baseline]
+                    [--impl reference] [--no-cpu-baseline] [--graph] [--pow2]
+                    [--gemm | --backward]
 
 One step = one forward pass of the whole layer (route, 1x128 quantisation,
 permutation, grouped GEMM 1 with fused SwiGLU + requantisation, grouped
@@ -20,6 +21,12 @@ during the timed region.
 ``--impl reference`` times the CPU oracle instead (rank 0 only) on a bounded
 sample of the same workload and prints the same JSON line with
 "impl": "reference".
+
+Other modes (one GPU, their own JSON line): ``--pow2`` runs the layer with
+power-of-two scales (the tensor core applies them); ``--graph`` times CUDA-graph
+replays of the step; ``--gemm`` times the standalone 4096x7168x2048
+block-scaled GEMM; ``--backward`` times the backward of the expert FFNs
+(Dgrad and Wgrad) per phase.
 """
 from __future__ import annotations
 
