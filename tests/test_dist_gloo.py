@@ -194,3 +194,19 @@ def test_expert_shard_bounds():
         ep.ExpertShard(250, 8, 0)
     with pytest.raises(ValueError):
         ep.ExpertShard(256, 8, 8)
+
+
+def test_expert_parallel_single_rank_is_identity():
+    """world = 1: the plan keeps every row and both exchanges are copies."""
+    from fp8_block_scaled_sigmoid_b200 import ep
+    counts, xq, xs, _ = _ep_rank_data(0)
+    shard = ep.ExpertShard(EP_E, 1, 0)
+    plan = ep.plan_dispatch(torch.from_numpy(counts), shard)
+    assert plan.send_splits == plan.recv_splits == [int(counts.sum())]
+    assert np.array_equal(plan.recv_counts.numpy()[0], counts)
+    rq, rs = ep.dispatch(torch.from_numpy(xq), torch.from_numpy(xs), plan)
+    assert np.array_equal(rq.numpy(), xq) and np.array_equal(rs.numpy(), xs)
+    y = torch.from_numpy(O.dequant_1x128(xq, xs).astype(np.float32))
+    assert torch.equal(ep.combine_return(y, plan), y)
+    with pytest.raises(ValueError):
+        ep.exchange_rows(torch.zeros(3, 4), [2], [2])
