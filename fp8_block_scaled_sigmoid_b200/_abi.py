@@ -40,6 +40,7 @@ _SIGS = {
     "moe_permute_noalloc": (_i, [_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p,
                                  _p, _p, _p, _p]),
     "moe_tile_table": (_i, [_p, _i, _i, _p, _p, _p, _p, _p]),
+    "moe_segment_ids": (_i, [_p, _i, _i, _i64, _p, _p, _p]),
     "grouped_gemm_fp8_blockscaled": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
                                           _i, _p, _p, _p, _p]),
     "grouped_gemm_fp8_pow2": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
@@ -76,7 +77,7 @@ LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant
                      "fp8_requant_128x1_pow2": 1, "fp8_transpose_128x128": 1,
                      "moe_unpermute_add": 1, "grouped_gemm_fp8_wgrad": 1,
                      "moe_route": 2, "moe_permute": 4, "moe_permute_noalloc": 4,
-                     "moe_tile_table": 1,
+                     "moe_tile_table": 1, "moe_segment_ids": 1,
                      "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1,
                      "moe_seq_balance_loss": 3}
 launch_count = 0
@@ -306,6 +307,17 @@ def moe_tile_table(offsets, max_tiles, tile_group=None, tile_start=None, n_tiles
                                 _ptr(tile_start), _ptr(n_tiles), _ptr(dev_err), _stream(stream)),
            "moe_tile_table")
     return tile_group, tile_start, n_tiles
+
+
+def moe_segment_ids(counts, E, n_rows, ids=None, dev_err=None, stream=None):
+    """counts int32 [sources][E] (or flat) -> ids int32 [n_rows]: the local
+    expert of every row of a source-major, expert-sorted receive buffer."""
+    c = counts.reshape(-1)
+    ids = torch.empty(n_rows, dtype=torch.int32, device=_dev(counts)) if ids is None else ids
+    _count("moe_segment_ids")
+    _check(lib().moe_segment_ids(_ptr(c), c.numel(), E, n_rows, _ptr(ids), _ptr(dev_err),
+                                 _stream(stream)), "moe_segment_ids")
+    return ids
 
 
 # ------------------------------------------------------------------ GEMM ---

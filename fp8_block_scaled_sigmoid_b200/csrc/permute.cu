@@ -248,6 +248,45 @@ __global__ void __launch_bounds__(kScanThreads) tile_table_kernel(
                smem);
 }
 
+// Segment ids of a source-major receive buffer (expert parallelism): the
+// rows of segment s = counts[s] come after those of segments 0..s-1, and
+// every row of segment s gets id s % E (its local expert).  Each CTA scans
+// the <= 1024 counts itself, then labels its 4096 rows by binary search.
+constexpr int kSegRowsPerCta = 4096;
+
+__global__ void __launch_bounds__(kScanThreads) segment_ids_kernel(
+    const int32_t* __restrict__ counts, int nseg, int E, int64_t n_rows,
+    int32_t* __restrict__ ids, int32_t* dev_err) {
+  __shared__ int64_t incl[kScanThreads];
+  const int t = threadIdx.x;
+  int64_t c = t < nseg ? __ldg(counts + t) : 0;
+  if (c < 0) {
+    set_dev_err(dev_err, MOE_DEVERR_BAD_TABLE);
+    c = 0;
+  }
+  incl[t] = c;
+  __syncthreads();
+  for (int d = 1; d < kScanThreads; d <<= 1) {
+    const int64_t v = t >= d ? incl[t - d] : 0;
+    __syncthreads();
+    incl[t] += v;
+    __syncthreads();
+  }
+  if (blockIdx.x == 0 && t == 0 && incl[kScanThreads - 1] != n_rows)
+    set_dev_err(dev_err, MOE_DEVERR_BAD_TABLE);
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kSegRowsPerCta;
+  for (int64_t r = r0 + t; r < n_rows && r < r0 + kSegRowsPerCta; r += kScanThreads) {
+    // first segment whose inclusive end exceeds r
+    int lo = 0, hi = nseg - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (incl[mid] > r) hi = mid;
+      else lo = mid + 1;
+    }
+    ids[r] = lo % E;
+  }
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int n_chunks_of(int T) { return (T + kChunkT - 1) / kChunkT; }
@@ -308,6 +347,24 @@ extern "C" moe_status moe_permute(const int32_t* topk_idx, int T, int K, int E, 
                                                        xscale_perm);
     MOE_CUDA_CHECK_LAUNCH();
   }
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_segment_ids(const int32_t* counts, int n_segments, int E,
+                                      int64_t n_rows, int32_t* ids, int32_t* dev_err,
+                                      moe_stream_t stream) {
+  using namespace moe;
+  if (n_segments <= 0 || E <= 0 || n_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (n_segments % E != 0) return MOE_ERR_SHAPE;
+  if (n_segments > kScanThreads) return MOE_ERR_UNSUPPORTED;
+  if (n_rows == 0) return MOE_OK;
+  if (!counts || !ids) return MOE_ERR_INVALID_ARG;
+  const int64_t ctas = (n_rows + kSegRowsPerCta - 1) / kSegRowsPerCta;
+  if (ctas > 0x7FFFFFFF) return MOE_ERR_UNSUPPORTED;
+  segment_ids_kernel<<<static_cast<unsigned>(ctas), kScanThreads, 0,
+                       static_cast<cudaStream_t>(stream)>>>(counts, n_segments, E, n_rows, ids,
+                                                             dev_err);
+  MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }
 

@@ -204,6 +204,19 @@ moe_status moe_tile_table(const int32_t* offsets, int groups, int max_tiles,
                           int32_t* dev_err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_segment_ids -- expert parallelism: the local expert of every row of a
+ * receive buffer that holds, for each source rank s in order, its rows of
+ * this rank's E local experts sorted by expert ([ANN] "Low-Precision
+ * Communication": FP8 rows dispatched to the experts' ranks).  counts int32
+ * [n_segments] (= [sources][E], row-major) -> ids int32 [n_rows], row r of
+ * segment s gets s % E; the ids feed moe_permute (K = 1) to regroup the rows
+ * by expert.  Counts that do not sum to n_rows, or negative counts, record
+ * MOE_DEVERR_BAD_TABLE.
+ * Limits: n_segments % E == 0, n_segments <= 1024. */
+moe_status moe_segment_ids(const int32_t* counts, int n_segments, int E, int64_t n_rows,
+                           int32_t* ids, int32_t* dev_err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * grouped_gemm_fp8_blockscaled -- D_g = A_g . B_g^T for every segment g, with
  * FP8 operands, per-128-K block scales and fp32 accumulation.
  * [ANN] "Fine-Grained Quantization" (per-group scales along the inner
