@@ -1,7 +1,7 @@
 """Benchmark: MoE-layer tokens/s of the V3-shaped prefill layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config v3_prefill]
-                    [--impl reference] [--no-cpu-baseline] [--graph] [--pow2]
+                    [--impl reference] [--no-cpu-baseline] [--graph] [--pow2] [--ep]
                     [--gemm | --backward]
 
 One step = one forward pass of the whole layer (route, 1x128 quantisation,
@@ -26,7 +26,8 @@ Other modes (one GPU, their own JSON line): ``--pow2`` runs the layer with
 power-of-two scales (the tensor core applies them); ``--graph`` times CUDA-graph
 replays of the step; ``--gemm`` times the standalone 4096x7168x2048
 block-scaled GEMM; ``--backward`` times the backward of the expert FFNs
-(Dgrad and Wgrad) per phase.
+(Dgrad and Wgrad) per phase; ``--ep`` shards the routed experts over the N
+ranks (expert parallelism, FP8 dispatch as NCCL all-to-alls).
 """
 from __future__ import annotations
 
@@ -263,6 +264,8 @@ def run_gpu(args):
 
     cfg = configs.PRESETS[args.config]
     cfg_rank = cfg.with_(seed=cfg.seed + rank)       # each rank its own token batch
+    if args.ep:
+        return run_ep(args, cfg, cfg_rank, dev, pg, world, rank, local)
     w1q, w1s, w2q, w2s = make_fp8_weights(cfg, dev, pow2=args.pow2)  # same on every rank
     cent = inputs.draw_centroids(cfg, dev)
     bias = inputs.draw_bias(cfg, dev)
@@ -613,6 +616,81 @@ def run_gemm(args):
         "clocks": clocks}), flush=True)
 
 
+def run_ep(args, cfg, cfg_rank, dev, pg, world, rank, local):
+    """Expert parallelism: each rank holds E/world routed experts (plus the
+    shared one) and its own batch of T tokens; the routed rows travel to
+    their experts' ranks and back as NCCL all-to-alls (ep.MoELayerEP).  Weak
+    scaling: T tokens per rank.  Timed per step with CUDA events, max over
+    ranks; clocks sampled as in the main mode."""
+    import torch
+    import torch.distributed as dist
+
+    from fp8_block_scaled_sigmoid_b200 import _abi, ep, inputs
+    from fp8_block_scaled_sigmoid_b200.layer import make_fp8_weights, max_over_ranks
+
+    shard = ep.ExpertShard(cfg.E, world, rank)
+    experts = list(range(shard.e0, shard.e1)) + [cfg.E + i for i in range(cfg.n_shared)]
+    w = make_fp8_weights(cfg, dev, experts=experts)
+    layer = ep.MoELayerEP(cfg, inputs.draw_centroids(cfg, dev), inputs.draw_bias(cfg, dev), *w,
+                          shard, process_group=pg)
+    u = inputs.draw_u(cfg_rank, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+
+    def barrier():
+        if pg is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        layer.forward(u)
+    barrier()
+    layer.check()
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        if sampler.proc is not None:
+            time.sleep(0.3)
+    barrier()
+    t_lo = time.perf_counter()
+    total = 0.0
+    lc0 = _abi.launch_count
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        layer.forward(u)
+        e1.record(st)
+        e1.synchronize()   # the next step's dispatch plan reads its split sizes on the host
+        total += e0.elapsed_time(e1)
+    barrier()
+    t_hi = time.perf_counter()
+    launches = _abi.launch_count - lc0
+    layer.check()
+    if sampler:
+        sampler.window(t_lo, t_hi)
+    clocks = sampler.stop() if sampler else None
+    ms = max_over_ranks(total, dev, pg)
+    result = {
+        "metric": METRIC + " (expert parallel)", "value": round(cfg.T * world * args.steps / (ms / 1e3), 1),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic (seeded)",
+        "config": {"workload": workload_name(cfg), "tokens_per_gpu": cfg.T,
+                   "parallelism": f"ep{world} ({shard.per_rank} routed experts per GPU + shared; "
+                                  "FP8 dispatch and output return as NCCL all-to-alls)",
+                   "l2": "512 MB buffer written between timed steps"},
+        "gpu_launches": launches, "roofline": None,
+        "roofline_note": "per-kernel times are not separated in this mode",
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if pg is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_backward(args):
     """Backward of the expert FFNs at the configured layer size (one GPU):
     forward_train once per step (untimed), then the timed backward with the
@@ -723,6 +801,8 @@ def main():
                     help="time CUDA-graph replays of the step instead of eager calls (one GPU)")
     ap.add_argument("--pow2", action="store_true",
                     help="power-of-two scale variant (tensor-core UE8M0 block scaling)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism: routed experts sharded over the N ranks")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward of the expert FFNs (Dgrad + Wgrad) instead")
     ap.add_argument("--gemm", action="store_true",

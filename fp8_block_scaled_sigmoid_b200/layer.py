@@ -68,20 +68,24 @@ def quantise_weight_stack(w_bf16: torch.Tensor, q=None, s=None, pow2: bool = Fal
     return _abi.fp8_quant_128x128(w_bf16, q, s, pow2=pow2)
 
 
-def make_fp8_weights(cfg: MoEConfig, device, chunk: int = 16, pow2: bool = False):
+def make_fp8_weights(cfg: MoEConfig, device, chunk: int = 16, pow2: bool = False,
+                     experts: list[int] | None = None):
     """Draw the bf16 expert weights (seeded, per expert) and quantise them on
     the device a few experts at a time; only the FP8 stacks stay resident.
     ``pow2`` rounds the block scales up to powers of two (for a layer built
-    with pow2=True)."""
-    G = cfg.E + cfg.n_shared
+    with pow2=True).  ``experts`` selects the stacked experts, in order
+    (default: all routed experts, then the shared one = index E); an
+    expert-parallel rank takes its own block plus the shared expert."""
+    ids = list(range(cfg.E + cfg.n_shared)) if experts is None else list(experts)
+    G = len(ids)
     w1q = torch.empty(G, 2 * cfg.I, cfg.d, dtype=torch.uint8, device=device)
     w1s = torch.empty(G, 2 * cfg.I // 128, cfg.d // 128, dtype=torch.float32, device=device)
     w2q = torch.empty(G, cfg.d, cfg.I, dtype=torch.uint8, device=device)
     w2s = torch.empty(G, cfg.d // 128, cfg.I // 128, dtype=torch.float32, device=device)
     for e0 in range(0, G, chunk):
         e1 = min(G, e0 + chunk)
-        w1 = torch.stack([_inputs.draw_w1(cfg, e, device) for e in range(e0, e1)])
-        w2 = torch.stack([_inputs.draw_w2(cfg, e, device) for e in range(e0, e1)])
+        w1 = torch.stack([_inputs.draw_w1(cfg, ids[e], device) for e in range(e0, e1)])
+        w2 = torch.stack([_inputs.draw_w2(cfg, ids[e], device) for e in range(e0, e1)])
         _abi.fp8_quant_128x128(w1, w1q[e0:e1], w1s[e0:e1], pow2=pow2)
         _abi.fp8_quant_128x128(w2, w2q[e0:e1], w2s[e0:e1], pow2=pow2)
         del w1, w2
