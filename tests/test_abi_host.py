@@ -101,6 +101,11 @@ def test_max_m_tiles_bound():
                                         None, None), 2),                      # ldt % 512
     (lambda L: L.grouped_gemm_fp8_wgrad(None, None, None, None, 512, 128, 256, None, 2, None,
                                         None, None), 1),                      # NULL buffers
+    # expert parallelism
+    (lambda L: L.moe_segment_ids(None, 12, 8, 100, None, None, None), 2),    # segments % E
+    (lambda L: L.moe_segment_ids(None, 2048, 8, 100, None, None, None), 4),  # > 1024 segments
+    (lambda L: L.moe_segment_ids(None, 16, 8, 100, None, None, None), 1),    # NULL buffers
+    (lambda L: L.moe_segment_ids(None, 16, 0, 100, None, None, None), 1),    # E = 0
 ])
 def test_host_validation(call, code):
     assert call(_abi.lib()) == code
@@ -117,3 +122,4 @@ def test_empty_batches_are_no_ops():
                                   None) == 0
     assert L.grouped_gemm_fp8_wgrad(None, None, None, None, 512, 128, 256, None, 0, None, None,
                                     None) == 0
+    assert L.moe_segment_ids(None, 16, 8, 0, None, None, None) == 0
