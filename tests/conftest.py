@@ -19,3 +19,15 @@ def cuda_dev():
     if not torch.cuda.is_available():
         pytest.fail("GPU test collected without a CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(params=["numpy", "cpp"])
+def O(request):
+    """The oracle under test: the numpy one (oracle/moe_oracle.py) or the
+    single-threaded C++ one (oracle/moe_oracle_ref.cpp).  Every pin that
+    takes this fixture runs against both."""
+    if request.param == "numpy":
+        from oracle import moe_oracle as m
+    else:
+        from oracle import cpp_oracle as m
+    return m

@@ -106,6 +106,10 @@ def test_max_m_tiles_bound():
     (lambda L: L.moe_segment_ids(None, 2048, 8, 100, None, None, None), 4),  # > 1024 segments
     (lambda L: L.moe_segment_ids(None, 16, 8, 100, None, None, None), 1),    # NULL buffers
     (lambda L: L.moe_segment_ids(None, 16, 0, 100, None, None, None), 1),    # E = 0
+    # FP8 peak measurement loop
+    (lambda L: L.moe_fp8_mma_peak(0, 0, 4, 16, None, None), 1),              # iters < 1
+    (lambda L: L.moe_fp8_mma_peak(1, 100, 4, None, None, None), 1),          # NULL sink
+    (lambda L: L.moe_fp8_mma_peak(0, (1 << 21) + 1, 4, 16, None, None), 4),  # beyond the wait
 ])
 def test_host_validation(call, code):
     assert call(_abi.lib()) == code

@@ -14,7 +14,7 @@ not any kernel.)
 """
 import numpy as np
 
-from oracle import moe_oracle as O
+from oracle import moe_oracle as ONP
 
 
 def _round_bits(x, bits=14):
@@ -22,7 +22,7 @@ def _round_bits(x, bits=14):
     return np.ldexp(np.rint(m * 2.0 ** bits) / 2.0 ** bits, e)
 
 
-def test_fourteen_bit_accumulation_misses_the_bar_promotion_meets_it():
+def test_fourteen_bit_accumulation_misses_the_bar_promotion_meets_it(O):
     rng = np.random.default_rng(21)
     M, N, K = 48, 48, 4096
     a = O.e4m3_decode(O.e4m3_encode(rng.normal(0, 1, (M, K)) * 16))

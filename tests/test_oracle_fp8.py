@@ -13,14 +13,14 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import moe_oracle as O
+from oracle import moe_oracle as ONP
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden", "e4m3_points.txt")
 FINITE_CODES = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
 
 
 def _finite_values():
-    return O.e4m3_decode(FINITE_CODES)
+    return ONP.e4m3_decode(FINITE_CODES)
 
 
 def _nearest_code_bruteforce(v: float) -> int:
@@ -39,7 +39,7 @@ def _nearest_code_bruteforce(v: float) -> int:
     return (even or cands)[0]
 
 
-def test_golden_points():
+def test_golden_points(O):
     rows = []
     with open(GOLD) as f:
         for line in f:
@@ -54,7 +54,7 @@ def test_golden_points():
         assert got == c, (v, hex(c), hex(got))
 
 
-def test_roundtrip_all_finite_codes():
+def test_roundtrip_all_finite_codes(O):
     vals = O.e4m3_decode(FINITE_CODES)
     assert np.array_equal(O.e4m3_encode(vals), FINITE_CODES)
     assert np.isnan(O.e4m3_decode(np.array([0x7F, 0xFF], np.uint8))).all()
@@ -63,7 +63,7 @@ def test_roundtrip_all_finite_codes():
     assert pos[-1] == 448.0 and pos[1] == 2.0 ** -9
 
 
-def test_encode_matches_bruteforce_nearest():
+def test_encode_matches_bruteforce_nearest(O):
     rng = np.random.default_rng(0)
     v = np.concatenate([
         rng.normal(0, 1, 400) * np.exp2(rng.integers(-12, 10, 400)),
@@ -76,7 +76,7 @@ def test_encode_matches_bruteforce_nearest():
     assert np.array_equal(got, want)
 
 
-def test_encode_agrees_with_torch_float8_in_range():
+def test_encode_agrees_with_torch_float8_in_range(O):
     rng = np.random.default_rng(1)
     v = (rng.normal(0, 60, 20000)).astype(np.float32)
     v = v[np.abs(v) <= 448]
@@ -85,7 +85,7 @@ def test_encode_agrees_with_torch_float8_in_range():
     assert np.array_equal(ours, theirs)
 
 
-def test_quant_1x128_properties():
+def test_quant_1x128_properties(O):
     rng = np.random.default_rng(2)
     x = rng.normal(0, 1, (9, 512)).astype(np.float32)
     x[3, 130] = -50.0                           # an outlier in tile (3, 1)
@@ -116,7 +116,7 @@ def test_quant_1x128_properties():
     assert np.all(np.abs(deq - x) <= half_step * np.repeat(s, 128, axis=1) * (1 + 1e-6))
 
 
-def test_quant_1x128_bruteforce_codes():
+def test_quant_1x128_bruteforce_codes(O):
     rng = np.random.default_rng(3)
     x = (rng.normal(0, 3, (2, 256)) * np.exp2(rng.integers(-6, 6, (2, 256)))).astype(np.float32)
     q, s = O.quant_1x128(x)
@@ -126,7 +126,7 @@ def test_quant_1x128_bruteforce_codes():
             assert q[r, c] == _nearest_code_bruteforce(float(y))
 
 
-def test_quant_128x128_blocks():
+def test_quant_128x128_blocks(O):
     rng = np.random.default_rng(4)
     w = rng.normal(0, 0.05, (200, 256)).astype(np.float32)   # ragged last row-block
     w[7, 200] = 3.0

@@ -10,10 +10,10 @@ itself a power of two.
 """
 import numpy as np
 
-from oracle import moe_oracle as O
+from oracle import moe_oracle as ONP
 
 FINITE_CODES = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
-FINITE_VALUES = O.e4m3_decode(FINITE_CODES)
+FINITE_VALUES = ONP.e4m3_decode(FINITE_CODES)
 
 
 def _nearest_code(v: float) -> int:
@@ -34,7 +34,7 @@ def _smallest_pow2_at_least(s: float) -> float:
     raise AssertionError("out of range")
 
 
-def test_pow2_ceil_bruteforce():
+def test_pow2_ceil_bruteforce(O):
     rng = np.random.default_rng(11)
     s = np.exp2(rng.uniform(-30, 20, 400)).astype(np.float32)
     exact = np.exp2(np.arange(-30, 20)).astype(np.float32)
@@ -50,7 +50,7 @@ def test_pow2_ceil_bruteforce():
     assert np.array_equal(O.pow2_ceil(above), 2 * exact)
 
 
-def test_quant_1x128_pow2_worked_example():
+def test_quant_1x128_pow2_worked_example(O):
     # amax 0.3: 0.3/448 = 6.70e-4 lies in (2^-11, 2^-10], so the scale is 2^-10;
     # 0.3 * 1024 = 307.2 lies between the E4M3 values 288 and 320 (step 32
     # in [256, 512)) and rounds to 320 = 1.25 * 2^8: exponent field 15,
@@ -66,7 +66,7 @@ def test_quant_1x128_pow2_worked_example():
     assert np.all(q[0, 3:] == 0)
 
 
-def test_quant_1x128_pow2_properties():
+def test_quant_1x128_pow2_properties(O):
     rng = np.random.default_rng(12)
     x = (rng.normal(0, 1, (7, 384)) * np.exp2(rng.integers(-8, 8, (7, 1)))).astype(np.float32)
     x[2, 130] = -77.0
@@ -93,7 +93,7 @@ def test_quant_1x128_pow2_properties():
             assert q[r, c] == _nearest_code(float(yy))
 
 
-def test_pow2_reduces_to_fp32_scale_when_exact():
+def test_pow2_reduces_to_fp32_scale_when_exact(O):
     # a tile whose amax/448 is a power of two gets the same scale and bytes
     rng = np.random.default_rng(13)
     x = rng.uniform(-1, 1, (3, 256)).astype(np.float32)
@@ -109,7 +109,7 @@ def test_pow2_reduces_to_fp32_scale_when_exact():
     assert np.array_equal(s1, s2) and np.array_equal(q1, q2)
 
 
-def test_quant_128x128_pow2():
+def test_quant_128x128_pow2(O):
     rng = np.random.default_rng(14)
     w = rng.normal(0, 0.02, (200, 256)).astype(np.float32)   # ragged last row-block
     w[150, 200] = 0.9
@@ -129,7 +129,7 @@ def test_quant_128x128_pow2():
         assert q[r, c] == _nearest_code(float(yy))
 
 
-def test_swiglu_quant_pow2():
+def test_swiglu_quant_pow2(O):
     rng = np.random.default_rng(15)
     gu = rng.normal(0, 2, (5, 512)).astype(np.float32)
     hq, hs = O.swiglu_quant(gu, 256, pow2=True)

@@ -14,7 +14,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 
-from oracle import moe_oracle as O
+from oracle import moe_oracle as ONP
 
 
 # ---------------------------------------------------------------- routing --
@@ -59,7 +59,7 @@ def _grid_logits(rng, T, E, ties=False):
 
 
 @pytest.mark.parametrize("G,M,K", [(4, 2, 4), (4, 4, 4), (8, 4, 8), (2, 1, 2), (1, 1, 3)])
-def test_route_select_matches_bruteforce(G, M, K):
+def test_route_select_matches_bruteforce(O, G, M, K):
     rng = np.random.default_rng(10 + G * 7 + M + K)
     E = 16
     for ties in (False, True):
@@ -72,7 +72,118 @@ def test_route_select_matches_bruteforce(G, M, K):
             assert list(idx[t]) == want, (t, list(idx[t]), want)
 
 
-def test_no_group_limit_is_plain_topk():
+def _bruteforce_select_int(s_int, b_int, G, M, K):
+    """Exhaustive selection on exact integers: beta = s + b, both given as
+    integer multiples of a common power of two (so every sum is exact).
+    Groups: every C(G, M) subset, scored by the sum over its groups of the
+    best K/M-subset sum of beta; experts: every K-subset of the allowed
+    experts.  Ties: the lexicographically smallest sorted index tuple."""
+    E = len(s_int)
+    beta = [s_int[e] + b_int[e] for e in range(E)]
+    gs = E // G
+    if M < G:
+        n = K // M
+        gscore = [max(sum(beta[e] for e in c) for c in itertools.combinations(range(g * gs, (g + 1) * gs), n))
+                  for g in range(G)]
+        best = max(itertools.combinations(range(G), M),
+                   key=lambda sub: (sum(gscore[g] for g in sub), [-g for g in sub]))
+        allowed = [e for g in sorted(best) for e in range(g * gs, (g + 1) * gs)]
+    else:
+        allowed = list(range(E))
+    best = max(itertools.combinations(allowed, K),
+               key=lambda sub: (sum(beta[e] for e in sub), [-e for e in sub]))
+    return sorted(best, key=lambda e: (-beta[e], e))
+
+
+SCALE = 2 ** 70   # s in (2^-16, 1) has its last bit at or above 2^-69
+
+
+def _as_int(x):
+    """Exact integer multiple of 2^-70 of an fp64 value (asserted exact)."""
+    v = float(x) * SCALE
+    assert v == int(v)
+    return int(v)
+
+
+@pytest.mark.parametrize("G,M,K,seed", [(4, 2, 4, 0), (8, 4, 8, 1), (4, 1, 2, 2), (2, 1, 4, 3)])
+def test_route_select_with_bias_matches_bruteforce(O, G, M, K, seed):
+    """Selection with a non-zero bias b_i ([ANN] eq. (16): the top-K is taken
+    over s_{i,t} + b_i) and the group limit of "Node-Limited Routing", each
+    group ranked by its biased scores.  Exhaustive enumeration over 2500
+    tokens per case (10^4 over the four), on exact integers: s comes from the
+    oracle's sigmoid (pinned against math.exp), b is a multiple of 1/64, and
+    beta = s + b is summed without rounding.  A third of the tokens copy
+    logits and biases between experts and between whole groups, forcing
+    exact ties in beta and in the group scores."""
+    rng = np.random.default_rng(100 + seed)
+    T, E = 2500, 16
+    gs = E // G
+    z = rng.uniform(-6, 6, (T, E))
+    bias = rng.integers(-4, 5, E) / 64.0
+    # forced ties: the same logit (and so the same s) on expert pairs that
+    # share a bias value, and whole groups copied onto another group
+    tied = rng.random(T) < 1 / 3
+    bias[gs:2 * gs] = bias[:gs]
+    for t in np.flatnonzero(tied):
+        z[t, gs:2 * gs] = z[t, :gs]                  # group 1 == group 0, exactly
+        same_b = [(i, j) for i in range(E) for j in range(i + 1, E) if bias[i] == bias[j]]
+        i, j = same_b[rng.integers(len(same_b))]
+        z[t, j] = z[t, i]
+    idx, gate, info = O.route_select(z, bias, G, M, K)
+    s = O.sigmoid(z)
+    b_int = [_as_int(v) for v in bias]
+    n_raw_differs = 0
+    for t in range(T):
+        s_int = [_as_int(v) for v in s[t]]
+        want = _bruteforce_select_int(s_int, b_int, G, M, K)
+        assert list(idx[t]) == want, (t, list(idx[t]), want)
+        # the gates come from the raw affinities of the chosen experts
+        assert np.allclose(gate[t], s[t, want] / s[t, want].sum(), rtol=1e-14, atol=0)
+        if M < G:
+            raw = _bruteforce_select_int(s_int, [0] * E, G, M, K)
+            if set(raw) != set(want):
+                n_raw_differs += 1
+    if M < G:
+        # the bias decides the selection of many tokens, so ranking the groups
+        # or the experts by raw affinity would fail this pin
+        assert n_raw_differs > T // 20, n_raw_differs
+
+
+def test_group_score_uses_the_biased_scores(O):
+    """Hand-built token (E = 8 experts in G = 4 groups of 2, M = 2, K = 2,
+    so each group is scored by its best biased score).  Raw affinities
+    s = (.9, .1 | .8, .1 | .5, .1 | .45, .1) rank the groups 0, 1, 2, 3;
+    a bias of +0.5 on expert 6 makes group 3 score .95 and beat groups 1 and
+    0.  The biased reading selects groups {3, 0} and experts (6, 0): beta
+    .95 > .9.  Ranking groups by raw s would pick groups {0, 1} and experts
+    (0, 2).  The gates are the raw s of the chosen experts normalised:
+    (.45, .9) / 1.35 = (1/3, 2/3)."""
+    s = np.array([0.9, 0.1, 0.8, 0.1, 0.5, 0.1, 0.45, 0.1])
+    z = np.log(s / (1.0 - s))[None, :]
+    b = np.array([0, 0, 0, 0, 0, 0, 0.5, 0.0])
+    idx, gate, _ = O.route_select(z, b, 4, 2, 2)
+    assert list(idx[0]) == [6, 0]
+    assert np.allclose(gate[0], [1 / 3, 2 / 3], rtol=1e-12, atol=0)
+    raw_idx, _, _ = O.route_select(z, b, 4, 2, 2, group_score="raw")
+    assert list(raw_idx[0]) == [0, 2]
+
+
+def test_raw_group_score_fails_the_pin(O):
+    """Negative control: the raw-affinity group ranking (a plausible mistake)
+    disagrees with the exhaustive biased selection on many tokens."""
+    rng = np.random.default_rng(7)
+    T, E, G, M, K = 400, 16, 4, 2, 4
+    z = rng.uniform(-6, 6, (T, E))
+    bias = rng.integers(-4, 5, E) / 64.0
+    idx, _, _ = O.route_select(z, bias, G, M, K, group_score="raw")
+    s = O.sigmoid(z)
+    b_int = [_as_int(v) for v in bias]
+    wrong = sum(list(idx[t]) != _bruteforce_select_int([_as_int(v) for v in s[t]], b_int, G, M, K)
+                for t in range(T))
+    assert wrong > T // 20, wrong
+
+
+def test_no_group_limit_is_plain_topk(O):
     rng = np.random.default_rng(5)
     T, E, K = 200, 64, 6
     z = rng.normal(0, 1, (T, E))
@@ -88,13 +199,13 @@ def test_no_group_limit_is_plain_topk():
     assert np.array_equal(idx, idx2)
 
 
-def test_sigmoid_against_math_exp():
+def test_sigmoid_against_math_exp(O):
     z = np.array([-30.0, -2.5, -1e-3, 0.0, 0.7, 12.0])
     want = np.array([1.0 / (1.0 + math.exp(-v)) for v in z])
     assert np.allclose(O.sigmoid(z), want, rtol=1e-15, atol=0)
 
 
-def test_gates_normalised_and_bias_only_selects():
+def test_gates_normalised_and_bias_only_selects(O):
     rng = np.random.default_rng(6)
     T, E, G, M, K = 300, 32, 4, 2, 4
     z = rng.normal(0, 1, (T, E))
@@ -119,7 +230,7 @@ def test_gates_normalised_and_bias_only_selects():
             assert math.isclose(m0[e], m1[e], rel_tol=2e-15, abs_tol=0)
 
 
-def test_route_with_group_limit_uses_at_most_m_groups():
+def test_route_with_group_limit_uses_at_most_m_groups(O):
     rng = np.random.default_rng(7)
     T, E, G, M, K = 500, 64, 8, 3, 6
     z = rng.normal(0, 1, (T, E))
@@ -130,7 +241,7 @@ def test_route_with_group_limit_uses_at_most_m_groups():
 
 
 # ----------------------------------------------------------- permutation --
-def test_permute_bruteforce():
+def test_permute_bruteforce(O):
     rng = np.random.default_rng(8)
     T, E, K = 97, 12, 3
     idx = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
@@ -148,7 +259,7 @@ def test_permute_bruteforce():
     assert offsets[E] == T * K
 
 
-def test_mtile_table_bruteforce():
+def test_mtile_table_bruteforce(O):
     offs = np.array([0, 0, 5, 133, 261, 262, 600], np.int64)
     grp, start = O.mtile_table(offs)
     want = []
@@ -162,7 +273,7 @@ def test_mtile_table_bruteforce():
 # -------------------------------------------------------------------- GEMM --
 def _exact_block_gemm(aq, sa, bq, sb):
     """D[m][n] = sum_kb sa[m,kb] sb[n/128,kb] sum_k deq(a) deq(b), exactly."""
-    dec = {c: Fraction(float(O.e4m3_decode(np.uint8(c)))) for c in range(256) if c not in (0x7F, 0xFF)}
+    dec = {c: Fraction(float(ONP.e4m3_decode(np.uint8(c)))) for c in range(256) if c not in (0x7F, 0xFF)}
     M, K = aq.shape
     N = bq.shape[0]
     out = np.zeros((M, N))
@@ -176,7 +287,7 @@ def _exact_block_gemm(aq, sa, bq, sb):
     return out
 
 
-def test_grouped_gemm_exact_small():
+def test_grouped_gemm_exact_small(O):
     rng = np.random.default_rng(9)
     K, N = 256, 128
     aq = rng.integers(0, 0x7E, (5, K)).astype(np.uint8) | (rng.integers(0, 2, (5, K)) << 7).astype(np.uint8)
@@ -192,7 +303,7 @@ def test_grouped_gemm_exact_small():
     assert np.allclose(got[2:][:, cols], want1, rtol=1e-13, atol=1e-13)
 
 
-def test_grouped_gemm_integer_operands_exact():
+def test_grouped_gemm_integer_operands_exact(O):
     # codes whose E4M3 values are small integers, unit scales: exact integers
     rng = np.random.default_rng(11)
     ints = {int(v): c for c, v in zip(range(0x7F), O.e4m3_decode(np.arange(0x7F, dtype=np.uint8)))
@@ -207,7 +318,7 @@ def test_grouped_gemm_integer_operands_exact():
     assert np.array_equal(got, want.astype(np.float64))
 
 
-def test_empty_segments_leave_rows_zero():
+def test_empty_segments_leave_rows_zero(O):
     aq = np.full((4, 128), 0x38, np.uint8)       # all 1.0
     bq = np.full((3, 128, 128), 0x38, np.uint8)
     sa = np.ones((4, 1), np.float32)
@@ -217,7 +328,7 @@ def test_empty_segments_leave_rows_zero():
 
 
 # ----------------------------------------------------------------- SwiGLU --
-def test_swiglu_layout_and_values():
+def test_swiglu_layout_and_values(O):
     rng = np.random.default_rng(12)
     I = 256
     gu = rng.normal(0, 2, (3, 2 * I))
@@ -233,7 +344,7 @@ def test_swiglu_layout_and_values():
     assert abs(float(O.silu(-40.0))) < 1e-15
 
 
-def test_swiglu_quant_roundtrip():
+def test_swiglu_quant_roundtrip(O):
     rng = np.random.default_rng(13)
     gu = rng.normal(0, 1, (4, 512)).astype(np.float32)
     q, s = O.swiglu_quant(gu, 256)
@@ -244,7 +355,7 @@ def test_swiglu_quant_roundtrip():
 
 
 # ---------------------------------------------------------------- combine --
-def test_combine_bruteforce():
+def test_combine_bruteforce(O):
     rng = np.random.default_rng(14)
     T, K, d = 5, 3, 8
     Y = rng.normal(0, 1, (T * K, d))
@@ -264,7 +375,7 @@ def test_combine_bruteforce():
 
 
 # ------------------------------------------------------------ bias update --
-def test_bias_update_hand_example():
+def test_bias_update_hand_example(O):
     counts = np.array([3, 1, 2, 2])               # T=2, K=4, E=4: mean load 2
     b = np.array([0.01, -0.02, 0.03, 0.0], np.float32)
     nb = O.bias_update(counts, 2, 4, 0.001, b)
@@ -275,7 +386,7 @@ def test_bias_update_hand_example():
     assert nb[2] == b[2] and nb[3] == b[3]        # at the mean: unchanged
 
 
-def test_bias_update_fp32_exact():
+def test_bias_update_fp32_exact(O):
     rng = np.random.default_rng(15)
     E = 256
     counts = rng.integers(0, 300, E)
@@ -292,7 +403,7 @@ def test_bias_update_fp32_exact():
 
 
 # ----------------------------------------------------------- whole layer --
-def test_tiny_layer_invariants():
+def test_tiny_layer_invariants(O):
     from fp8_block_scaled_sigmoid_b200 import configs, inputs
     cfg = configs.TINY
     inp = inputs.draw_layer(cfg)
@@ -322,7 +433,7 @@ def test_tiny_layer_invariants():
 
 # ----------------------------------------------- sequence-wise balance loss --
 # [ANN] "Complementary Sequence-Wise Auxiliary Loss", eqs. (17)-(20).
-def test_seq_balance_loss_hand_example():
+def test_seq_balance_loss_hand_example(O):
     """Two tokens, three experts, K=1, one sequence, alpha=1.  The logits are
     chosen so the affinities are exact: sigmoid(ln 3) = 3/4, sigmoid(0) = 1/2,
     sigmoid(-ln 3) = 1/4.
@@ -340,7 +451,7 @@ def test_seq_balance_loss_hand_example():
 
 
 @pytest.mark.parametrize("E,K,S", [(4, 2, 4), (16, 4, 8), (64, 8, 16)])
-def test_seq_balance_loss_uniform_affinities(E, K, S):
+def test_seq_balance_loss_uniform_affinities(O, E, K, S):
     """Equal logits: every s' = 1/E, the ties go to experts 0..K-1, so
     f = E/K on them and 0 elsewhere, and L = alpha * K * (E/K) * (1/E) = alpha."""
     z = np.full((2 * S, E), 0.3)
@@ -352,7 +463,7 @@ def test_seq_balance_loss_uniform_affinities(E, K, S):
     assert np.allclose(P, 1.0 / E, rtol=1e-14, atol=0)
 
 
-def test_seq_balance_loss_invariants_and_sequences():
+def test_seq_balance_loss_invariants_and_sequences(O):
     """Random logits: sum_i f_i = N_r (each token counts K experts, scaled by
     N_r/(K T)); sum_i P_i = 1 (each s' row sums to 1); 0 < L <= alpha*N_r/K
     (P sums to 1, f_i <= N_r/K); sequences are independent (the loss of each
