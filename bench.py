@@ -189,6 +189,80 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 200 ms"}
 
 
+# ------------------------------------------------------- FP8 tensor peak ---
+def measure_fp8_peak(dev, block_scaled: bool, launches: int = 8, iters: int = 8192,
+                     sustain_s: float = 0.0) -> dict:
+    """Dense FP8 rate of this GPU, measured live with the library's MMA loop
+    (moe_fp8_mma_peak: one CTA per SM, 128x256x32 E4M3 tcgen05 MMAs from
+    shared memory, no global traffic).  ``block_scaled`` times the
+    kind::mxf8f6f4.block_scale instruction the power-of-two GEMM issues,
+    otherwise the kind::f8f6f4 one of the promoting GEMM.  Burst = the best of
+    ``launches`` separate launches (about 2 ms each at full clock); with
+    sustain_s > 0 the launches also run back to back for that long and the
+    median of the second half is the sustained rate."""
+    import torch
+
+    from fp8_block_scaled_sigmoid_b200 import _abi
+
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sink = torch.empty(sms, dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flops = 0
+    for _ in range(2):
+        flops = _abi.moe_fp8_mma_peak(block_scaled, iters, sms, sink, err)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(launches)]
+    for a, b in ev:
+        torch.cuda.synchronize()
+        a.record()
+        _abi.moe_fp8_mma_peak(block_scaled, iters, sms, sink, err)
+        b.record()
+    torch.cuda.synchronize()
+    burst = max(flops / (a.elapsed_time(b) / 1e3) / 1e12 for a, b in ev)
+    out = {"tflops": round(burst, 1), "kind": "mxf8f6f4.block_scale" if block_scaled
+           else "f8f6f4", "sms": sms, "iters": iters}
+    if sustain_s > 0:
+        rates = []
+        t_end = time.perf_counter() + sustain_s
+        while time.perf_counter() < t_end:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(10):
+                _abi.moe_fp8_mma_peak(block_scaled, iters, sms, sink, err)
+            b.record()
+            b.synchronize()
+            rates.append(10 * flops / (a.elapsed_time(b) / 1e3) / 1e12)
+        tail = rates[len(rates) // 2:]
+        out["sustained_tflops"] = round(statistics.median(tail), 1)
+        out["sustained_s"] = sustain_s
+    _abi.raise_dev_err(err)
+    return out
+
+
+def run_peak(args):
+    """Measure the FP8 tensor peak (both MMA kinds, burst and sustained) with
+    clocks sampled during each, one JSON line."""
+    import torch
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    res = {"metric": "dense FP8 tensor-core TFLOP/s (tcgen05 MMA loop, no global memory)",
+           "unit": "TFLOP/s", "n_gpus": 1}
+    for bs in (False, True):
+        sampler = ClockSampler(0)
+        sampler.start()
+        if sampler.proc is not None:
+            time.sleep(0.3)
+        t0 = time.perf_counter()
+        r = measure_fp8_peak(dev, bs, launches=10, sustain_s=4.0)
+        sampler.window(t0, time.perf_counter())
+        r["clocks"] = sampler.stop()
+        res["block_scaled" if bs else "f8f6f4"] = r
+        time.sleep(2.0)
+    print(json.dumps(res), flush=True)
+
+
 # ------------------------------------------------------- CPU oracle leg ---
 def oracle_sample_rate(cfg, u_host, cent_host, bias_host, expert_weights, route_tokens,
                        ffn_tokens):
@@ -415,7 +489,8 @@ def run_gpu(args):
     t2 = per_kernel["gemm2"] / 1e3
     peaks, peak_src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    fp8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    fp8 = measure_fp8_peak(dev, args.pow2)
+    fp8_peak = fp8["tflops"]
     achieved = g1_bytes / t1 / 1e9
     gemm_name = "grouped_gemm_fp8_pow2" if args.pow2 else "grouped_gemm_fp8"
     traffic = read_traffic(gemm_name, cfg.name)
@@ -433,7 +508,8 @@ def run_gpu(args):
         roofline = {"kernel": f"{gemm_name} (GEMM 1, SwiGLU+quant epilogue)",
                     "bound": "tensor", "achieved": round(tf1, 1), "peak": fp8_peak,
                     "unit": "TFLOP/s", "frac": round(tf1 / fp8_peak, 4), "traffic": traffic,
-                    "peak_source": f"2 x bf16_tflops, {src_note} (nominal fp8:bf16 ratio)",
+                    "peak_source": f"measured in this run: tcgen05 kind::{fp8['kind']} MMA loop, "
+                                   "best of 8 launches (moe_fp8_mma_peak)",
                     "algorithmic_flops": int(g1_flops), "algorithmic_bytes": int(g1_bytes)}
     gemm = {"gemm1_tflops": round(g1_flops / t1 / 1e12, 1),
             "gemm2_tflops": round(g2_flops / t2 / 1e12, 1),
@@ -441,7 +517,8 @@ def run_gpu(args):
             "layer_gemm_tflops": round((g1_flops + g2_flops) / (t1 + t2) / 1e12, 1),
             "fp8_peak_tflops": fp8_peak,
             "frac_fp8_peak": round((g1_flops + g2_flops) / (t1 + t2) / 1e12 / fp8_peak, 4),
-            "fp8_peak_note": "2 x measured bf16 burst (nominal fp8:bf16 ratio)"}
+            "fp8_peak_note": f"measured in this run: tcgen05 kind::{fp8['kind']} MMA loop on all "
+                             f"{fp8['sms']} SMs, best of 8 launches (moe_fp8_mma_peak)"}
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
@@ -597,8 +674,8 @@ def run_gemm(args):
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
     clocks = sampler.stop()
-    peaks, src = load_peaks()
-    fp8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    fp8 = measure_fp8_peak(dev, args.pow2)
+    fp8_peak = fp8["tflops"]
     ms = statistics.median(times)
     tf = cfg.flops / (ms / 1e3) / 1e12
     print(json.dumps({
@@ -612,7 +689,8 @@ def run_gemm(args):
                    "l2": "512 MB buffer written between timed launches"},
         "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4),
-                     "peak_source": f"2 x {src} bf16_tflops (nominal fp8:bf16 ratio)"},
+                     "peak_source": f"measured in this run: tcgen05 kind::{fp8['kind']} MMA "
+                                    "loop, best of 8 launches (moe_fp8_mma_peak)"},
         "clocks": clocks}), flush=True)
 
 
@@ -756,7 +834,7 @@ def run_backward(args):
     ldt = _abi.wgrad_ld(layer.max_tiles)
     peaks, src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    fp8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    fp8_peak = measure_fp8_peak(dev, True)["tflops"]   # Wgrad is block-scaled
     # Wgrad of W1: both token-major operands once, the fp32 gradient of every expert written
     ktot = 128 * int(layer.perm["n_tiles"].item())
     w1_bytes = (2 * cfg.I + cfg.d) * ktot * (1 + 1.0 / 128) + G * 2 * cfg.I * cfg.d * 4
@@ -807,11 +885,15 @@ def main():
                     help="time the backward of the expert FFNs (Dgrad + Wgrad) instead")
     ap.add_argument("--gemm", action="store_true",
                     help="time the standalone 4096x7168x2048 block-scaled GEMM instead")
+    ap.add_argument("--peak", action="store_true",
+                    help="measure the dense FP8 tensor-core peak (MMA loop) instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.peak:
+        run_peak(args)
     elif args.gemm:
         run_gemm(args)
     elif args.backward:

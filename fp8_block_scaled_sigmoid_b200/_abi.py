@@ -59,6 +59,7 @@ _SIGS = {
     "moe_bias_update": (_i, [_p, _i, _i64, _i, _f, _p, _p]),
     "moe_seq_balance_loss_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
     "moe_seq_balance_loss": (_i, [_p, _i, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
+    "moe_fp8_mma_peak": (_i, [_i, _i, _i, _p, _p, _p]),
 }
 
 EP_F32 = 0
@@ -79,7 +80,7 @@ LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant
                      "moe_route": 2, "moe_permute": 4, "moe_permute_noalloc": 4,
                      "moe_tile_table": 1, "moe_segment_ids": 1,
                      "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1,
-                     "moe_seq_balance_loss": 3}
+                     "moe_seq_balance_loss": 3, "moe_fp8_mma_peak": 1}
 launch_count = 0
 
 
@@ -395,6 +396,15 @@ def moe_bias_update(counts, T, K, gamma, bias, stream=None):
     _check(lib().moe_bias_update(_ptr(counts), E, T, K, float(gamma), _ptr(bias),
                                  _stream(stream)), "moe_bias_update")
     return bias
+
+
+def moe_fp8_mma_peak(block_scaled, iters, ctas, sink, dev_err=None, stream=None):
+    """Queue one FP8 MMA-loop launch (the caller times it); sink fp32 [ctas].
+    Returns the launch's FLOP count."""
+    _count("moe_fp8_mma_peak")
+    _check(lib().moe_fp8_mma_peak(int(bool(block_scaled)), int(iters), int(ctas), _ptr(sink),
+                                  _ptr(dev_err), _stream(stream)), "moe_fp8_mma_peak")
+    return ctas * iters * 4 * (2 * 128 * 256 * 32)
 
 
 def read_dev_err(dev_err) -> int:

@@ -422,6 +422,25 @@ moe_status moe_seq_balance_loss(const float* logits, int T, int E, int K, int se
                                 float alpha, float* loss, float* f, float* P, void* ws,
                                 size_t ws_bytes, moe_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * moe_fp8_mma_peak -- measurement helper: the dense FP8 tensor-core rate of
+ * this GPU, the denominator of the expert GEMMs' roofline ([ANN]
+ * "Fine-Grained Quantization": both GEMM operands are E4M3; "Suggestions on
+ * Hardware Design" asks for tensor cores that take the group scales, which
+ * block_scaled = 1 exercises).  One CTA per SM (ctas of them) runs `iters` K
+ * blocks of four 128x256x32 E4M3 tcgen05 MMAs from shared memory into TMEM
+ * and touches no global memory except sink.  block_scaled = 0:
+ * kind::f8f6f4 (what grouped_gemm_fp8_blockscaled issues); 1:
+ * kind::mxf8f6f4.block_scale with unit UE8M0 scales (what
+ * grouped_gemm_fp8_pow2 issues).  The caller times the launch:
+ *   FLOPs = ctas * iters * 4 * (2 * 128 * 256 * 32).
+ *   sink fp32 [ctas] (one accumulator value per CTA, ignore it)
+ * Limits: 1 <= iters <= 2^21 (the kernel's bounded wait is 2 s); a wait that
+ * gives up records MOE_DEVERR_TIMEOUT.
+ */
+moe_status moe_fp8_mma_peak(int block_scaled, int iters, int ctas, float* sink,
+                            int32_t* dev_err, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
