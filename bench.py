@@ -197,7 +197,8 @@ def measure_fp8_peak(dev, block_scaled: bool, launches: int = 8, iters: int = 81
     shared memory, no global traffic).  ``block_scaled`` times the
     kind::mxf8f6f4.block_scale instruction the power-of-two GEMM issues,
     otherwise the kind::f8f6f4 one of the promoting GEMM.  Burst = the best of
-    ``launches`` separate launches (about 2 ms each at full clock); with
+    ``launches`` separate launches (about 2 ms each at full clock, 30 ms
+    apart); with
     sustain_s > 0 the launches also run back to back for that long and the
     median of the second half is the sustained rate."""
     import torch
@@ -215,6 +216,7 @@ def measure_fp8_peak(dev, block_scaled: bool, launches: int = 8, iters: int = 81
           for _ in range(launches)]
     for a, b in ev:
         torch.cuda.synchronize()
+        time.sleep(0.03)          # let the power controller settle between bursts
         a.record()
         _abi.moe_fp8_mma_peak(block_scaled, iters, sms, sink, err)
         b.record()
@@ -265,55 +267,58 @@ def run_peak(args):
 
 # ------------------------------------------------------- CPU oracle leg ---
 def oracle_sample_rate(cfg, u_host, cent_host, bias_host, expert_weights, route_tokens,
-                       ffn_tokens):
-    """Time the oracle on a bounded sample of the layer and return
-    (seconds per token, description).  Route + 1x128 quantisation +
-    permutation + bias update run over ``route_tokens`` tokens; the expert
-    FFNs (routed and shared) and the combine over ``ffn_tokens`` of them.
-    ``expert_weights(e)`` returns the quantised (w1q, w1s, w2q, w2s) of one
-    expert as numpy arrays (weight preparation is not timed, as on the GPU)."""
+                       ffn_tokens: int):
+    """Time the single-threaded C++ oracle (oracle/moe_oracle_ref.cpp, fp64)
+    on a bounded sample of the layer and return (seconds per token,
+    description).  Router logits, selection, 1x128 quantisation, permutation
+    and the bias update run over ``route_tokens`` tokens; the expert FFNs
+    (grouped GEMM 1, SwiGLU + requantisation, grouped GEMM 2; routed and
+    shared) and the combine over the first ``ffn_tokens`` of them, one expert
+    at a time.  ``expert_weights(e)`` returns the quantised (w1q, w1s, w2q,
+    w2s) of one expert as numpy arrays (weight preparation is not timed, as on
+    the GPU)."""
     import numpy as np
-    from oracle import moe_oracle as O
+    from oracle import cpp_oracle as C
 
     ur = u_host[:route_tokens]
     t0 = time.perf_counter()
-    idx, gate, _ = O.route(ur, cent_host, bias_host, cfg.G, cfg.M, cfg.K)
-    xq, xs = O.quant_1x128(ur)
-    counts, offsets, src_row, dst_of = O.permute(idx, cfg.E)
+    idx, gate, _ = C.route(ur, cent_host, bias_host, cfg.G, cfg.M, cfg.K)
+    xq, xs = C.quant_1x128(ur)
+    counts, offsets, src_row, dst_of = C.permute(idx, cfg.E)
     _ = xq[src_row], xs[src_row]
-    O.bias_update(counts, route_tokens, cfg.K, cfg.gamma, bias_host)
+    C.bias_update(counts, route_tokens, cfg.K, cfg.gamma, bias_host)
     t_route = time.perf_counter() - t0
-    # expert FFNs of the sampled tokens, one expert at a time
+    # the sampled tokens' pairs, grouped by expert, plus the shared expert's rows
+    S = ffn_tokens
+    c_s, off_s, src_s, dst_s = C.permute(idx[:S], cfg.E)
+    P = S * cfg.K
+    xq_s = np.concatenate([xq[src_s], xq[:S]])
+    xs_s = np.concatenate([xs[src_s], xs[:S]])
+    offs = C.segment_offsets_with_shared(off_s, S)
+    Y = np.zeros((P + S, cfg.d))
     t_ffn = 0.0
-    for t in ffn_tokens:
-        x = O.dequant_1x128(xq[t:t + 1], xs[t:t + 1])
-        ys = []
-        for e in [cfg.E] + list(idx[t]):
-            w1q, w1s, w2q, w2s = expert_weights(int(e))
-            t1 = time.perf_counter()
-            gu = x @ O.dequant_128x128(w1q, w1s).T
-            hq, hs = O.swiglu_quant(gu, cfg.I)
-            ys.append(O.dequant_1x128(hq, hs) @ O.dequant_128x128(w2q, w2s).T)
-            t_ffn += time.perf_counter() - t1
+    n_exp = 0
+    for e in range(cfg.E + 1):
+        r0, r1 = int(offs[e]), int(offs[e + 1])
+        if r1 == r0:
+            continue
+        w1q, w1s, w2q, w2s = expert_weights(e)
+        n_exp += 1
+        seg = np.array([0, r1 - r0], np.int32)
         t1 = time.perf_counter()
-        Y = np.concatenate(ys[1:])
-        O.combine(Y, np.arange(cfg.K)[None, :], gate[t:t + 1], ys[0], ur[t:t + 1])
+        gu = C.grouped_gemm(xq_s[r0:r1], xs_s[r0:r1], w1q[None], w1s[None], seg)
+        hq, hs = C.swiglu_quant(gu, cfg.I)
+        Y[r0:r1] = C.grouped_gemm(hq, hs, w2q[None], w2s[None], seg)
         t_ffn += time.perf_counter() - t1
-    per_token = t_route / route_tokens + t_ffn / len(ffn_tokens)
-    desc = (f"route+quant+permute+bias-update over {route_tokens} tokens "
-            f"({t_route:.2f} s); expert FFNs ({cfg.K} routed + 1 shared) + combine for "
-            f"{len(ffn_tokens)} token(s) ({t_ffn:.2f} s); rate = 1/(route time per token + "
-            f"FFN time per token)")
+    t1 = time.perf_counter()
+    C.combine(Y[:P], dst_s, gate[:S], Y[P:], ur[:S])
+    t_ffn += time.perf_counter() - t1
+    per_token = t_route / route_tokens + t_ffn / S
+    desc = (f"C++ oracle, 1 thread: logits+select+quant+permute+bias-update over {route_tokens} "
+            f"tokens ({t_route:.2f} s); expert FFNs ({cfg.K} routed + 1 shared per token: "
+            f"{P} + {S} rows over {n_exp} experts) + combine for {S} tokens ({t_ffn:.2f} s); "
+            f"rate = 1/(route time per token + FFN time per token)")
     return per_token, desc
-
-
-def blas_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
 
 
 # ------------------------------------------------------------- GPU arm ---
@@ -574,8 +579,9 @@ def read_traffic(kernel: str, workload: str):
 
 
 def cpu_baseline(cfg, layer, u, bias):
-    import numpy as np
-    import torch
+    """The C++ oracle on the host, one thread, on a bounded sample of the
+    same workload (the layer's own inputs and FP8 weights, copied to the
+    host one expert at a time)."""
     u_h = u.float().cpu().numpy()
     cent_h = layer.centroids.float().cpu().numpy()
     b_h = bias.cpu().numpy()
@@ -584,24 +590,29 @@ def cpu_baseline(cfg, layer, u, bias):
         return (layer.w1q[e].cpu().numpy(), layer.w1s[e].cpu().numpy(),
                 layer.w2q[e].cpu().numpy(), layer.w2s[e].cpu().numpy())
 
-    route_tokens = min(cfg.T, 2048)
-    per_token, desc = oracle_sample_rate(cfg, u_h, cent_h, b_h, weights, route_tokens, [0])
-    return {"value": round(1.0 / per_token, 3), "unit": "tokens/s", "cores": blas_threads(),
-            "kind": "oracle", "sample": desc}
+    per_token, desc = oracle_sample_rate(cfg, u_h, cent_h, b_h, weights, min(cfg.T, 256),
+                                         min(cfg.T, 32))
+    return {"value": round(1.0 / per_token, 3), "unit": "tokens/s", "cores": 1,
+            "host_cpus": os.cpu_count(), "kind": "oracle", "sample": desc}
 
 
 # ------------------------------------------------------- reference arm ---
 def run_reference(args):
+    """The reference arm: the C++ oracle (one thread, fp64) on the host cores,
+    each step a bounded sample of the workload -- the route over 64 tokens,
+    the FFNs and the combine of the first 2.  The FP8 weights of the experts
+    those tokens use are prepared once, before timing (numpy oracle
+    quantiser, as the GPU arm quantises its weights outside the step)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import numpy as np
-
     from fp8_block_scaled_sigmoid_b200 import configs, inputs
+    from oracle import cpp_oracle as C
     from oracle import moe_oracle as O
 
     cfg = configs.PRESETS[args.config]
-    u = inputs.draw_u(cfg).float().numpy()
+    route_tokens, ffn_tokens = min(cfg.T, 64), min(cfg.T, 2)
+    u = inputs.draw_u(cfg).float().numpy()[:route_tokens]
     cent = inputs.draw_centroids(cfg).float().numpy()
     bias = inputs.draw_bias(cfg).numpy()
     cache = {}
@@ -613,27 +624,27 @@ def run_reference(args):
             cache[e] = O.quant_128x128(w1) + O.quant_128x128(w2)
         return cache[e]
 
-    route_tokens = min(cfg.T, 256)
-    # prepare the sampled token's experts before timing
-    idx0, _, _ = O.route(u[:1], cent, bias, cfg.G, cfg.M, cfg.K)
-    for e in [cfg.E] + list(idx0[0]):
+    # prepare the sampled tokens' experts before timing
+    idx0, _, _ = C.route(u[:ffn_tokens], cent, bias, cfg.G, cfg.M, cfg.K)
+    for e in sorted(set(idx0.reshape(-1).tolist()) | {cfg.E}):
         weights(int(e))
     times, desc = [], ""
     for i in range(args.warmup + args.steps):
-        per_token, desc = oracle_sample_rate(cfg, u, cent, bias, weights, route_tokens, [0])
+        per_token, desc = oracle_sample_rate(cfg, u, cent, bias, weights, route_tokens,
+                                             ffn_tokens)
         if i >= args.warmup:
             times.append(per_token)
     per_token = sum(times) / len(times)
     value = 1.0 / per_token
-    cb = {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-          "sample": desc}
+    cb = {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "host_cpus": os.cpu_count(),
+          "kind": "oracle", "sample": desc}
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(per_token * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
         "config": {"workload": workload_name(cfg), "tokens_per_gpu": cfg.T,
-                   "parallelism": "CPU oracle, rank 0 only"},
+                   "parallelism": "CPU oracle (C++, one thread), rank 0 only"},
         "cpu_baseline": cb,
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
