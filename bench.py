@@ -457,26 +457,43 @@ def run_gpu(args):
     e2e_value = tokens / (e2e_ms / 1e3)
     out_host = out_hosts[0]
 
-    # the sequence-wise balance loss (eqs. 17-20) of this batch's router logits,
-    # one sequence of T tokens; off the step (a training-time reduction)
+    # the sequence-wise balance loss (eqs. 17-20) of this batch, one sequence
+    # of T tokens: its per-token rows come out of the router's selection pass
+    # (aux_rows), two short reductions finish it.  Its cost is the route with
+    # the rows minus the route without them, plus the reductions; the
+    # three-pass form from kept logits is timed beside it.
     logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
-    _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K, logits_out=logits)
+    rows = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
+    rws = torch.empty(max(_abi.moe_route_workspace_size(cfg.T, cfg.d, cfg.E), 16),
+                      dtype=torch.uint8, device=dev)
     bl_ws = torch.empty(max(_abi.moe_seq_balance_loss_ws(cfg.T, cfg.E, cfg.T), 16),
                         dtype=torch.uint8, device=dev)
-    for _ in range(3):
-        _abi.moe_seq_balance_loss(logits, cfg.K, cfg.T, ws=bl_ws)
-    bl0, bl1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    bl0.record(st)
-    for _ in range(args.steps):
-        _abi.moe_seq_balance_loss(logits, cfg.K, cfg.T, ws=bl_ws)
-    bl1.record(st)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(st)
+        for _ in range(n):
+            fn()
+        b_.record(st)
+        b_.synchronize()
+        return a_.elapsed_time(b_) * 1e3 / n
+
+    reps = max(args.steps, 10)
+    t_plain = timed(lambda: _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K,
+                                           ws=rws), reps)
+    t_aux = timed(lambda: _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K,
+                                         ws=rws, aux_rows=rows), reps)
+    t_red = timed(lambda: _abi.moe_seq_balance_loss_rows(rows, cfg.K, cfg.T, ws=bl_ws), reps)
+    _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K, logits_out=logits, ws=rws)
+    t_3p = timed(lambda: _abi.moe_seq_balance_loss(logits, cfg.K, cfg.T, ws=bl_ws), reps)
     barrier()
-    bl_us = bl0.elapsed_time(bl1) * 1e3 / args.steps
-    # logits read twice, normalised rows written once and read once
-    bl_bytes = 4 * cfg.T * cfg.E * 4
-    balance_loss = {"us": round(bl_us, 2), "seq_len": cfg.T, "bytes": bl_bytes,
-                    "gbs": round(bl_bytes / (bl_us * 1e-6) / 1e9, 1)}
-    del logits, bl_ws
+    balance_loss = {"extra_us": round(t_aux - t_plain + t_red, 2),
+                    "route_us": round(t_plain, 2), "route_with_rows_us": round(t_aux, 2),
+                    "reductions_us": round(t_red, 2), "three_pass_from_logits_us": round(t_3p, 2),
+                    "seq_len": cfg.T}
+    del logits, rows, rws, bl_ws
 
     # roofline of the dominant kernel (grouped GEMM 1 with the SwiGLU epilogue)
     counts = layer.perm["counts"].cpu()
@@ -718,7 +735,7 @@ def run_ep(args, cfg, cfg_rank, dev, pg, world, rank, local):
     from fp8_block_scaled_sigmoid_b200.layer import make_fp8_weights, max_over_ranks
 
     shard = ep.ExpertShard(cfg.E, world, rank)
-    experts = list(range(shard.e0, shard.e1)) + [cfg.E + i for i in range(cfg.n_shared)]
+    experts = [cfg.E] + list(range(shard.e0, shard.e1))      # the shared expert first
     w = make_fp8_weights(cfg, dev, experts=experts)
     layer = ep.MoELayerEP(cfg, inputs.draw_centroids(cfg, dev), inputs.draw_bias(cfg, dev), *w,
                           shard, process_group=pg)

@@ -32,7 +32,8 @@ _SIGS = {
     "fp8_quant_1x128_pow2": (_i, [_p, _i64, _i, _i, _p, _p, _p]),
     "fp8_quant_128x128_pow2": (_i, [_p, _i64, _i, _i, _p, _p, _p]),
     "moe_route_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
-    "moe_route": (_i, [_p, _i64, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _sz, _p, _p]),
+    "moe_route": (_i, [_p, _i64, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p,
+                       _p]),
     "moe_max_m_tiles": (_i, [_i, _i, _i, _i]),
     "moe_permute_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
     "moe_permute": (_i, [_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p,
@@ -40,11 +41,11 @@ _SIGS = {
     "moe_permute_noalloc": (_i, [_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p,
                                  _p, _p, _p, _p]),
     "moe_tile_table": (_i, [_p, _i, _i, _p, _p, _p, _p, _p]),
-    "moe_segment_ids": (_i, [_p, _i, _i, _i64, _p, _p, _p]),
+    "moe_segment_ids": (_i, [_p, _i, _i, _i64, _i64, _p, _p, _p]),
     "grouped_gemm_fp8_blockscaled": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
-                                          _i, _p, _p, _p, _p]),
+                                          _i, _p, _p, _p, _p, _p]),
     "grouped_gemm_fp8_pow2": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
-                                   _i, _p, _p, _p, _p]),
+                                   _i, _p, _p, _p, _p, _p]),
     "swiglu_quant": (_i, [_p, _i, _i, _p, _p, _p]),
     "swiglu_quant_pow2": (_i, [_p, _i, _i, _p, _p, _p]),
     "fp8_quant_1x128_f32": (_i, [_p, _i64, _i, _i, _i, _p, _p, _p]),
@@ -60,6 +61,8 @@ _SIGS = {
     "moe_seq_balance_loss_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
     "moe_seq_balance_loss": (_i, [_p, _i, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
     "moe_fp8_mma_peak": (_i, [_i, _i, _i, _p, _p, _p]),
+    "moe_seq_balance_loss_rows_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
+    "moe_seq_balance_loss_rows": (_i, [_p, _i, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
 }
 
 EP_F32 = 0
@@ -80,7 +83,8 @@ LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant
                      "moe_route": 2, "moe_permute": 4, "moe_permute_noalloc": 4,
                      "moe_tile_table": 1, "moe_segment_ids": 1,
                      "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1,
-                     "moe_seq_balance_loss": 3, "moe_fp8_mma_peak": 1}
+                     "moe_seq_balance_loss": 3, "moe_fp8_mma_peak": 1,
+                     "moe_seq_balance_loss_rows": 2}
 launch_count = 0
 
 
@@ -191,7 +195,7 @@ def moe_route_workspace_size(T, d, E) -> int:
 
 
 def moe_route(u, centroids, bias, G, M, K, topk_idx=None, topk_gate=None, logits_out=None,
-              ws=None, dev_err=None, stream=None):
+              ws=None, dev_err=None, stream=None, aux_rows=None):
     T, d = u.shape
     E = centroids.shape[0]
     dev = _dev(u)
@@ -202,8 +206,9 @@ def moe_route(u, centroids, bias, G, M, K, topk_idx=None, topk_gate=None, logits
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     _count("moe_route")
     _check(lib().moe_route(_ptr(u), u.stride(0), _ptr(centroids), _ptr(bias), T, d, E, G, M, K,
-                           _ptr(topk_idx), _ptr(topk_gate), _ptr(logits_out), _ptr(ws),
-                           ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream)),
+                           _ptr(topk_idx), _ptr(topk_gate), _ptr(logits_out), _ptr(aux_rows),
+                           _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_err),
+                           _stream(stream)),
            "moe_route")
     return topk_idx, topk_gate
 
@@ -310,23 +315,26 @@ def moe_tile_table(offsets, max_tiles, tile_group=None, tile_start=None, n_tiles
     return tile_group, tile_start, n_tiles
 
 
-def moe_segment_ids(counts, E, n_rows, ids=None, dev_err=None, stream=None):
+def moe_segment_ids(counts, E, n_rows, ids=None, dev_err=None, stream=None, lead_rows=0):
     """counts int32 [sources][E] (or flat) -> ids int32 [n_rows]: the local
-    expert of every row of a source-major, expert-sorted receive buffer."""
+    expert of every row of a source-major, expert-sorted receive buffer; with
+    lead_rows > 0 the first lead_rows rows are group 0 and the received rows
+    after them get 1 + their expert."""
     c = counts.reshape(-1)
     ids = torch.empty(n_rows, dtype=torch.int32, device=_dev(counts)) if ids is None else ids
     _count("moe_segment_ids")
-    _check(lib().moe_segment_ids(_ptr(c), c.numel(), E, n_rows, _ptr(ids), _ptr(dev_err),
-                                 _stream(stream)), "moe_segment_ids")
+    _check(lib().moe_segment_ids(_ptr(c), c.numel(), E, lead_rows, n_rows, _ptr(ids),
+                                 _ptr(dev_err), _stream(stream)), "moe_segment_ids")
     return ids
 
 
 # ------------------------------------------------------------------ GEMM ---
 def grouped_gemm_fp8_blockscaled(A, sa, B, sb, offsets, tile_group, tile_start, n_tiles,
                                  max_tiles, ep=EP_F32, D=None, d_scale=None, dev_err=None,
-                                 stream=None, pow2=False):
+                                 stream=None, pow2=False, d_rows=None):
     """A uint8 [rows][K], sa fp32 [rows][K/128], B uint8 [G][N][K], sb fp32
-    [G][N/128][K/128].  ep=EP_F32 -> D fp32 [rows][N]; ep=EP_SWIGLU_QUANT ->
+    [G][N/128][K/128].  ep=EP_F32 -> D fp32 [rows][N] (d_rows int32 [rows]
+    optionally sends row j's output to D row d_rows[j]); ep=EP_SWIGLU_QUANT ->
     (h uint8 [rows][N/2], h_scale fp32 [rows][N/256]).  pow2 calls
     grouped_gemm_fp8_pow2 (every scale a power of two; the tensor core
     applies them)."""
@@ -342,7 +350,8 @@ def grouped_gemm_fp8_blockscaled(A, sa, B, sb, offsets, tile_group, tile_start, 
     _count(name)
     _check(getattr(lib(), name)(_ptr(A), _ptr(sa), rows, _ptr(B), _ptr(sb), _ptr(offsets),
                                 _ptr(tile_group), _ptr(tile_start), _ptr(n_tiles), max_tiles, G,
-                                N, K, ep, _ptr(D), _ptr(d_scale), _ptr(dev_err), _stream(stream)),
+                                N, K, ep, _ptr(D), _ptr(d_scale), _ptr(d_rows), _ptr(dev_err),
+                                _stream(stream)),
            name)
     return D if ep == EP_F32 else (D, d_scale)
 
@@ -390,7 +399,39 @@ def moe_seq_balance_loss(logits, K, seq_len, alpha=1e-4, with_fp=False, ws=None,
     return loss
 
 
+def moe_seq_balance_loss_rows_ws(T, E, seq_len) -> int:
+    n = _sz(0)
+    _check(lib().moe_seq_balance_loss_rows_workspace_size(T, E, seq_len, ctypes.byref(n)),
+           "moe_seq_balance_loss_rows_workspace_size")
+    return n.value
+
+
+def moe_seq_balance_loss_rows(rows, K, seq_len, alpha=1e-4, with_fp=False, ws=None, stream=None):
+    """The balance loss from moe_route's aux_rows fp32 [T][E] (K = the routing
+    K).  Returns loss fp32 [T/seq_len], or (loss, f, P) with with_fp."""
+    T, E = rows.shape
+    dev = _dev(rows)
+    n_seq = T // seq_len if seq_len > 0 else 0
+    loss = torch.empty(max(n_seq, 1), dtype=torch.float32, device=dev)
+    f = torch.empty(max(n_seq, 1), E, dtype=torch.float32, device=dev) if with_fp else None
+    P = torch.empty(max(n_seq, 1), E, dtype=torch.float32, device=dev) if with_fp else None
+    need = moe_seq_balance_loss_rows_ws(T, E, seq_len)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _count("moe_seq_balance_loss_rows")
+    _check(lib().moe_seq_balance_loss_rows(_ptr(rows), T, E, K, seq_len, float(alpha), _ptr(loss),
+                                           _ptr(f), _ptr(P), _ptr(ws),
+                                           ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_seq_balance_loss_rows")
+    loss = loss[:n_seq]
+    if with_fp:
+        return loss, f[:n_seq], P[:n_seq]
+    return loss
+
+
 def moe_bias_update(counts, T, K, gamma, bias, stream=None):
+    if counts.dtype != torch.int32 or bias.dtype != torch.float32:
+        raise MoEError("moe_bias_update: counts must be int32 and bias fp32")
     E = counts.numel()
     _count("moe_bias_update")
     _check(lib().moe_bias_update(_ptr(counts), E, T, K, float(gamma), _ptr(bias),

@@ -217,3 +217,46 @@ extern "C" moe_status moe_seq_balance_loss(const float* logits, int T, int E, in
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }
+
+extern "C" moe_status moe_seq_balance_loss_rows_workspace_size(int T, int E, int seq_len,
+                                                                size_t* bytes) {
+  using namespace moe;
+  if (!bytes || T < 0 || E <= 0 || seq_len <= 0) return MOE_ERR_INVALID_ARG;
+  const int64_t chunks = static_cast<int64_t>(T / seq_len) * ((seq_len + kAuxChunk - 1) / kAuxChunk);
+  *bytes = align256(static_cast<size_t>(chunks) * E * sizeof(float)) +
+           align256(static_cast<size_t>(chunks) * E * sizeof(int32_t));
+  return MOE_OK;
+}
+
+// The loss from the per-token rows moe_route wrote (aux_rows): the chunk and
+// final passes of moe_seq_balance_loss, without its token pass.
+extern "C" moe_status moe_seq_balance_loss_rows(const float* rows, int T, int E, int K,
+                                                int seq_len, float alpha, float* loss,
+                                                float* f_out, float* p_out, void* ws,
+                                                size_t ws_bytes, moe_stream_t stream) {
+  using namespace moe;
+  if (T < 0 || E <= 0 || K <= 0 || seq_len <= 0) return MOE_ERR_INVALID_ARG;
+  if (K > E || K > 32 || T % seq_len != 0) return MOE_ERR_SHAPE;
+  if (E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!rows || !loss) return MOE_ERR_INVALID_ARG;
+  size_t need = 0;
+  moe_seq_balance_loss_rows_workspace_size(T, E, seq_len, &need);
+  if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int n_seq = T / seq_len;
+  const int cps = (seq_len + kAuxChunk - 1) / kAuxChunk;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* psum = reinterpret_cast<float*>(w);
+  w += align256(static_cast<size_t>(n_seq) * cps * E * sizeof(float));
+  int32_t* pcnt = reinterpret_cast<int32_t*>(w);
+  const int ethreads = (E + 31) / 32 * 32;
+  aux_chunk_kernel<<<n_seq * cps, ethreads, 0, st>>>(rows, E, seq_len, cps, psum, pcnt);
+  MOE_CUDA_CHECK_LAUNCH();
+  int fthreads = 32;
+  while (fthreads < E) fthreads <<= 1;
+  aux_final_kernel<<<n_seq, fthreads, fthreads * sizeof(float), st>>>(
+      psum, pcnt, E, K, seq_len, cps, alpha, loss, f_out, p_out);
+  MOE_CUDA_CHECK_LAUNCH();
+  return MOE_OK;
+}

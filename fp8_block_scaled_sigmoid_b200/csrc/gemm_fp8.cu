@@ -75,6 +75,7 @@ struct GemmArgs {
   void* D;
   float* d_scale;
   int32_t* dev_err;
+  const int32_t* d_rows;  // fp32 epilogue: output row of A row j (NULL: row j)
 };
 
 struct Work {
@@ -144,8 +145,23 @@ __device__ __forceinline__ bool write_tile(const GemmArgs& args, const Work& t, 
     // instruction writes 4 rows x 128 contiguous bytes (whole lines).
     const int li = lane & 7;
     const int rb = r_in - li;  // first row of this lane's group inside the tile
-    float* base = static_cast<float*>(args.D) + (static_cast<int64_t>(t.row0) + rb) * N +
-                  t.n_idx * kBN + 128 * g + 4 * li;
+    // output row of each of the group's 8 rows: the tile's own rows, or the
+    // caller's row map (lane rb + j reads row rb + j's entry and the group's
+    // lanes exchange them); a bad map entry skips its row
+    int my_drow = -1;
+    if (args.d_rows != nullptr && row_ok) {
+      my_drow = __ldg(args.d_rows + arow);
+      if (static_cast<uint32_t>(my_drow) >= static_cast<uint32_t>(args.a_rows)) {
+        set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
+        my_drow = -1;
+      }
+    }
+    int drow[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      drow[j] = args.d_rows != nullptr ? __shfl_sync(0xffffffffu, my_drow, (lane & ~7) | j)
+                                       : t.row0 + rb + j;
+    float* const D0 = static_cast<float*>(args.D) + t.n_idx * kBN + 128 * g + 4 * li;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       float4 e[8];  // e[j] = columns 32b + 4j .. 32b + 4j + 3 of this lane's row
@@ -176,8 +192,8 @@ __device__ __forceinline__ bool write_tile(const GemmArgs& args, const Work& t, 
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (rb + j < t.rows)
-          *reinterpret_cast<float4*>(base + static_cast<int64_t>(j) * N + 32 * b) = e[j];
+        if (rb + j < t.rows && drow[j] >= 0)
+          *reinterpret_cast<float4*>(D0 + static_cast<int64_t>(drow[j]) * N + 32 * b) = e[j];
     }
   } else {
     // h = SiLU(gate) * up overwrites the gate accumulators: h[2i], h[2i+1]
@@ -928,12 +944,13 @@ moe_status gemm_launch(bool pow2, const uint8_t* A, const float* sa, int64_t a_r
                        const uint8_t* B, const float* sb, const int32_t* offsets,
                        const int32_t* tile_group, const int32_t* tile_start,
                        const int32_t* n_tiles, int max_tiles, int groups, int N, int K,
-                       moe_epilogue ep, void* D, float* d_scale, int32_t* dev_err,
-                       moe_stream_t stream) {
+                       moe_epilogue ep, void* D, float* d_scale, const int32_t* d_rows,
+                       int32_t* dev_err, moe_stream_t stream) {
   using namespace moe;
   if (a_rows < 0 || groups <= 0 || N <= 0 || K <= 0 || max_tiles < 0) return MOE_ERR_INVALID_ARG;
   if (K % kBK != 0 || N % kBN != 0) return MOE_ERR_SHAPE;
   if (ep != MOE_EP_F32 && ep != MOE_EP_SWIGLU_QUANT) return MOE_ERR_INVALID_ARG;
+  if (d_rows != nullptr && ep != MOE_EP_F32) return MOE_ERR_INVALID_ARG;
   if (a_rows == 0 || max_tiles == 0) return MOE_OK;
   if (!A || !sa || !B || !sb || !offsets || !tile_group || !tile_start || !n_tiles || !D)
     return MOE_ERR_INVALID_ARG;
@@ -966,6 +983,7 @@ moe_status gemm_launch(bool pow2, const uint8_t* A, const float* sa, int64_t a_r
   a.D = D;
   a.d_scale = d_scale;
   a.dev_err = dev_err;
+  a.d_rows = d_rows;
   static int configured = 0;
   if (!configured) {
     const void* fs[4] = {kernel_ptr<MOE_EP_F32>(), kernel_ptr<MOE_EP_SWIGLU_QUANT>(),
@@ -1001,18 +1019,18 @@ extern "C" moe_status grouped_gemm_fp8_blockscaled(
     const uint8_t* A, const float* sa, int64_t a_rows, const uint8_t* B, const float* sb,
     const int32_t* offsets, const int32_t* tile_group, const int32_t* tile_start,
     const int32_t* n_tiles, int max_tiles, int groups, int N, int K, moe_epilogue ep, void* D,
-    float* d_scale, int32_t* dev_err, moe_stream_t stream) {
+    float* d_scale, const int32_t* d_rows, int32_t* dev_err, moe_stream_t stream) {
   return gemm_launch(false, A, sa, a_rows, B, sb, offsets, tile_group, tile_start, n_tiles,
-                     max_tiles, groups, N, K, ep, D, d_scale, dev_err, stream);
+                     max_tiles, groups, N, K, ep, D, d_scale, d_rows, dev_err, stream);
 }
 
 extern "C" moe_status grouped_gemm_fp8_pow2(
     const uint8_t* A, const float* sa, int64_t a_rows, const uint8_t* B, const float* sb,
     const int32_t* offsets, const int32_t* tile_group, const int32_t* tile_start,
     const int32_t* n_tiles, int max_tiles, int groups, int N, int K, moe_epilogue ep, void* D,
-    float* d_scale, int32_t* dev_err, moe_stream_t stream) {
+    float* d_scale, const int32_t* d_rows, int32_t* dev_err, moe_stream_t stream) {
   return gemm_launch(true, A, sa, a_rows, B, sb, offsets, tile_group, tile_start, n_tiles,
-                     max_tiles, groups, N, K, ep, D, d_scale, dev_err, stream);
+                     max_tiles, groups, N, K, ep, D, d_scale, d_rows, dev_err, stream);
 }
 
 extern "C" moe_status grouped_gemm_fp8_wgrad(const uint8_t* At, const uint8_t* sfa_atoms,

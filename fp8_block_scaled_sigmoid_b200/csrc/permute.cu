@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kScanThreads) tile_table_kernel(
 constexpr int kSegRowsPerCta = 4096;
 
 __global__ void __launch_bounds__(kScanThreads) segment_ids_kernel(
-    const int32_t* __restrict__ counts, int nseg, int E, int64_t n_rows,
+    const int32_t* __restrict__ counts, int nseg, int E, int64_t lead, int64_t n_rows,
     int32_t* __restrict__ ids, int32_t* dev_err) {
   __shared__ int64_t incl[kScanThreads];
   const int t = threadIdx.x;
@@ -266,24 +266,31 @@ __global__ void __launch_bounds__(kScanThreads) segment_ids_kernel(
   }
   incl[t] = c;
   __syncthreads();
-  for (int d = 1; d < kScanThreads; d <<= 1) {
+  // inclusive scan over the segments actually present (log2 of their count
+  // rounded up steps)
+  for (int d = 1; d < nseg; d <<= 1) {
     const int64_t v = t >= d ? incl[t - d] : 0;
     __syncthreads();
     incl[t] += v;
     __syncthreads();
   }
-  if (blockIdx.x == 0 && t == 0 && incl[kScanThreads - 1] != n_rows)
-    set_dev_err(dev_err, MOE_DEVERR_BAD_TABLE);
+  if (t == 0 && incl[nseg - 1] + lead != n_rows) set_dev_err(dev_err, MOE_DEVERR_BAD_TABLE);
+  const int shift = lead > 0 ? 1 : 0;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kSegRowsPerCta;
   for (int64_t r = r0 + t; r < n_rows && r < r0 + kSegRowsPerCta; r += kScanThreads) {
-    // first segment whose inclusive end exceeds r
+    if (r < lead) {
+      ids[r] = 0;
+      continue;
+    }
+    const int64_t rr = r - lead;
+    // first segment whose inclusive end exceeds rr
     int lo = 0, hi = nseg - 1;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (incl[mid] > r) hi = mid;
+      if (incl[mid] > rr) hi = mid;
       else lo = mid + 1;
     }
-    ids[r] = lo % E;
+    ids[r] = shift + lo % E;
   }
 }
 
@@ -351,10 +358,11 @@ extern "C" moe_status moe_permute(const int32_t* topk_idx, int T, int K, int E, 
 }
 
 extern "C" moe_status moe_segment_ids(const int32_t* counts, int n_segments, int E,
-                                      int64_t n_rows, int32_t* ids, int32_t* dev_err,
-                                      moe_stream_t stream) {
+                                      int64_t lead_rows, int64_t n_rows, int32_t* ids,
+                                      int32_t* dev_err, moe_stream_t stream) {
   using namespace moe;
-  if (n_segments <= 0 || E <= 0 || n_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (n_segments <= 0 || E <= 0 || n_rows < 0 || lead_rows < 0 || lead_rows > n_rows)
+    return MOE_ERR_INVALID_ARG;
   if (n_segments % E != 0) return MOE_ERR_SHAPE;
   if (n_segments > kScanThreads) return MOE_ERR_UNSUPPORTED;
   if (n_rows == 0) return MOE_OK;
@@ -362,8 +370,8 @@ extern "C" moe_status moe_segment_ids(const int32_t* counts, int n_segments, int
   const int64_t ctas = (n_rows + kSegRowsPerCta - 1) / kSegRowsPerCta;
   if (ctas > 0x7FFFFFFF) return MOE_ERR_UNSUPPORTED;
   segment_ids_kernel<<<static_cast<unsigned>(ctas), kScanThreads, 0,
-                       static_cast<cudaStream_t>(stream)>>>(counts, n_segments, E, n_rows, ids,
-                                                             dev_err);
+                       static_cast<cudaStream_t>(stream)>>>(counts, n_segments, E, lead_rows,
+                                                             n_rows, ids, dev_err);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }

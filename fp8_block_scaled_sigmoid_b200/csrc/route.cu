@@ -175,6 +175,65 @@ __device__ __forceinline__ Cand warp_best(Cand c) {
   return c;
 }
 
+// The balance loss's per-token row ("Complementary Sequence-Wise Auxiliary
+// Loss", eqs. (17)-(20)) from the raw affinities s this warp already holds:
+// s' = s / sum_j s_j (the sum in a fixed order: each lane's experts in turn,
+// then a butterfly over the lanes) and the raw top-K of s over all E experts
+// (ties to the lower index, no bias, no group limit); writes s' with the sign
+// bit set on the K members (s' > 0, so the sign carries the membership).
+// The arithmetic and orders are those of moe_seq_balance_loss's token pass,
+// so both give the same bytes.
+template <int P>
+__device__ __forceinline__ void aux_token_row(const float (&s)[P], int t, int E, int K, int lane,
+                                              float* __restrict__ rows) {
+  const int e0 = lane * P;
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+    if (e0 + i < E) sum = __fadd_rn(sum, s[i]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
+  uint32_t taken = 0;
+  int bi = -1;
+  float bv = 0.f;
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+    if (e0 + i < E && (bi < 0 || s[i] > bv)) {
+      bi = i;
+      bv = s[i];
+    }
+  for (int k = 0; k < K; ++k) {
+    uint32_t key = bi < 0 ? 0u : __float_as_uint(bv);  // s > 0 orders like its bits
+    int ex = bi < 0 ? INT_MAX : e0 + bi;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const uint32_t ok = __shfl_xor_sync(0xffffffffu, key, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, ex, off);
+      if (ok > key || (ok == key && oe < ex)) {
+        key = ok;
+        ex = oe;
+      }
+    }
+    if (ex / P == lane) {
+      taken |= 1u << (ex - e0);
+      bi = -1;
+      bv = 0.f;
+#pragma unroll
+      for (int i = 0; i < P; ++i)
+        if (e0 + i < E && !((taken >> i) & 1u) && (bi < 0 || s[i] > bv)) {
+          bi = i;
+          bv = s[i];
+        }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+    if (e0 + i < E) {
+      const float v = __fdiv_rn(s[i], sum);
+      rows[static_cast<int64_t>(t) * E + e0 + i] = ((taken >> i) & 1u) ? -v : v;
+    }
+}
+
 constexpr int kSelThreads = 256;
 
 // P = experts per lane (lane l owns experts l*P .. l*P+P-1).
@@ -182,7 +241,7 @@ template <int P>
 __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
     const float* __restrict__ part, int splits, int T, int E, int G, int M, int K,
     const float* __restrict__ bias, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
-    float* __restrict__ logits_out) {
+    float* __restrict__ logits_out, float* __restrict__ aux_rows) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (kSelThreads / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -364,14 +423,15 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
     idx_out[static_cast<int64_t>(t) * K + lane] = my_idx;
     gate_out[static_cast<int64_t>(t) * K + lane] = __fdiv_rn(my_s, ssum);
   }
+  if (aux_rows != nullptr) aux_token_row<P>(sc, t, E, K, lane, aux_rows);
 }
 
 template <int P>
 void launch_select(int blocks, cudaStream_t st, const float* part, int splits, int T, int E,
                    int G, int M, int K, const float* bias, int32_t* idx, float* gate,
-                   float* logits) {
+                   float* logits, float* aux) {
   route_select_kernel<P><<<blocks, kSelThreads, 0, st>>>(part, splits, T, E, G, M, K, bias, idx,
-                                                          gate, logits);
+                                                          gate, logits, aux);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -390,8 +450,9 @@ extern "C" moe_status moe_route_workspace_size(int T, int d, int E, size_t* byte
 
 extern "C" moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* centroids,
                                 const float* bias, int T, int d, int E, int G, int M, int K,
-                                int32_t* topk_idx, float* topk_gate, float* logits_out, void* ws,
-                                size_t ws_bytes, int32_t* dev_err, moe_stream_t stream) {
+                                int32_t* topk_idx, float* topk_gate, float* logits_out,
+                                float* aux_rows, void* ws, size_t ws_bytes, int32_t* dev_err,
+                                moe_stream_t stream) {
   using namespace moe;
   if (T < 0 || d <= 0 || E <= 0 || G <= 0 || M <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
   if (d % 128 != 0 || E % 16 != 0 || E % G != 0 || M > G || K > E || ldu < d) return MOE_ERR_SHAPE;
@@ -428,13 +489,13 @@ extern "C" moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* 
 
   const int blocks = (T + kSelThreads / 32 - 1) / (kSelThreads / 32);
   const int P = (E + 31) / 32;
-  if (P <= 1) launch_select<1>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
-  else if (P <= 2) launch_select<2>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
-  else if (P <= 4) launch_select<4>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
-  else if (P <= 8) launch_select<8>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
-  else if (P <= 12) launch_select<12>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
-  else if (P <= 16) launch_select<16>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
-  else launch_select<32>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out);
+  if (P <= 1) launch_select<1>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
+  else if (P <= 2) launch_select<2>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
+  else if (P <= 4) launch_select<4>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
+  else if (P <= 8) launch_select<8>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
+  else if (P <= 12) launch_select<12>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
+  else if (P <= 16) launch_select<16>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
+  else launch_select<32>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }

@@ -102,7 +102,7 @@ class MoELayer:
 
     def __init__(self, cfg: MoEConfig, centroids: torch.Tensor, bias: torch.Tensor,
                  w1q, w1s, w2q, w2s, T: int | None = None, process_group=None,
-                 keep_logits: bool = False, pow2: bool = False):
+                 keep_logits: bool = False, pow2: bool = False, balance_loss: bool = False):
         self.cfg = cfg
         self.pow2 = pow2
         self.T = cfg.T if T is None else T
@@ -117,8 +117,10 @@ class MoELayer:
         dev = self.dev
         i32, f32, u8 = torch.int32, torch.float32, torch.uint8
         self.idx = torch.empty(T, K, dtype=i32, device=dev)
-        # router logits of the last step, kept for seq_balance_loss
+        # router logits of the last step (keep_logits), and the balance loss's
+        # per-token rows written by the router's selection pass (balance_loss)
         self.logits = torch.empty(T, E, dtype=f32, device=dev) if keep_logits else None
+        self.aux_rows = torch.empty(T, E, dtype=f32, device=dev) if balance_loss else None
         self.gate = torch.empty(T, K, dtype=f32, device=dev)
         self.route_ws = torch.empty(max(_abi.moe_route_workspace_size(T, d, E), 16), dtype=u8, device=dev)
         self.Xq = torch.empty(P + T, d, dtype=u8, device=dev)
@@ -144,7 +146,8 @@ class MoELayer:
     def step_route(self, u):
         c = self.cfg
         _abi.moe_route(u, self.centroids, self.bias, c.G, c.M, c.K, self.idx, self.gate,
-                       logits_out=self.logits, ws=self.route_ws, dev_err=self.dev_err)
+                       logits_out=self.logits, ws=self.route_ws, dev_err=self.dev_err,
+                       aux_rows=self.aux_rows)
 
     def step_quant(self, u):
         _abi.fp8_quant_1x128(u, self.Xq[self.pairs:], self.Xs[self.pairs:], pow2=self.pow2)
@@ -291,9 +294,14 @@ class MoELayer:
 
     def seq_balance_loss(self, seq_len: int, alpha: float = 1e-4, with_fp: bool = False):
         """The complementary sequence-wise balance loss (eqs. 17-20) of the
-        last step's router logits, per sequence of seq_len tokens (the layer
-        must be built with keep_logits=True)."""
-        assert self.logits is not None, "build the layer with keep_logits=True"
+        last step's routing, per sequence of seq_len tokens.  With
+        balance_loss=True the router's selection pass already wrote the
+        per-token rows and two short reductions finish the loss; with
+        keep_logits=True the loss is computed from the kept logits."""
+        if self.aux_rows is not None:
+            return _abi.moe_seq_balance_loss_rows(self.aux_rows, self.cfg.K, seq_len, alpha,
+                                                  with_fp)
+        assert self.logits is not None, "build the layer with balance_loss or keep_logits"
         return _abi.moe_seq_balance_loss(self.logits, self.cfg.K, seq_len, alpha, with_fp)
 
     def capture(self, u: torch.Tensor, update_bias: bool = True):

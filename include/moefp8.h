@@ -128,6 +128,13 @@ moe_status fp8_quant_128x128_pow2(const uint16_t* w, int64_t ldw, int rows, int 
  *   u          bf16 [T][ldu];  centroids bf16 [E][d];  bias fp32 [E]
  *   topk_idx   int32 [T][K];   topk_gate fp32 [T][K]
  *   logits_out fp32 [T][E] or NULL (the logits the selection used)
+ *   aux_rows   fp32 [T][E] or NULL: the per-token rows of the complementary
+ *              sequence-wise balance loss ([ANN] eqs. (17)-(20)), computed
+ *              from the same affinities in the same pass: s' = s / sum_j s_j
+ *              with the sign bit set on the token's raw top-K (over all E
+ *              experts, no bias, no group limit, ties to the lower index, K
+ *              the routing K); moe_seq_balance_loss_rows turns them into the
+ *              loss.  The bytes equal moe_seq_balance_loss's own token pass.
  *   ws         scratch of moe_route_workspace_size() bytes (may be NULL if 0)
  * Limits: d % 128 == 0, E % 16 == 0, 16 <= E <= 1024, E % G == 0,
  * 1 <= M <= G <= 32, K <= E, K % M == 0 when M < G, K <= 32.
@@ -135,8 +142,9 @@ moe_status fp8_quant_128x128_pow2(const uint16_t* w, int64_t ldw, int rows, int 
 moe_status moe_route_workspace_size(int T, int d, int E, size_t* bytes);
 moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* centroids,
                      const float* bias, int T, int d, int E, int G, int M, int K,
-                     int32_t* topk_idx, float* topk_gate, float* logits_out, void* ws,
-                     size_t ws_bytes, int32_t* dev_err, moe_stream_t stream);
+                     int32_t* topk_idx, float* topk_gate, float* logits_out,
+                     float* aux_rows, void* ws, size_t ws_bytes, int32_t* dev_err,
+                     moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * moe_permute -- local permutation of (token, expert) pairs by expert, the
@@ -204,17 +212,19 @@ moe_status moe_tile_table(const int32_t* offsets, int groups, int max_tiles,
                           int32_t* dev_err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
- * moe_segment_ids -- expert parallelism: the local expert of every row of a
- * receive buffer that holds, for each source rank s in order, its rows of
- * this rank's E local experts sorted by expert ([ANN] "Low-Precision
- * Communication": FP8 rows dispatched to the experts' ranks).  counts int32
- * [n_segments] (= [sources][E], row-major) -> ids int32 [n_rows], row r of
- * segment s gets s % E; the ids feed moe_permute (K = 1) to regroup the rows
- * by expert.  Counts that do not sum to n_rows, or negative counts, record
- * MOE_DEVERR_BAD_TABLE.
- * Limits: n_segments % E == 0, n_segments <= 1024. */
-moe_status moe_segment_ids(const int32_t* counts, int n_segments, int E, int64_t n_rows,
-                           int32_t* ids, int32_t* dev_err, moe_stream_t stream);
+ * moe_segment_ids -- expert parallelism: the group of every row of a receive
+ * buffer that holds, for each source rank s in order, its rows of this rank's
+ * E local experts sorted by expert ([ANN] "Low-Precision Communication": FP8
+ * rows dispatched to the experts' ranks).  counts int32 [n_segments] (=
+ * [sources][E], row-major).  With lead_rows == 0: ids int32 [n_rows], row r of
+ * segment s gets s % E.  With lead_rows > 0 the buffer starts with lead_rows
+ * rows of group 0 (the rank's own tokens, which the shared expert takes) and
+ * the received rows after them get 1 + s % E.  The ids feed moe_permute
+ * (K = 1) to regroup the rows by group.  Counts that do not sum to n_rows -
+ * lead_rows, or negative counts, record MOE_DEVERR_BAD_TABLE.
+ * Limits: n_segments % E == 0, n_segments <= 1024, 0 <= lead_rows <= n_rows. */
+moe_status moe_segment_ids(const int32_t* counts, int n_segments, int E, int64_t lead_rows,
+                           int64_t n_rows, int32_t* ids, int32_t* dev_err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * grouped_gemm_fp8_blockscaled -- D_g = A_g . B_g^T for every segment g, with
@@ -232,12 +242,19 @@ moe_status moe_segment_ids(const int32_t* counts, int n_segments, int E, int64_t
  *   (group, n-tile, m-tile) work items from tile_start (the per-group tile
  *   prefix) and offsets; max_tiles bounds its grid.
  *   ep == MOE_EP_F32:  D fp32 [a_rows][N] (rows outside every segment are
- *                      left untouched); d_scale unused.
+ *                      left untouched); d_scale unused.  d_rows (optional,
+ *                      int32 [a_rows], NULL = identity) sends A row j's
+ *                      output to D row d_rows[j]: expert parallelism writes
+ *                      the outputs of rows regrouped by expert straight back
+ *                      in receive order ([ANN] "Low-Precision
+ *                      Communication": the combine's rows return to their
+ *                      senders).  A map entry outside [0, a_rows) records
+ *                      MOE_DEVERR_BAD_TABLE and its row is not written.
  *   ep == MOE_EP_SWIGLU_QUANT: B rows are gate/up block-interleaved (rows
  *      [256j, 256j+128) gate channels 128j.., the next 128 the matching up
  *      channels); D is E4M3 h [a_rows][N/2] with h = SiLU(gate) * up
  *      ([ANN] SwiGLU operator notes, Swish with beta = 1) quantised 1x128 as
- *      in fp8_quant_1x128, d_scale fp32 [a_rows][N/256].
+ *      in fp8_quant_1x128, d_scale fp32 [a_rows][N/256]; d_rows must be NULL.
  * Limits: K % 128 == 0, N % 256 == 0.
  */
 moe_status grouped_gemm_fp8_blockscaled(const uint8_t* A, const float* sa, int64_t a_rows,
@@ -246,7 +263,8 @@ moe_status grouped_gemm_fp8_blockscaled(const uint8_t* A, const float* sa, int64
                                         const int32_t* tile_start, const int32_t* n_tiles,
                                         int max_tiles, int groups, int N, int K,
                                         moe_epilogue ep, void* D, float* d_scale,
-                                        int32_t* dev_err, moe_stream_t stream);
+                                        const int32_t* d_rows, int32_t* dev_err,
+                                        moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * grouped_gemm_fp8_pow2 -- grouped_gemm_fp8_blockscaled for operands whose
@@ -269,8 +287,8 @@ moe_status grouped_gemm_fp8_pow2(const uint8_t* A, const float* sa, int64_t a_ro
                                  const uint8_t* B, const float* sb, const int32_t* offsets,
                                  const int32_t* tile_group, const int32_t* tile_start,
                                  const int32_t* n_tiles, int max_tiles, int groups, int N, int K,
-                                 moe_epilogue ep, void* D, float* d_scale, int32_t* dev_err,
-                                 moe_stream_t stream);
+                                 moe_epilogue ep, void* D, float* d_scale,
+                                 const int32_t* d_rows, int32_t* dev_err, moe_stream_t stream);
 
 /* ===========================================================================
  * Backward of the expert FFNs.  [ANN] "Mixed Precision Framework": Fprop,
@@ -421,6 +439,16 @@ moe_status moe_seq_balance_loss_workspace_size(int T, int E, int seq_len, size_t
 moe_status moe_seq_balance_loss(const float* logits, int T, int E, int K, int seq_len,
                                 float alpha, float* loss, float* f, float* P, void* ws,
                                 size_t ws_bytes, moe_stream_t stream);
+
+/* moe_seq_balance_loss_rows -- the same loss from the per-token rows that
+ * moe_route wrote to aux_rows (its chunk and final passes only; the token
+ * pass is fused into the router's selection).  Same outputs, limits and
+ * determinism as moe_seq_balance_loss; K must be the routing K the rows were
+ * made with.  ws: moe_seq_balance_loss_rows_workspace_size bytes. */
+moe_status moe_seq_balance_loss_rows_workspace_size(int T, int E, int seq_len, size_t* bytes);
+moe_status moe_seq_balance_loss_rows(const float* rows, int T, int E, int K, int seq_len,
+                                     float alpha, float* loss, float* f, float* P, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * moe_fp8_mma_peak -- measurement helper: the dense FP8 tensor-core rate of

@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(_abi.exported_symbols())
-    assert L.moe_abi_version() == 1
+    assert L.moe_abi_version() == 2
 
 
 def test_status_strings():
@@ -49,17 +49,24 @@ def test_max_m_tiles_bound():
     (lambda L: L.fp8_quant_1x128(16, 128, 4, 128, 8, 4, None), 3),          # misaligned
     (lambda L: L.fp8_quant_128x128(None, 64, 4, 128, None, None, None), 2),  # ld < cols
     (lambda L: L.moe_route(None, 256, None, None, 8, 256, 20, 4, 2, 4, None, None, None,
-                           None, 0, None, None), 2),                          # E % 16
+                           None, None, 0, None, None), 2),                    # E % 16
     (lambda L: L.moe_route(None, 256, None, None, 8, 256, 64, 8, 3, 8, None, None, None,
-                           None, 0, None, None), 2),                          # K % M
+                           None, None, 0, None, None), 2),                    # K % M
     (lambda L: L.moe_route(None, 256, None, None, 8, 256, 2048, 8, 4, 8, None, None, None,
-                           None, 0, None, None), 4),                          # E > 1024
+                           None, None, 0, None, None), 4),                    # E > 1024
+    (lambda L: L.moe_seq_balance_loss_rows(None, 100, 16, 4, 30, ctypes.c_float(1e-4), None,
+                                           None, None, None, 0, None), 2),   # T % seq_len
+    (lambda L: L.moe_seq_balance_loss_rows(None, 100, 16, 4, 50, ctypes.c_float(1e-4), None,
+                                           None, None, None, 0, None), 1),   # NULL rows
     (lambda L: L.grouped_gemm_fp8_blockscaled(None, None, 10, None, None, None, None, None,
                                               None, 4, 1, 384, 128, 0, None, None, None,
-                                              None), 2),                      # N % 256
+                                              None, None), 2),                # N % 256
     (lambda L: L.grouped_gemm_fp8_blockscaled(None, None, 10, None, None, None, None, None,
                                               None, 4, 1, 256, 128, 7, None, None, None,
-                                              None), 1),                      # bad epilogue
+                                              None, None), 1),                # bad epilogue
+    (lambda L: L.grouped_gemm_fp8_blockscaled(None, None, 10, None, None, None, None, None,
+                                              None, 4, 1, 256, 128, 1, None, None, 16, None,
+                                              None), 1),                      # row map with SwiGLU
     (lambda L: L.swiglu_quant(None, 4, 100, None, None, None), 2),
     (lambda L: L.moe_seq_balance_loss(None, 100, 16, 4, 30, ctypes.c_float(1e-4), None, None,
                                       None, None, 0, None), 2),              # T % seq_len
@@ -75,7 +82,7 @@ def test_max_m_tiles_bound():
     (lambda L: L.fp8_quant_1x128_pow2(None, 200, 4, 200, None, None, None), 2),
     (lambda L: L.fp8_quant_128x128_pow2(None, 64, 4, 128, None, None, None), 2),
     (lambda L: L.grouped_gemm_fp8_pow2(None, None, 10, None, None, None, None, None, None, 4, 1,
-                                       384, 128, 0, None, None, None, None), 2),  # N % 256
+                                       384, 128, 0, None, None, None, None, None), 2),  # N % 256
     (lambda L: L.swiglu_quant_pow2(None, 4, 100, None, None, None), 2),
     # backward
     (lambda L: L.fp8_quant_1x128_f32(None, 200, 4, 200, 0, None, None, None), 2),
@@ -102,10 +109,11 @@ def test_max_m_tiles_bound():
     (lambda L: L.grouped_gemm_fp8_wgrad(None, None, None, None, 512, 128, 256, None, 2, None,
                                         None, None), 1),                      # NULL buffers
     # expert parallelism
-    (lambda L: L.moe_segment_ids(None, 12, 8, 100, None, None, None), 2),    # segments % E
-    (lambda L: L.moe_segment_ids(None, 2048, 8, 100, None, None, None), 4),  # > 1024 segments
-    (lambda L: L.moe_segment_ids(None, 16, 8, 100, None, None, None), 1),    # NULL buffers
-    (lambda L: L.moe_segment_ids(None, 16, 0, 100, None, None, None), 1),    # E = 0
+    (lambda L: L.moe_segment_ids(None, 12, 8, 0, 100, None, None, None), 2),    # segments % E
+    (lambda L: L.moe_segment_ids(None, 2048, 8, 0, 100, None, None, None), 4),  # > 1024 segments
+    (lambda L: L.moe_segment_ids(None, 16, 8, 0, 100, None, None, None), 1),    # NULL buffers
+    (lambda L: L.moe_segment_ids(None, 16, 0, 0, 100, None, None, None), 1),    # E = 0
+    (lambda L: L.moe_segment_ids(None, 16, 8, 101, 100, None, None, None), 1),  # lead > rows
     # FP8 peak measurement loop
     (lambda L: L.moe_fp8_mma_peak(0, 0, 4, 16, None, None), 1),              # iters < 1
     (lambda L: L.moe_fp8_mma_peak(1, 100, 4, None, None, None), 1),          # NULL sink
@@ -126,4 +134,4 @@ def test_empty_batches_are_no_ops():
                                   None) == 0
     assert L.grouped_gemm_fp8_wgrad(None, None, None, None, 512, 128, 256, None, 0, None, None,
                                     None) == 0
-    assert L.moe_segment_ids(None, 16, 8, 0, None, None, None) == 0
+    assert L.moe_segment_ids(None, 16, 8, 0, 0, None, None, None) == 0

@@ -66,7 +66,7 @@ def test_layer_seq_balance_loss(cuda_dev):
     cfg = configs.TINY
     w1q, w1s, w2q, w2s = make_fp8_weights(cfg, cuda_dev)
     layer = MoELayer(cfg, inputs.draw_centroids(cfg, cuda_dev), inputs.draw_bias(cfg, cuda_dev),
-                     w1q, w1s, w2q, w2s, keep_logits=True)
+                     w1q, w1s, w2q, w2s, keep_logits=True, balance_loss=True)
     layer.forward(inputs.draw_u(cfg, cuda_dev))
     loss = layer.seq_balance_loss(cfg.T // 2)
     torch.cuda.synchronize()
@@ -74,3 +74,31 @@ def test_layer_seq_balance_loss(cuda_dev):
                                           cfg.T // 2, 1e-4)
     clean = (margin < 1e-6).reshape(2, -1).sum(axis=1) == 0
     assert np.allclose(npraw(loss)[clean], lo[clean], rtol=1e-4, atol=0)
+
+
+@pytest.mark.parametrize("cfg_name,S", [("tiny", 64), ("v3_prefill", 4096), ("v3_prefill", 1024),
+                                        ("v4_pro", 2048)])
+def test_route_fused_rows_match_three_pass(cuda_dev, cfg_name, S):
+    """The token pass fused into the router's selection writes the same rows
+    as the standalone token pass on the same logits, so both routes to the
+    loss give identical bytes (loss, f, P)."""
+    from fp8_block_scaled_sigmoid_b200 import configs, inputs
+    cfg = configs.PRESETS[cfg_name]
+    if cfg.T > 4096:
+        cfg = cfg.with_(T=4096)
+    u = inputs.draw_u(cfg, cuda_dev)
+    cent = inputs.draw_centroids(cfg, cuda_dev)
+    bias = inputs.draw_bias(cfg, cuda_dev)
+    logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=cuda_dev)
+    rows = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=cuda_dev)
+    idx, gate = _abi.moe_route(u, cent, bias, cfg.G, cfg.M, cfg.K, logits_out=logits,
+                               aux_rows=rows)
+    idx2, gate2 = _abi.moe_route(u, cent, bias, cfg.G, cfg.M, cfg.K)
+    a = _abi.moe_seq_balance_loss_rows(rows, cfg.K, S, with_fp=True)
+    b = _abi.moe_seq_balance_loss(logits, cfg.K, S, with_fp=True)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(gate, gate2)   # routing unchanged
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    # membership: exactly K negative entries per token
+    assert torch.all((rows < 0).sum(1) == cfg.K)

@@ -10,7 +10,8 @@
   vs (M+1)-th group score) differ by less than 1e-6 -- those are counted and
   only checked for validity; tokens whose chosen experts are tied inside the
   top-K (ordering only) are compared as sets;
-* gates: within 8 fp32 ulps (relative 2^-20) of the fp64 value.
+* gates: within 4 fp32 ulps of the fp64 value (an ulp of the gate's own
+  binade), as the parity contract states.
 """
 import numpy as np
 import pytest
@@ -42,8 +43,11 @@ def _check_selection(z32, bias, G, M, K, idx_g, gate_g):
         if M < G:
             assert len(set(idx_g[t] // (E // G))) <= M
     ok = exact | sets
-    rel = np.abs(gate_g[ok] - gate_o[ok]) / np.abs(gate_o[ok])
-    assert rel.max() <= 2.0 ** -20, f"gate rel err {rel.max():.3e}"
+    go = gate_o[ok]
+    ulp = np.ldexp(1.0, np.frexp(go)[1] - 24)          # fp32 ulp at |gate|
+    ulps = np.abs(gate_g[ok] - go) / ulp
+    print(f"gate error: max {ulps.max():.2f} fp32 ulps, mean {ulps.mean():.3f}")
+    assert ulps.max() <= 4.0, f"gate error {ulps.max():.2f} fp32 ulps"
     # gates of every token renormalise its own chosen raw scores
     s = 1.0 / (1.0 + np.exp(-z32.astype(np.float64)))
     for t in range(0, T, max(1, T // 64)):
