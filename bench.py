@@ -364,7 +364,9 @@ def run_gpu(args):
     barrier()
     layer.check()
 
-    names = ["route", "quant", "permute", "gemm1", "gemm2", "combine", "bias"]
+    # permute = counts, offsets, row maps and tile table; quant = the 1x128
+    # quantisation with the dispatch's row scatter fused in
+    names = ["route", "permute", "quant", "gemm1", "gemm2", "combine", "bias"]
     use_graph = world == 1 and args.graph
     sampler = ClockSampler(local) if rank == 0 else None
 
@@ -389,9 +391,9 @@ def run_gpu(args):
         e[0].record(st)
         layer.step_route(u)
         e[1].record(st)
-        layer.step_quant(u)
-        e[2].record(st)
         layer.step_permute()
+        e[2].record(st)
+        layer.step_quant(u)
         e[3].record(st)
         layer.step_gemm1()
         e[4].record(st)
@@ -533,6 +535,21 @@ def run_gpu(args):
                     "peak_source": f"measured in this run: tcgen05 kind::{fp8['kind']} MMA loop, "
                                    "best of 8 launches (moe_fp8_mma_peak)",
                     "algorithmic_flops": int(g1_flops), "algorithmic_bytes": int(g1_bytes)}
+    # the memory-bound kernels against the measured copy bandwidth, with
+    # their algorithmic bytes: quant reads u (2 B/elem) and writes every FP8
+    # row once per destination (the token copy and K routed rows, 1 B/elem +
+    # 4 B per 128); combine reads K+1 fp32 rows and u, writes fp32
+    Tn, dn = cfg.T, cfg.d
+    q_bytes = Tn * dn * 2 + (cfg.pairs + Tn) * dn * (1 + 4.0 / 128)
+    c_bytes = Tn * ((cfg.K + 1) * 4 * dn + 2 * dn + 4 * dn)
+    tq, tc = per_kernel["quant"] / 1e3, per_kernel["combine"] / 1e3
+    memory_kernels = {
+        "quant_scatter": {"bytes": int(q_bytes), "gbs": round(q_bytes / tq / 1e9, 1),
+                          "frac": round(q_bytes / tq / 1e9 / hbm, 4)},
+        "combine": {"bytes": int(c_bytes), "gbs": round(c_bytes / tc / 1e9, 1),
+                    "frac": round(c_bytes / tc / 1e9 / hbm, 4)},
+        "permute_index_us": round(per_kernel["permute"] * 1e3, 1),
+        "peak": hbm, "unit": "GB/s"}
     gemm = {"gemm1_tflops": round(g1_flops / t1 / 1e12, 1),
             "gemm2_tflops": round(g2_flops / t2 / 1e12, 1),
             "gemm1_gbs": round(achieved, 1), "gemm2_gbs": round(g2_bytes / t2 / 1e9, 1),
@@ -563,6 +580,7 @@ def run_gpu(args):
         "roofline": roofline,
         "gemm": gemm,
         "kernel_ms": {k: round(v, 4) for k, v in per_kernel.items()},
+        "memory_kernels": memory_kernels,
         "seq_balance_loss": balance_loss,
         "loads": {"max": int(counts.max()), "mean": float(counts.float().mean()),
                   "active_experts": active - cfg.n_shared},

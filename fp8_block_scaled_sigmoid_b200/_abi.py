@@ -41,6 +41,8 @@ _SIGS = {
     "moe_permute_noalloc": (_i, [_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p,
                                  _p, _p, _p, _p]),
     "moe_tile_table": (_i, [_p, _i, _i, _p, _p, _p, _p, _p]),
+    "moe_permute_index": (_i, [_p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p, _p]),
+    "fp8_quant_1x128_scatter": (_i, [_p, _i64, _i, _i, _p, _i, _i, _p, _p, _p, _p, _p]),
     "moe_segment_ids": (_i, [_p, _i, _i, _i64, _i64, _p, _p, _p]),
     "grouped_gemm_fp8_blockscaled": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
                                           _i, _p, _p, _p, _p, _p]),
@@ -80,7 +82,8 @@ LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant
                      "moe_combine_backward": 1, "swiglu_backward": 1, "fp8_quant_128x1_pow2": 1,
                      "fp8_requant_128x1_pow2": 1, "fp8_transpose_128x128": 1,
                      "moe_unpermute_add": 1, "grouped_gemm_fp8_wgrad": 1,
-                     "moe_route": 2, "moe_permute": 4, "moe_permute_noalloc": 4,
+                     "moe_route": 2, "moe_permute": 3, "moe_permute_noalloc": 3,
+                     "moe_permute_index": 2, "fp8_quant_1x128_scatter": 1,
                      "moe_tile_table": 1, "moe_segment_ids": 1,
                      "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1,
                      "moe_seq_balance_loss": 3, "moe_fp8_mma_peak": 1,
@@ -262,6 +265,55 @@ def moe_permute(topk_idx, E, xq, xscale, with_shared=True, out=None, ws=None, de
            "moe_permute")
     o["max_tiles"] = mt
     return o
+
+
+def moe_permute_index(topk_idx, E, with_shared=True, out=None, ws=None, dev_err=None,
+                      stream=None):
+    """moe_permute without the row gather: counts, offsets, src_row, dst_of
+    and the tile table in a dict (allocated here unless ``out`` holds them)."""
+    T, K = topk_idx.shape
+    dev = _dev(topk_idx)
+    groups = E + (1 if with_shared else 0)
+    o = {} if out is None else out
+    mt = moe_max_m_tiles(T, K, E, with_shared)
+
+    def get(name, shape, dtype):
+        if name not in o:
+            o[name] = torch.empty(shape, dtype=dtype, device=dev)
+        return o[name]
+
+    counts = get("counts", (E,), torch.int32)
+    offsets = get("offsets", (groups + 1,), torch.int32)
+    src_row = get("src_row", (T * K,), torch.int32)
+    dst_of = get("dst_of", (T, K), torch.int32)
+    tile_group = get("tile_group", (max(mt, 1),), torch.int32)
+    tile_start = get("tile_start", (groups + 1,), torch.int32)
+    n_tiles = get("n_tiles", (1,), torch.int32)
+    need = moe_permute_workspace_size(T, K, E)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _count("moe_permute_index")
+    _check(lib().moe_permute_index(_ptr(topk_idx), T, K, E, int(bool(with_shared)),
+                                   _ptr(counts), _ptr(offsets), _ptr(src_row), _ptr(dst_of),
+                                   _ptr(tile_group), _ptr(tile_start), _ptr(n_tiles), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _ptr(dev_err),
+                                   _stream(stream)), "moe_permute_index")
+    o["max_tiles"] = mt
+    return o
+
+
+def fp8_quant_1x128_scatter(x, dst_of, q_perm, s_perm, q_tok=None, s_tok=None, pow2=False,
+                            stream=None):
+    """x bf16 [rows][cols] -> its 1x128 FP8 tiles at every dst_of[t][k] row of
+    q_perm / s_perm, and (when given) in token order in q_tok / s_tok."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    K = dst_of.shape[1]
+    _count("fp8_quant_1x128_scatter")
+    _check(lib().fp8_quant_1x128_scatter(_ptr(x), x.stride(0), rows, cols, _ptr(dst_of), K,
+                                         int(bool(pow2)), _ptr(q_tok), _ptr(s_tok), _ptr(q_perm),
+                                         _ptr(s_perm), _stream(stream)), "fp8_quant_1x128_scatter")
+    return q_perm, s_perm
 
 
 def moe_permute_noalloc(topk_idx, E, xq, xscale, with_shared=True, out=None, dev_err=None,

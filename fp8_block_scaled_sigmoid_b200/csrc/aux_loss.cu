@@ -6,6 +6,11 @@
 // the TopK taken over the raw affinities of all E routed experts (ties to
 // the lower index).
 //
+// The token pass spreads a row's experts over the lanes exactly as the
+// router's selection kernel does (same experts per lane, same orders), so
+// the rows the selection writes when fused (moe_route's aux_rows) are the
+// same bytes.
+//
 // Three deterministic passes, no atomics:
 //  1. token  -- one warp per token: s, its row sum (fixed butterfly), the
 //               normalised s' and the raw top-K; writes s' with the sign bit
@@ -204,6 +209,7 @@ extern "C" moe_status moe_seq_balance_loss(const float* logits, int T, int E, in
   else if (P <= 2) launch_token<2>(T, E, K, logits, srow, st);
   else if (P <= 4) launch_token<4>(T, E, K, logits, srow, st);
   else if (P <= 8) launch_token<8>(T, E, K, logits, srow, st);
+  else if (P <= 12) launch_token<12>(T, E, K, logits, srow, st);
   else if (P <= 16) launch_token<16>(T, E, K, logits, srow, st);
   else launch_token<32>(T, E, K, logits, srow, st);
   MOE_CUDA_CHECK_LAUNCH();

@@ -210,6 +210,110 @@ __global__ void __launch_bounds__(32 * kScatterWarps) perm_scatter_kernel(
   }
 }
 
+// Scan and scatter fused: one CTA per chunk.  Every CTA sums the per-chunk
+// counts itself -- the chunks before its own (its bases) and all of them
+// (the expert totals) -- and scans the totals over the experts, so no
+// separate single-CTA scan kernel runs between the count and the scatter.
+// CTA 0 also writes counts, offsets and the tile table.  Warps 0..3 then
+// place the chunk's pairs exactly as perm_scatter_kernel does.
+__global__ void __launch_bounds__(kScanThreads) perm_scan_scatter_kernel(
+    const int32_t* __restrict__ idx, int T, int K, int E, int with_shared,
+    const int32_t* __restrict__ ccount, int n_chunks, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ tile_group,
+    int32_t* __restrict__ tile_start, int32_t* __restrict__ n_tiles, int max_tiles,
+    int32_t* __restrict__ src_row, int32_t* __restrict__ dst_of, int32_t* dev_err) {
+  extern __shared__ int32_t sm[];
+  __shared__ int scan_smem[40];
+  int32_t* cursor = sm;                        // [kScatterWarps][E]
+  int32_t* hist = sm + kScatterWarps * E;      // [kScatterWarps][E]
+  int32_t* sidx = sm + 2 * kScatterWarps * E;  // [kChunkT * K]
+  int32_t* cbase = sidx + kChunkT * K;         // [E]
+  const int e = threadIdx.x;
+  const int my = blockIdx.x;
+  int before = 0, total = 0;
+  if (e < E) {
+    int c = 0;
+    for (; c + 8 <= n_chunks; c += 8) {  // eight loads in flight
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = __ldg(ccount + static_cast<int64_t>(c + j) * E + e);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        before += (c + j < my) ? v[j] : 0;
+        total += v[j];
+      }
+    }
+    for (; c < n_chunks; ++c) {
+      const int v = __ldg(ccount + static_cast<int64_t>(c) * E + e);
+      before += (c < my) ? v : 0;
+      total += v;
+    }
+  }
+  int* warp_sums = scan_smem;
+  const int off = block_excl_scan(e < E ? total : 0, warp_sums, &scan_smem[32]);
+  if (e < E) cbase[e] = off + before;
+  if (my == 0) {
+    if (e < E) counts[e] = total;
+    const int groups = E + (with_shared ? 1 : 0);
+    const int cnt = (e < E) ? total : ((with_shared && e == E) ? T : 0);
+    write_tables(cnt, e, groups, offsets, tile_group, tile_start, n_tiles, max_tiles, dev_err,
+                 scan_smem);
+  }
+  const int lane = threadIdx.x & 31, wj = threadIdx.x >> 5;
+  const int t0 = my * kChunkT;
+  const int nt = min(kChunkT, T - t0);
+  for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) hist[i] = 0;
+  for (int p = threadIdx.x; p < nt * K; p += blockDim.x) sidx[p] = idx[static_cast<int64_t>(t0) * K + p];
+  __syncthreads();
+  const int wt0 = wj * kTokPerWarp, wt1 = min(nt, wt0 + kTokPerWarp);
+  if (wj < kScatterWarps)
+    for (int p = wt0 * K + lane; p < wt1 * K; p += 32) {
+      const int ex = sidx[p];
+      if (ex >= 0 && ex < E) atomicAdd(&hist[wj * E + ex], 1);
+    }
+  __syncthreads();
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {
+    int run = cbase[x];
+    for (int j = 0; j < kScatterWarps; ++j) {
+      cursor[j * E + x] = run;
+      run += hist[j * E + x];
+    }
+  }
+  __syncthreads();
+  if (wj >= kScatterWarps) return;
+  int32_t* cur = cursor + wj * E;
+  const int tpi = 32 / K;  // tokens per step
+  const int tl = lane / K, k = lane - (lane / K) * K;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int tb = wt0; tb < wt1; tb += tpi) {
+    const int tt = tb + tl;
+    int ex = -1;
+    if (tl < tpi && tt < wt1) ex = sidx[tt * K + k];
+    const bool active = ex >= 0 && ex < E;
+    const unsigned amask = __ballot_sync(0xffffffffu, active);
+    unsigned peers = 0;
+    int pos = 0;
+    if (active) {
+      peers = __match_any_sync(amask, ex);
+      pos = cur[ex] + __popc(peers & lt_mask);
+    }
+    __syncwarp();
+    if (active && lane == __ffs(peers) - 1) cur[ex] += __popc(peers);
+    __syncwarp();
+    if (active) {
+      const int t = t0 + tt;
+      src_row[pos] = t;
+      dst_of[static_cast<int64_t>(t) * K + k] = pos;
+    } else if (tl < tpi && tt < wt1) {
+      dst_of[static_cast<int64_t>(t0 + tt) * K + k] = -1;  // flagged bad index: no row
+    }
+  }
+}
+
+size_t scan_scatter_smem(int E, int K) {
+  return (2 * kScatterWarps * static_cast<size_t>(E) + kChunkT * K + E) * sizeof(int32_t);
+}
+
 // One warp per destination row: d bytes of FP8 plus d/128 fp32 scales.
 __global__ void __launch_bounds__(256) perm_gather_kernel(
     const int32_t* __restrict__ src_row, int rows, int T, const uint8_t* __restrict__ xq,
@@ -316,6 +420,56 @@ extern "C" moe_status moe_permute_workspace_size(int T, int K, int E, size_t* by
   return MOE_OK;
 }
 
+namespace {
+
+// Count, then the fused scan + scatter: counts, offsets, the tile table,
+// src_row and dst_of (no row moves).  Arguments already validated.
+moe_status permute_index_launch(const int32_t* topk_idx, int T, int K, int E, int with_shared,
+                                int32_t* counts, int32_t* offsets, int32_t* src_row,
+                                int32_t* dst_of, int32_t* tile_group, int32_t* tile_start,
+                                int32_t* n_tiles, void* ws, int32_t* dev_err, cudaStream_t st) {
+  using namespace moe;
+  const int nch = n_chunks_of(T);
+  int32_t* ccount = static_cast<int32_t*>(ws);
+  const int max_tiles = moe_max_m_tiles(T, K, E, with_shared);
+  if (nch == 0) {
+    perm_scan_kernel<<<1, kScanThreads, 0, st>>>(ccount, nch, E, T, with_shared, counts, offsets,
+                                                 tile_group, tile_start, n_tiles, max_tiles,
+                                                 dev_err);
+    MOE_CUDA_CHECK_LAUNCH();
+    return MOE_OK;
+  }
+  perm_count_kernel<<<nch, 256, E * sizeof(int32_t), st>>>(topk_idx, T, K, E, ccount, dev_err);
+  MOE_CUDA_CHECK_LAUNCH();
+  const size_t sm = scan_scatter_smem(E, K);
+  if (sm > 48 * 1024 &&
+      cudaFuncSetAttribute(perm_scan_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sm)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  perm_scan_scatter_kernel<<<nch, kScanThreads, sm, st>>>(
+      topk_idx, T, K, E, with_shared, ccount, nch, counts, offsets, tile_group, tile_start,
+      n_tiles, max_tiles, src_row, dst_of, dev_err);
+  MOE_CUDA_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+moe_status permute_index_check(const int32_t* topk_idx, int T, int K, int E, int32_t* counts,
+                               int32_t* offsets, int32_t* src_row, int32_t* dst_of,
+                               int32_t* tile_group, int32_t* tile_start, int32_t* n_tiles,
+                               void* ws, size_t ws_bytes) {
+  using namespace moe;
+  if (T < 0 || K <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+  if (K > 32 || K > E) return MOE_ERR_UNSUPPORTED;
+  if (!counts || !offsets || !tile_start || !n_tiles || !tile_group) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_idx || !src_row || !dst_of)) return MOE_ERR_INVALID_ARG;
+  size_t need = 0;
+  moe_permute_workspace_size(T, K, E, &need);
+  if (ws_bytes < need || (!ws && need)) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+}  // namespace
+
 extern "C" moe_status moe_permute(const int32_t* topk_idx, int T, int K, int E, int with_shared,
                                   const uint8_t* xq, const float* xscale, int d, int32_t* counts,
                                   int32_t* offsets, int32_t* src_row, int32_t* dst_of,
@@ -325,36 +479,36 @@ extern "C" moe_status moe_permute(const int32_t* topk_idx, int T, int K, int E, 
   using namespace moe;
   if (T < 0 || K <= 0 || E <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
   if (d % 128 != 0) return MOE_ERR_SHAPE;
-  if (K > 32 || K > E || E + (with_shared ? 1 : 0) > kScanThreads) return MOE_ERR_UNSUPPORTED;
-  if (!counts || !offsets || !tile_start || !n_tiles || !tile_group) return MOE_ERR_INVALID_ARG;
-  if (T > 0 && (!topk_idx || !xq || !xscale || !src_row || !dst_of || !xq_perm || !xscale_perm))
-    return MOE_ERR_INVALID_ARG;
+  if (E + (with_shared ? 1 : 0) > kScanThreads) return MOE_ERR_UNSUPPORTED;
+  moe_status r = permute_index_check(topk_idx, T, K, E, counts, offsets, src_row, dst_of,
+                                     tile_group, tile_start, n_tiles, ws, ws_bytes);
+  if (r != MOE_OK) return r;
+  if (T > 0 && (!xq || !xscale || !xq_perm || !xscale_perm)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(xq_perm)) return MOE_ERR_ALIGN;
-  size_t need = 0;
-  moe_permute_workspace_size(T, K, E, &need);
-  if (ws_bytes < need || (!ws && need)) return MOE_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int nch = n_chunks_of(T);
-  int32_t* ccount = static_cast<int32_t*>(ws);
-  const int max_tiles = moe_max_m_tiles(T, K, E, with_shared);
-  if (nch > 0) {
-    perm_count_kernel<<<nch, 256, E * sizeof(int32_t), st>>>(topk_idx, T, K, E, ccount, dev_err);
-    MOE_CUDA_CHECK_LAUNCH();
-  }
-  perm_scan_kernel<<<1, kScanThreads, 0, st>>>(ccount, nch, E, T, with_shared, counts, offsets,
-                                               tile_group, tile_start, n_tiles, max_tiles, dev_err);
+  r = permute_index_launch(topk_idx, T, K, E, with_shared, counts, offsets, src_row, dst_of,
+                           tile_group, tile_start, n_tiles, ws, dev_err, st);
+  if (r != MOE_OK || T == 0) return r;
+  const int rows = T * K;
+  perm_gather_kernel<<<(rows + 7) / 8, 256, 0, st>>>(src_row, rows, T, xq, xscale, d, xq_perm,
+                                                     xscale_perm);
   MOE_CUDA_CHECK_LAUNCH();
-  if (nch > 0) {
-    const size_t sm = (2 * kScatterWarps * static_cast<size_t>(E) + kChunkT * K) * sizeof(int32_t);
-    perm_scatter_kernel<<<nch, 32 * kScatterWarps, sm, st>>>(topk_idx, T, K, E, ccount, src_row,
-                                                             dst_of);
-    MOE_CUDA_CHECK_LAUNCH();
-    const int rows = T * K;
-    perm_gather_kernel<<<(rows + 7) / 8, 256, 0, st>>>(src_row, rows, T, xq, xscale, d, xq_perm,
-                                                       xscale_perm);
-    MOE_CUDA_CHECK_LAUNCH();
-  }
   return MOE_OK;
+}
+
+extern "C" moe_status moe_permute_index(const int32_t* topk_idx, int T, int K, int E,
+                                        int with_shared, int32_t* counts, int32_t* offsets,
+                                        int32_t* src_row, int32_t* dst_of, int32_t* tile_group,
+                                        int32_t* tile_start, int32_t* n_tiles, void* ws,
+                                        size_t ws_bytes, int32_t* dev_err, moe_stream_t stream) {
+  using namespace moe;
+  if (E + (with_shared ? 1 : 0) > kScanThreads) return MOE_ERR_UNSUPPORTED;
+  const moe_status r = permute_index_check(topk_idx, T, K, E, counts, offsets, src_row, dst_of,
+                                           tile_group, tile_start, n_tiles, ws, ws_bytes);
+  if (r != MOE_OK) return r;
+  return permute_index_launch(topk_idx, T, K, E, with_shared, counts, offsets, src_row, dst_of,
+                              tile_group, tile_start, n_tiles, ws, dev_err,
+                              static_cast<cudaStream_t>(stream));
 }
 
 extern "C" moe_status moe_segment_ids(const int32_t* counts, int n_segments, int E,

@@ -31,10 +31,16 @@ constexpr int kQ1Threads = 256;
 constexpr int kTilesPerHW = 4;
 constexpr int kQ1TilesPerBlock = (kQ1Threads / 16) * kTilesPerHW;
 
-template <bool POW2>
+// With SCATTER the tile is also written to the K routed rows of its token
+// (dst_of[row][k] >= 0: row of q_perm / s_perm; the permutation's gather
+// fused into the quantiser, so each token is read once and its FP8 bytes go
+// straight to every destination).  K <= 16: lane k of a half-warp holds the
+// row's k-th destination.
+template <bool POW2, bool SCATTER>
 __global__ void __launch_bounds__(kQ1Threads) quant_1x128_kernel(
     const uint16_t* __restrict__ x, int64_t ldx, int rows, int tiles_per_row,
-    uint8_t* __restrict__ q, float* __restrict__ scale) {
+    uint8_t* __restrict__ q, float* __restrict__ scale, const int32_t* __restrict__ dst_of,
+    int K, uint8_t* __restrict__ q_perm, float* __restrict__ s_perm) {
   const int lane16 = threadIdx.x & 15;
   const int hw = threadIdx.x >> 4;
   const int64_t total = static_cast<int64_t>(rows) * tiles_per_row;
@@ -78,16 +84,33 @@ __global__ void __launch_bounds__(kQ1Threads) quant_1x128_kernel(
 #pragma unroll
     for (int off = 8; off > 0; off >>= 1)
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float s = tile_scale<POW2>(amax);
+    const float rs = __frcp_rn(s);
+    uint2 out;
+    out.x = e4m3x4(div_by_scale(f[0], s, rs), div_by_scale(f[1], s, rs),
+                   div_by_scale(f[2], s, rs), div_by_scale(f[3], s, rs));
+    out.y = e4m3x4(div_by_scale(f[4], s, rs), div_by_scale(f[5], s, rs),
+                   div_by_scale(f[6], s, rs), div_by_scale(f[7], s, rs));
     if (t < total) {
-      const float s = tile_scale<POW2>(amax);
-      const float rs = __frcp_rn(s);
-      uint2 out;
-      out.x = e4m3x4(div_by_scale(f[0], s, rs), div_by_scale(f[1], s, rs),
-                     div_by_scale(f[2], s, rs), div_by_scale(f[3], s, rs));
-      out.y = e4m3x4(div_by_scale(f[4], s, rs), div_by_scale(f[5], s, rs),
-                     div_by_scale(f[6], s, rs), div_by_scale(f[7], s, rs));
-      *reinterpret_cast<uint2*>(q + r * cols + j * 128 + lane16 * 8) = out;
-      if (lane16 == 0) scale[t] = s;
+      if (q != nullptr) {
+        *reinterpret_cast<uint2*>(q + r * cols + j * 128 + lane16 * 8) = out;
+        if (lane16 == 0) scale[t] = s;
+      }
+    }
+    if (SCATTER) {
+      // every lane of the warp takes part in the exchange (the two half-warps
+      // may be at different rows, or one past the end)
+      const int64_t rr = t < total ? r : 0;
+      const int my_dst = lane16 < K ? __ldg(dst_of + rr * K + lane16) : -1;
+      const int hbase = threadIdx.x & 16;
+      for (int k = 0; k < K; ++k) {
+        const int dr = __shfl_sync(0xffffffffu, my_dst, hbase + k);
+        if (t < total && dr >= 0) {
+          *reinterpret_cast<uint2*>(q_perm + static_cast<int64_t>(dr) * cols + j * 128 +
+                                    lane16 * 8) = out;
+          if (lane16 == 0) s_perm[static_cast<int64_t>(dr) * tiles_per_row + j] = s;
+        }
+      }
     }
     if (++j == tiles_per_row) {
       j = 0;
@@ -202,9 +225,33 @@ moe_status quant_1x128_launch(bool pow2, const uint16_t* x, int64_t ldx, int row
   const int64_t tiles = static_cast<int64_t>(rows) * (cols / 128);
   const int64_t blocks = (tiles + kQ1TilesPerBlock - 1) / kQ1TilesPerBlock;
   if (blocks > 0x7FFFFFFF) return MOE_ERR_UNSUPPORTED;
-  auto kern = pow2 ? quant_1x128_kernel<true> : quant_1x128_kernel<false>;
+  auto kern = pow2 ? quant_1x128_kernel<true, false> : quant_1x128_kernel<false, false>;
   kern<<<static_cast<unsigned>(blocks), kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      x, ldx, rows, cols / 128, q, scale);
+      x, ldx, rows, cols / 128, q, scale, nullptr, 0, nullptr, nullptr);
+  MOE_CUDA_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+moe_status quant_1x128_scatter_launch(bool pow2, const uint16_t* x, int64_t ldx, int rows,
+                                      int cols, const int32_t* dst_of, int K, uint8_t* q_tok,
+                                      float* s_tok, uint8_t* q_perm, float* s_perm,
+                                      moe_stream_t stream) {
+  using namespace moe;
+  if (rows < 0 || cols < 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (cols % 128 != 0 || ldx < cols) return MOE_ERR_SHAPE;
+  if (K > 16) return MOE_ERR_UNSUPPORTED;
+  if (rows == 0 || cols == 0) return MOE_OK;
+  if (!x || !dst_of || !q_perm || !s_perm || (q_tok == nullptr) != (s_tok == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || (q_tok && !aligned16(q_tok)) || !aligned16(q_perm) || (ldx % 8) != 0 ||
+      (reinterpret_cast<uintptr_t>(s_tok) & 3) || (reinterpret_cast<uintptr_t>(s_perm) & 3))
+    return MOE_ERR_ALIGN;
+  const int64_t tiles = static_cast<int64_t>(rows) * (cols / 128);
+  const int64_t blocks = (tiles + kQ1TilesPerBlock - 1) / kQ1TilesPerBlock;
+  if (blocks > 0x7FFFFFFF) return MOE_ERR_UNSUPPORTED;
+  auto kern = pow2 ? quant_1x128_kernel<true, true> : quant_1x128_kernel<false, true>;
+  kern<<<static_cast<unsigned>(blocks), kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, ldx, rows, cols / 128, q_tok, s_tok, dst_of, K, q_perm, s_perm);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }
@@ -237,6 +284,14 @@ extern "C" moe_status fp8_quant_1x128(const uint16_t* x, int64_t ldx, int rows, 
 extern "C" moe_status fp8_quant_1x128_pow2(const uint16_t* x, int64_t ldx, int rows, int cols,
                                            uint8_t* q, float* scale, moe_stream_t stream) {
   return quant_1x128_launch(true, x, ldx, rows, cols, q, scale, stream);
+}
+
+extern "C" moe_status fp8_quant_1x128_scatter(const uint16_t* x, int64_t ldx, int rows, int cols,
+                                              const int32_t* dst_of, int K, int pow2,
+                                              uint8_t* q_tok, float* s_tok, uint8_t* q_perm,
+                                              float* s_perm, moe_stream_t stream) {
+  return quant_1x128_scatter_launch(pow2 != 0, x, ldx, rows, cols, dst_of, K, q_tok, s_tok,
+                                    q_perm, s_perm, stream);
 }
 
 extern "C" moe_status fp8_quant_128x128(const uint16_t* w, int64_t ldw, int rows, int cols,

@@ -141,9 +141,10 @@ class MoELayerEP:
     kernels; this class owns the buffers (all allocated once, here) and
     sequences the calls around the two exchanges:
 
-        stage_dispatch:  moe_route -> fp8_quant_1x128 (into the receive
-                         buffer's head) -> moe_permute over all E experts
-                         (the send buffer, expert-sorted)
+        stage_dispatch:  moe_route -> moe_permute_index over all E experts
+                         -> fp8_quant_1x128_scatter (the tokens into the
+                         receive buffer's head, their routed rows into the
+                         send buffer, expert-sorted)
         plan + dispatch: per-expert counts all-to-all, split sizes to the host,
                          FP8 rows + scales all-to-all into the receive buffer
         stage_experts:   moe_segment_ids (the rank's T own tokens = group 0,
@@ -199,16 +200,22 @@ class MoELayerEP:
         self.route_ws = torch.empty(max(_abi.moe_route_workspace_size(T, d, E), 16), dtype=u8,
                                     device=dev)
         self.dev_err = torch.zeros(1, dtype=i32, device=dev)
-        # send side: routed rows sorted by expert over all E experts
-        self.Xsend = torch.empty(P, d, dtype=u8, device=dev)
-        self.Xs_send = torch.empty(P, d // 128, dtype=f32, device=dev)
-        self.perm = {"xq_perm": self.Xsend, "xs_perm": self.Xs_send}
-        self.perm_ws = torch.empty(max(_abi.moe_permute_workspace_size(T, K, E), 16), dtype=u8,
-                                   device=dev)
         # receive side: [own T tokens | received rows], then regrouped copies
         rows = T + Rcap
         self.RX = torch.empty(rows, d, dtype=u8, device=dev)
         self.RXs = torch.empty(rows, d // 128, dtype=f32, device=dev)
+        # send side: routed rows sorted by expert over all E experts.  With one
+        # rank every row goes to this rank in send order, so the send buffer
+        # is the receive area itself and the dispatch moves nothing.
+        self.local = shard.world == 1
+        if self.local:
+            self.Xsend, self.Xs_send = self.RX[T:T + P], self.RXs[T:T + P]
+        else:
+            self.Xsend = torch.empty(P, d, dtype=u8, device=dev)
+            self.Xs_send = torch.empty(P, d // 128, dtype=f32, device=dev)
+        self.perm = {"xq_perm": self.Xsend, "xs_perm": self.Xs_send}
+        self.perm_ws = torch.empty(max(_abi.moe_permute_workspace_size(T, K, E), 16), dtype=u8,
+                                   device=dev)
         self.ids = torch.empty(rows, dtype=i32, device=dev)
         self.X2 = torch.empty(rows, d, dtype=u8, device=dev)
         self.X2s = torch.empty(rows, d // 128, dtype=f32, device=dev)
@@ -226,7 +233,8 @@ class MoELayerEP:
         self.H2 = torch.empty(rows, I, dtype=u8, device=dev)
         self.H2s = torch.empty(rows, I // 128, dtype=f32, device=dev)
         self.Yr = torch.empty(rows, d, dtype=f32, device=dev)     # receive order
-        self.Yback = torch.empty(P, d, dtype=f32, device=dev)     # send order
+        # send order (with one rank the same rows: receive order is send order)
+        self.Yback = self.Yr[T:T + P] if self.local else torch.empty(P, d, dtype=f32, device=dev)
         self.recv_counts = torch.empty(shard.world, El, dtype=i32, device=dev)
         self.out = torch.empty(T, d, dtype=f32, device=dev)
         self.plan: DispatchPlan | None = None
@@ -234,17 +242,18 @@ class MoELayerEP:
 
     # -- stages (the emulation of several ranks on one GPU calls them) -----
     def stage_dispatch(self, u: torch.Tensor) -> torch.Tensor:
-        """Route, quantise the rank's tokens into the receive buffer's head,
-        sort the routed rows by expert into the send buffer.  Returns the
-        per-expert counts (device int32 [E])."""
+        """Route, then quantise the rank's tokens once: into the receive
+        buffer's head, and their routed rows, sorted by expert, into the send
+        buffer.  Returns the per-expert counts (device int32 [E])."""
         a, c = self._abi, self.cfg
         T = self.T
         assert u.shape == (T, c.d) and u.dtype == torch.bfloat16
         a.moe_route(u, self.centroids, self.bias, c.G, c.M, c.K, self.idx, self.gate,
                     ws=self.route_ws, dev_err=self.dev_err)
-        a.fp8_quant_1x128(u, self.RX[:T], self.RXs[:T])
-        a.moe_permute(self.idx, c.E, self.RX[:T], self.RXs[:T], False, out=self.perm,
-                      ws=self.perm_ws, dev_err=self.dev_err)
+        a.moe_permute_index(self.idx, c.E, False, out=self.perm, ws=self.perm_ws,
+                            dev_err=self.dev_err)
+        a.fp8_quant_1x128_scatter(u, self.perm["dst_of"], self.Xsend, self.Xs_send,
+                                  self.RX[:T], self.RXs[:T])
         return self.perm["counts"]
 
     def send_rows(self):
@@ -303,15 +312,23 @@ class MoELayerEP:
     # -- one step with the process group's exchanges ------------------------
     def forward(self, u: torch.Tensor, update_bias: bool = True) -> torch.Tensor:
         counts = self.stage_dispatch(u)
-        plan = plan_dispatch(counts, self.shard, self.pg, dev_err=self.dev_err,
-                             recv_counts=self.recv_counts)
-        rq, rs = self.recv_rows(plan)
-        xq, xs = self.send_rows()
-        exchange_rows(xq, plan.send_splits, plan.recv_splits, self.pg, out=rq)
-        exchange_rows(xs, plan.send_splits, plan.recv_splits, self.pg, out=rs)
-        self.stage_experts()
-        exchange_rows(self.return_rows(), plan.recv_splits, plan.send_splits, self.pg,
-                      out=self.Yback)
+        if self.local:
+            # one rank: every split is known on the host (all T*K rows stay),
+            # the counts "exchange" is a device copy and the rows are already
+            # in place, so the step needs no host synchronisation
+            self.recv_counts.copy_(counts.view(1, -1))
+            self.recv_rows(DispatchPlan([self.pairs], [self.pairs], self.recv_counts))
+            self.stage_experts()
+        else:
+            plan = plan_dispatch(counts, self.shard, self.pg, dev_err=self.dev_err,
+                                 recv_counts=self.recv_counts)
+            rq, rs = self.recv_rows(plan)
+            xq, xs = self.send_rows()
+            exchange_rows(xq, plan.send_splits, plan.recv_splits, self.pg, out=rq)
+            exchange_rows(xs, plan.send_splits, plan.recv_splits, self.pg, out=rs)
+            self.stage_experts()
+            exchange_rows(self.return_rows(), plan.recv_splits, plan.send_splits, self.pg,
+                          out=self.Yback)
         out = self.stage_combine(u)
         if update_bias:
             from .layer import reduce_load_counts

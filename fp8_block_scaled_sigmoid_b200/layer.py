@@ -3,7 +3,9 @@
 The steps ("DeepSeek_V3_Report：Annotation", eqs. (12)-(16); quantise before
 dispatch per "Low-Precision Communication"):
 
-    moe_route -> fp8_quant_1x128(u) -> moe_permute
+    moe_route -> moe_permute_index (counts, offsets, row maps, tile table)
+      -> fp8_quant_1x128_scatter(u): each token quantised once, its FP8 row
+         written in token order and at each of its K expert-sorted rows
       -> grouped GEMM 1 (W1, fused SwiGLU + 1x128 requantisation)
       -> grouped GEMM 2 (W2, fp32 rows) -> moe_combine -> moe_bias_update
 
@@ -15,8 +17,8 @@ every step runs in libmoefp8.so.
 Row layout of the permuted activations (and of h and Y): rows [0, T*K) are
 the routed pairs sorted by expert, rows [T*K, T*K+T) are the T tokens in
 order, which the shared expert (group E of the grouped GEMMs) consumes.  The
-quantiser writes the tokens straight into that tail and the permutation
-gathers the routed rows from it, so the shared expert costs no copy.
+quantiser writes the tokens into that tail and the routed rows in the same
+pass, so neither the shared expert nor the dispatch costs a separate copy.
 """
 from __future__ import annotations
 
@@ -149,13 +151,17 @@ class MoELayer:
                        logits_out=self.logits, ws=self.route_ws, dev_err=self.dev_err,
                        aux_rows=self.aux_rows)
 
-    def step_quant(self, u):
-        _abi.fp8_quant_1x128(u, self.Xq[self.pairs:], self.Xs[self.pairs:], pow2=self.pow2)
-
     def step_permute(self):
-        c = self.cfg
-        _abi.moe_permute(self.idx, c.E, self.Xq[self.pairs:], self.Xs[self.pairs:], True,
-                         out=self.perm, ws=self.perm_ws, dev_err=self.dev_err)
+        """Counts, offsets, row maps and the tile table (no row moves yet)."""
+        _abi.moe_permute_index(self.idx, self.cfg.E, True, out=self.perm, ws=self.perm_ws,
+                               dev_err=self.dev_err)
+
+    def step_quant(self, u):
+        """1x128 quantisation of u, written in token order (the shared
+        expert's rows) and at every routed row (the dispatch)."""
+        P = self.pairs
+        _abi.fp8_quant_1x128_scatter(u, self.perm["dst_of"], self.Xq[:P], self.Xs[:P],
+                                     self.Xq[P:], self.Xs[P:], pow2=self.pow2)
 
     def step_gemm1(self):
         p = self.perm
@@ -188,8 +194,8 @@ class MoELayer:
         assert u.shape == (self.T, self.cfg.d) and u.dtype == torch.bfloat16
         out = self.out if out is None else out
         self.step_route(u)
-        self.step_quant(u)
         self.step_permute()
+        self.step_quant(u)
         self.step_gemm1()
         self.step_gemm2()
         self.step_combine(u, out)
@@ -213,8 +219,8 @@ class MoELayer:
             self.GUq = torch.empty(rows, 2 * c.I, dtype=torch.uint8, device=dev)
             self.GUs = torch.empty(rows, 2 * c.I // 128, dtype=torch.float32, device=dev)
         self.step_route(u)
-        self.step_quant(u)
         self.step_permute()
+        self.step_quant(u)
         p = self.perm
         _abi.grouped_gemm_fp8_blockscaled(self.Xq, self.Xs, self.w1q, self.w1s, p["offsets"],
                                           p["tile_group"], p["tile_start"], p["n_tiles"],

@@ -176,6 +176,40 @@ moe_status moe_permute(const int32_t* topk_idx, int T, int K, int E, int with_sh
                        moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_permute_index -- moe_permute without moving any row: counts, offsets,
+ * src_row, dst_of and the tile table only (same arguments, layouts, limits
+ * and errors, minus xq/xscale/d/xq_perm/xscale_perm).  The rows are then
+ * written by fp8_quant_1x128_scatter, which quantises each token once and
+ * stores its FP8 bytes straight at every destination row ([ANN]
+ * "Low-Precision Communication": the tokens are quantised to FP8 and the FP8
+ * rows are what the dispatch moves).
+ */
+moe_status moe_permute_index(const int32_t* topk_idx, int T, int K, int E, int with_shared,
+                             int32_t* counts, int32_t* offsets, int32_t* src_row,
+                             int32_t* dst_of, int32_t* tile_group, int32_t* tile_start,
+                             int32_t* n_tiles, void* ws, size_t ws_bytes, int32_t* dev_err,
+                             moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * fp8_quant_1x128_scatter -- fp8_quant_1x128 (or its power-of-two form,
+ * pow2 != 0) with the permutation's gather fused in: every 1x128 tile of row
+ * t is quantised once ([ANN] "Fine-Grained Quantization", "Online
+ * Quantization") and written to the token-order copy q_tok / s_tok (row t;
+ * both may be NULL) and to row dst_of[t][k] of q_perm / s_perm for every k
+ * with dst_of[t][k] >= 0 (moe_permute_index's output; a -1 entry, left by a
+ * flagged bad expert index, writes nothing).  The bytes and scales equal
+ * fp8_quant_1x128 followed by moe_permute's gather.
+ *   x bf16 [rows][ldx]; dst_of int32 [rows][K]; q_tok E4M3 [rows][cols],
+ *   s_tok fp32 [rows][cols/128]; q_perm E4M3 [rows*K][cols], s_perm fp32
+ *   [rows*K][cols/128].
+ * Limits: cols % 128 == 0, 1 <= K <= 16.
+ */
+moe_status fp8_quant_1x128_scatter(const uint16_t* x, int64_t ldx, int rows, int cols,
+                                   const int32_t* dst_of, int K, int pow2, uint8_t* q_tok,
+                                   float* s_tok, uint8_t* q_perm, float* s_perm,
+                                   moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_permute_noalloc -- moe_permute without a caller workspace.  The pages
  * have no counterpart: it is a deployment convenience.  It serves callers
  * that cannot allocate device memory at call time -- plugins of inference

@@ -192,7 +192,8 @@ def test_captured_step_matches_forward(cuda_dev):
     u = inputs.draw_u(cfg, cuda_dev)
     graph, n = layer.capture(u)       # runs one eager step first
     assert n == sum(_abi.LAUNCHES_PER_CALL[k] for k in (
-        "moe_route", "fp8_quant_1x128", "moe_permute", "moe_combine", "moe_bias_update")) + 2
+        "moe_route", "moe_permute_index", "fp8_quant_1x128_scatter", "moe_combine",
+        "moe_bias_update")) + 2
     torch.cuda.synchronize()
     layer.bias.copy_(bias0)
     ref = layer.forward(u).clone()
