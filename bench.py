@@ -460,12 +460,12 @@ def run_gpu(args):
     out_host = out_hosts[0]
 
     # the sequence-wise balance loss (eqs. 17-20) of this batch, one sequence
-    # of T tokens: its per-token rows come out of the router's selection pass
-    # (aux_rows), two short reductions finish it.  Its cost is the route with
-    # the rows minus the route without them, plus the reductions; the
+    # of T tokens: the router's selection pass writes its per-8-token partial
+    # sums (aux_part), one short reduction finishes it.  Its cost is the route
+    # with the partials minus the route without them, plus the reduction; the
     # three-pass form from kept logits is timed beside it.
     logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
-    rows = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
+    part = torch.empty((cfg.T + 7) // 8, 2, cfg.E, dtype=torch.float32, device=dev)
     rws = torch.empty(max(_abi.moe_route_workspace_size(cfg.T, cfg.d, cfg.E), 16),
                       dtype=torch.uint8, device=dev)
     bl_ws = torch.empty(max(_abi.moe_seq_balance_loss_ws(cfg.T, cfg.E, cfg.T), 16),
@@ -486,16 +486,16 @@ def run_gpu(args):
     t_plain = timed(lambda: _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K,
                                            ws=rws), reps)
     t_aux = timed(lambda: _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K,
-                                         ws=rws, aux_rows=rows), reps)
-    t_red = timed(lambda: _abi.moe_seq_balance_loss_rows(rows, cfg.K, cfg.T, ws=bl_ws), reps)
+                                         ws=rws, aux_part=part), reps)
+    t_red = timed(lambda: _abi.moe_seq_balance_loss_part(part, cfg.T, cfg.K, cfg.T), reps)
     _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K, logits_out=logits, ws=rws)
     t_3p = timed(lambda: _abi.moe_seq_balance_loss(logits, cfg.K, cfg.T, ws=bl_ws), reps)
     barrier()
     balance_loss = {"extra_us": round(t_aux - t_plain + t_red, 2),
-                    "route_us": round(t_plain, 2), "route_with_rows_us": round(t_aux, 2),
-                    "reductions_us": round(t_red, 2), "three_pass_from_logits_us": round(t_3p, 2),
+                    "route_us": round(t_plain, 2), "route_with_partials_us": round(t_aux, 2),
+                    "reduction_us": round(t_red, 2), "three_pass_from_logits_us": round(t_3p, 2),
                     "seq_len": cfg.T}
-    del logits, rows, rws, bl_ws
+    del logits, part, rws, bl_ws
 
     # roofline of the dominant kernel (grouped GEMM 1 with the SwiGLU epilogue)
     counts = layer.perm["counts"].cpu()

@@ -7,9 +7,9 @@
 // the lower index).
 //
 // The token pass spreads a row's experts over the lanes exactly as the
-// router's selection kernel does (same experts per lane, same orders), so
-// the rows the selection writes when fused (moe_route's aux_rows) are the
-// same bytes.
+// router's selection kernel does (same experts per lane, same orders), so the
+// per-token values the selection computes when the loss is fused into it
+// (moe_route's aux_part, finished by moe_seq_balance_loss_part) are the same.
 //
 // Three deterministic passes, no atomics:
 //  1. token  -- one warp per token: s, its row sum (fixed butterfly), the
@@ -224,45 +224,90 @@ extern "C" moe_status moe_seq_balance_loss(const float* logits, int T, int E, in
   return MOE_OK;
 }
 
-extern "C" moe_status moe_seq_balance_loss_rows_workspace_size(int T, int E, int seq_len,
-                                                                size_t* bytes) {
-  using namespace moe;
-  if (!bytes || T < 0 || E <= 0 || seq_len <= 0) return MOE_ERR_INVALID_ARG;
-  const int64_t chunks = static_cast<int64_t>(T / seq_len) * ((seq_len + kAuxChunk - 1) / kAuxChunk);
-  *bytes = align256(static_cast<size_t>(chunks) * E * sizeof(float)) +
-           align256(static_cast<size_t>(chunks) * E * sizeof(int32_t));
-  return MOE_OK;
+namespace moe {
+namespace {
+
+// The loss from the per-8-token partials moe_route wrote (aux_part): one CTA
+// per sequence; thread (e, j) sums blocks j, j + R, ... of expert e in order,
+// the R partial sums are added in j order, then f, P and a fixed-order tree
+// over the experts give the loss.
+__global__ void __launch_bounds__(1024) aux_part_final_kernel(
+    const float* __restrict__ part, int E, int Ep, int R, int K, int seq_len, float alpha,
+    float* __restrict__ loss, float* __restrict__ f_out, float* __restrict__ p_out) {
+  __shared__ float ssum[1024];
+  __shared__ float scnt[1024];
+  __shared__ float red[1024];
+  const int e = threadIdx.x % Ep, j = threadIdx.x / Ep;
+  const int q = blockIdx.x;
+  const int nb = seq_len / 8;
+  float acc = 0.f, cnt = 0.f;
+  if (e < E) {
+    const float* base = part + static_cast<int64_t>(q) * nb * 2 * E + e;
+    int b = j;
+    for (; b + 7 * R < nb; b += 8 * R) {  // eight loads in flight, added in block order
+      float v[8], c[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[i] = __ldg(base + static_cast<int64_t>(b + i * R) * 2 * E);
+        c[i] = __ldg(base + static_cast<int64_t>(b + i * R) * 2 * E + E);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc = __fadd_rn(acc, v[i]);
+        cnt = __fadd_rn(cnt, c[i]);
+      }
+    }
+    for (; b < nb; b += R) {
+      acc = __fadd_rn(acc, __ldg(base + static_cast<int64_t>(b) * 2 * E));
+      cnt = __fadd_rn(cnt, __ldg(base + static_cast<int64_t>(b) * 2 * E + E));
+    }
+  }
+  ssum[threadIdx.x] = acc;
+  scnt[threadIdx.x] = cnt;
+  __syncthreads();
+  float term = 0.f;
+  if (j == 0) {
+    if (e < E) {
+      float a2 = ssum[e], c2 = scnt[e];
+      for (int jj = 1; jj < R; ++jj) {
+        a2 = __fadd_rn(a2, ssum[jj * Ep + e]);
+        c2 = __fadd_rn(c2, scnt[jj * Ep + e]);
+      }
+      // f_i = E/(K S) * count, P_i = sum / S
+      const float f = __fdiv_rn(static_cast<float>(E) * c2,
+                                static_cast<float>(K) * static_cast<float>(seq_len));
+      const float pv = __fdiv_rn(a2, static_cast<float>(seq_len));
+      if (f_out) f_out[static_cast<int64_t>(q) * E + e] = f;
+      if (p_out) p_out[static_cast<int64_t>(q) * E + e] = pv;
+      term = __fmul_rn(f, pv);
+    }
+    red[e] = term;
+  }
+  __syncthreads();
+  for (int wdt = Ep >> 1; wdt > 0; wdt >>= 1) {
+    if (threadIdx.x < wdt) red[threadIdx.x] = __fadd_rn(red[threadIdx.x], red[threadIdx.x + wdt]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) loss[q] = __fmul_rn(alpha, red[0]);
 }
 
-// The loss from the per-token rows moe_route wrote (aux_rows): the chunk and
-// final passes of moe_seq_balance_loss, without its token pass.
-extern "C" moe_status moe_seq_balance_loss_rows(const float* rows, int T, int E, int K,
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_seq_balance_loss_part(const float* aux_part, int T, int E, int K,
                                                 int seq_len, float alpha, float* loss,
-                                                float* f_out, float* p_out, void* ws,
-                                                size_t ws_bytes, moe_stream_t stream) {
+                                                float* f_out, float* p_out, moe_stream_t stream) {
   using namespace moe;
   if (T < 0 || E <= 0 || K <= 0 || seq_len <= 0) return MOE_ERR_INVALID_ARG;
-  if (K > E || K > 32 || T % seq_len != 0) return MOE_ERR_SHAPE;
+  if (K > E || K > 32 || T % seq_len != 0 || seq_len % 8 != 0) return MOE_ERR_SHAPE;
   if (E > 1024) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
-  if (!rows || !loss) return MOE_ERR_INVALID_ARG;
-  size_t need = 0;
-  moe_seq_balance_loss_rows_workspace_size(T, E, seq_len, &need);
-  if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int n_seq = T / seq_len;
-  const int cps = (seq_len + kAuxChunk - 1) / kAuxChunk;
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  float* psum = reinterpret_cast<float*>(w);
-  w += align256(static_cast<size_t>(n_seq) * cps * E * sizeof(float));
-  int32_t* pcnt = reinterpret_cast<int32_t*>(w);
-  const int ethreads = (E + 31) / 32 * 32;
-  aux_chunk_kernel<<<n_seq * cps, ethreads, 0, st>>>(rows, E, seq_len, cps, psum, pcnt);
-  MOE_CUDA_CHECK_LAUNCH();
-  int fthreads = 32;
-  while (fthreads < E) fthreads <<= 1;
-  aux_final_kernel<<<n_seq, fthreads, fthreads * sizeof(float), st>>>(
-      psum, pcnt, E, K, seq_len, cps, alpha, loss, f_out, p_out);
+  if (!aux_part || !loss) return MOE_ERR_INVALID_ARG;
+  int Ep = 32;
+  while (Ep < E) Ep <<= 1;
+  const int R = 1024 / Ep;
+  aux_part_final_kernel<<<T / seq_len, Ep * R, 0, static_cast<cudaStream_t>(stream)>>>(
+      aux_part, E, Ep, R, K, seq_len, alpha, loss, f_out, p_out);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }

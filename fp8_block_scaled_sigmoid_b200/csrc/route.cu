@@ -179,13 +179,13 @@ __device__ __forceinline__ Cand warp_best(Cand c) {
 // Loss", eqs. (17)-(20)) from the raw affinities s this warp already holds:
 // s' = s / sum_j s_j (the sum in a fixed order: each lane's experts in turn,
 // then a butterfly over the lanes) and the raw top-K of s over all E experts
-// (ties to the lower index, no bias, no group limit); writes s' with the sign
-// bit set on the K members (s' > 0, so the sign carries the membership).
-// The arithmetic and orders are those of moe_seq_balance_loss's token pass,
-// so both give the same bytes.
+// (ties to the lower index, no bias, no group limit), as s' and a 0/1
+// membership per expert.  The arithmetic and orders are those of
+// moe_seq_balance_loss's token pass.
 template <int P>
-__device__ __forceinline__ void aux_token_row(const float (&s)[P], int t, int E, int K, int lane,
-                                              float* __restrict__ rows) {
+__device__ __forceinline__ void aux_token_row(const float (&s)[P], int E, int K, int lane,
+                                              float* __restrict__ s_norm,
+                                              uint8_t* __restrict__ member) {
   const int e0 = lane * P;
   float sum = 0.f;
 #pragma unroll
@@ -229,25 +229,23 @@ __device__ __forceinline__ void aux_token_row(const float (&s)[P], int t, int E,
 #pragma unroll
   for (int i = 0; i < P; ++i)
     if (e0 + i < E) {
-      const float v = __fdiv_rn(s[i], sum);
-      rows[static_cast<int64_t>(t) * E + e0 + i] = ((taken >> i) & 1u) ? -v : v;
+      s_norm[e0 + i] = __fdiv_rn(s[i], sum);
+      member[e0 + i] = static_cast<uint8_t>((taken >> i) & 1u);
     }
 }
 
 constexpr int kSelThreads = 256;
 
-// P = experts per lane (lane l owns experts l*P .. l*P+P-1).
+// One token per warp; P = experts per lane (lane l owns experts l*P ..
+// l*P+P-1).  Leaves the token's raw affinities in sc.
 template <int P>
-__global__ void __launch_bounds__(kSelThreads) route_select_kernel(
-    const float* __restrict__ part, int splits, int T, int E, int G, int M, int K,
+__device__ __forceinline__ void select_token(
+    const float* __restrict__ part, int splits, int t, int T, int E, int G, int M, int K,
     const float* __restrict__ bias, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
-    float* __restrict__ logits_out, float* __restrict__ aux_rows) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (kSelThreads / 32) + (threadIdx.x >> 5);
-  if (t >= T) return;
+    float* __restrict__ logits_out, int lane, float (&sc)[P]) {
   const int e0 = lane * P;
   const int gs = E / G;
-  float beta[P], sc[P], z[P];
+  float beta[P], z[P];
   if (P % 4 == 0 && e0 + P <= E) {
     // whole lane in range: 16-byte loads (E % 16 == 0 keeps them aligned)
 #pragma unroll
@@ -423,15 +421,58 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
     idx_out[static_cast<int64_t>(t) * K + lane] = my_idx;
     gate_out[static_cast<int64_t>(t) * K + lane] = __fdiv_rn(my_s, ssum);
   }
-  if (aux_rows != nullptr) aux_token_row<P>(sc, t, E, K, lane, aux_rows);
+}
+
+// Selection, and with aux_part the balance loss's per-block partials: each
+// warp writes its token's s' and raw top-K membership to shared memory, then
+// the CTA sums its 8 tokens in token order per expert -> aux_part[blk][0][e]
+// (sum of s') and aux_part[blk][1][e] (members, an exact small integer).
+template <int P>
+__global__ void __launch_bounds__(kSelThreads) route_select_kernel(
+    const float* __restrict__ part, int splits, int T, int E, int G, int M, int K,
+    const float* __restrict__ bias, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+    float* __restrict__ logits_out, float* __restrict__ aux_part) {
+  extern __shared__ float aux_sm[];  // [8][E] s', then [8][E] membership bytes
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int t = blockIdx.x * (kSelThreads / 32) + w;
+  float sc[P];
+  if (t < T)
+    select_token<P>(part, splits, t, T, E, G, M, K, bias, idx_out, gate_out, logits_out, lane, sc);
+  if (aux_part == nullptr) return;  // the same for the whole grid
+  float* sp = aux_sm + w * E;
+  uint8_t* sm8 = reinterpret_cast<uint8_t*>(aux_sm + (kSelThreads / 32) * E) + w * E;
+  if (t < T) {
+    aux_token_row<P>(sc, E, K, lane, sp, sm8);
+  } else {
+    for (int e = lane; e < E; e += 32) {
+      sp[e] = 0.f;
+      sm8[e] = 0;
+    }
+  }
+  __syncthreads();
+  const uint8_t* mem = reinterpret_cast<const uint8_t*>(aux_sm + (kSelThreads / 32) * E);
+  float* dst = aux_part + static_cast<int64_t>(blockIdx.x) * 2 * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float acc = 0.f;
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < kSelThreads / 32; ++j) {
+      acc = __fadd_rn(acc, aux_sm[j * E + e]);
+      cnt += mem[j * E + e];
+    }
+    dst[e] = acc;
+    dst[E + e] = static_cast<float>(cnt);
+  }
 }
 
 template <int P>
 void launch_select(int blocks, cudaStream_t st, const float* part, int splits, int T, int E,
                    int G, int M, int K, const float* bias, int32_t* idx, float* gate,
                    float* logits, float* aux) {
-  route_select_kernel<P><<<blocks, kSelThreads, 0, st>>>(part, splits, T, E, G, M, K, bias, idx,
-                                                          gate, logits, aux);
+  // 8 tokens x E x (4 + 1) bytes <= 40 KB for E <= 1024
+  const size_t sm = aux ? static_cast<size_t>(kSelThreads / 32) * E * 5 : 0;
+  route_select_kernel<P><<<blocks, kSelThreads, sm, st>>>(part, splits, T, E, G, M, K, bias, idx,
+                                                           gate, logits, aux);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -451,7 +492,7 @@ extern "C" moe_status moe_route_workspace_size(int T, int d, int E, size_t* byte
 extern "C" moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* centroids,
                                 const float* bias, int T, int d, int E, int G, int M, int K,
                                 int32_t* topk_idx, float* topk_gate, float* logits_out,
-                                float* aux_rows, void* ws, size_t ws_bytes, int32_t* dev_err,
+                                float* aux_part, void* ws, size_t ws_bytes, int32_t* dev_err,
                                 moe_stream_t stream) {
   using namespace moe;
   if (T < 0 || d <= 0 || E <= 0 || G <= 0 || M <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
@@ -489,13 +530,13 @@ extern "C" moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* 
 
   const int blocks = (T + kSelThreads / 32 - 1) / (kSelThreads / 32);
   const int P = (E + 31) / 32;
-  if (P <= 1) launch_select<1>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
-  else if (P <= 2) launch_select<2>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
-  else if (P <= 4) launch_select<4>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
-  else if (P <= 8) launch_select<8>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
-  else if (P <= 12) launch_select<12>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
-  else if (P <= 16) launch_select<16>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
-  else launch_select<32>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_rows);
+  if (P <= 1) launch_select<1>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
+  else if (P <= 2) launch_select<2>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
+  else if (P <= 4) launch_select<4>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
+  else if (P <= 8) launch_select<8>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
+  else if (P <= 12) launch_select<12>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
+  else if (P <= 16) launch_select<16>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
+  else launch_select<32>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }

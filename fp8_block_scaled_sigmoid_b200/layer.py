@@ -120,9 +120,11 @@ class MoELayer:
         i32, f32, u8 = torch.int32, torch.float32, torch.uint8
         self.idx = torch.empty(T, K, dtype=i32, device=dev)
         # router logits of the last step (keep_logits), and the balance loss's
-        # per-token rows written by the router's selection pass (balance_loss)
+        # per-8-token partial sums written by the router's selection pass
+        # (balance_loss)
         self.logits = torch.empty(T, E, dtype=f32, device=dev) if keep_logits else None
-        self.aux_rows = torch.empty(T, E, dtype=f32, device=dev) if balance_loss else None
+        self.aux_part = (torch.empty((T + 7) // 8, 2, E, dtype=f32, device=dev)
+                         if balance_loss else None)
         self.gate = torch.empty(T, K, dtype=f32, device=dev)
         self.route_ws = torch.empty(max(_abi.moe_route_workspace_size(T, d, E), 16), dtype=u8, device=dev)
         self.Xq = torch.empty(P + T, d, dtype=u8, device=dev)
@@ -149,7 +151,7 @@ class MoELayer:
         c = self.cfg
         _abi.moe_route(u, self.centroids, self.bias, c.G, c.M, c.K, self.idx, self.gate,
                        logits_out=self.logits, ws=self.route_ws, dev_err=self.dev_err,
-                       aux_rows=self.aux_rows)
+                       aux_part=self.aux_part)
 
     def step_permute(self):
         """Counts, offsets, row maps and the tile table (no row moves yet)."""
@@ -302,11 +304,11 @@ class MoELayer:
         """The complementary sequence-wise balance loss (eqs. 17-20) of the
         last step's routing, per sequence of seq_len tokens.  With
         balance_loss=True the router's selection pass already wrote the
-        per-token rows and two short reductions finish the loss; with
-        keep_logits=True the loss is computed from the kept logits."""
-        if self.aux_rows is not None:
-            return _abi.moe_seq_balance_loss_rows(self.aux_rows, self.cfg.K, seq_len, alpha,
-                                                  with_fp)
+        per-8-token partial sums and one short reduction finishes the loss;
+        with keep_logits=True the loss is computed from the kept logits."""
+        if self.aux_part is not None:
+            return _abi.moe_seq_balance_loss_part(self.aux_part, self.T, self.cfg.K, seq_len,
+                                                  alpha, with_fp)
         assert self.logits is not None, "build the layer with balance_loss or keep_logits"
         return _abi.moe_seq_balance_loss(self.logits, self.cfg.K, seq_len, alpha, with_fp)
 

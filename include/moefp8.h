@@ -128,13 +128,14 @@ moe_status fp8_quant_128x128_pow2(const uint16_t* w, int64_t ldw, int rows, int 
  *   u          bf16 [T][ldu];  centroids bf16 [E][d];  bias fp32 [E]
  *   topk_idx   int32 [T][K];   topk_gate fp32 [T][K]
  *   logits_out fp32 [T][E] or NULL (the logits the selection used)
- *   aux_rows   fp32 [T][E] or NULL: the per-token rows of the complementary
- *              sequence-wise balance loss ([ANN] eqs. (17)-(20)), computed
- *              from the same affinities in the same pass: s' = s / sum_j s_j
- *              with the sign bit set on the token's raw top-K (over all E
- *              experts, no bias, no group limit, ties to the lower index, K
- *              the routing K); moe_seq_balance_loss_rows turns them into the
- *              loss.  The bytes equal moe_seq_balance_loss's own token pass.
+ *   aux_part   fp32 [ceil(T/8)][2][E] or NULL: the complementary sequence-wise
+ *              balance loss's partial sums ([ANN] eqs. (17)-(20)), computed from
+ *              the same affinities in the same pass.  For each block b of 8
+ *              tokens (8b .. 8b+7): [b][0][i] = the sum over its tokens of
+ *              s'_{i,t} = s_{i,t} / sum_j s_{j,t}, [b][1][i] = how many of them
+ *              have expert i in their raw top-K (over all E experts, no bias,
+ *              no group limit, ties to the lower index, K the routing K).
+ *              moe_seq_balance_loss_part turns them into the loss.
  *   ws         scratch of moe_route_workspace_size() bytes (may be NULL if 0)
  * Limits: d % 128 == 0, E % 16 == 0, 16 <= E <= 1024, E % G == 0,
  * 1 <= M <= G <= 32, K <= E, K % M == 0 when M < G, K <= 32.
@@ -143,7 +144,7 @@ moe_status moe_route_workspace_size(int T, int d, int E, size_t* bytes);
 moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* centroids,
                      const float* bias, int T, int d, int E, int G, int M, int K,
                      int32_t* topk_idx, float* topk_gate, float* logits_out,
-                     float* aux_rows, void* ws, size_t ws_bytes, int32_t* dev_err,
+                     float* aux_part, void* ws, size_t ws_bytes, int32_t* dev_err,
                      moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
@@ -474,15 +475,16 @@ moe_status moe_seq_balance_loss(const float* logits, int T, int E, int K, int se
                                 float alpha, float* loss, float* f, float* P, void* ws,
                                 size_t ws_bytes, moe_stream_t stream);
 
-/* moe_seq_balance_loss_rows -- the same loss from the per-token rows that
- * moe_route wrote to aux_rows (its chunk and final passes only; the token
- * pass is fused into the router's selection).  Same outputs, limits and
- * determinism as moe_seq_balance_loss; K must be the routing K the rows were
- * made with.  ws: moe_seq_balance_loss_rows_workspace_size bytes. */
-moe_status moe_seq_balance_loss_rows_workspace_size(int T, int E, int seq_len, size_t* bytes);
-moe_status moe_seq_balance_loss_rows(const float* rows, int T, int E, int K, int seq_len,
-                                     float alpha, float* loss, float* f, float* P, void* ws,
-                                     size_t ws_bytes, moe_stream_t stream);
+/* moe_seq_balance_loss_part -- the same loss from the per-8-token partial
+ * sums that moe_route wrote to aux_part (the token pass fused into the
+ * router's selection; one more launch, no workspace).  Per sequence the
+ * partials are added in a fixed order (deterministic); the result equals
+ * moe_seq_balance_loss's up to the order of the fp32 sums.  f and P may be
+ * NULL.  Limits: T % seq_len == 0, seq_len % 8 == 0, K <= min(E, 32),
+ * E <= 1024; K must be the routing K the partials were made with. */
+moe_status moe_seq_balance_loss_part(const float* aux_part, int T, int E, int K, int seq_len,
+                                     float alpha, float* loss, float* f, float* P,
+                                     moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * moe_fp8_mma_peak -- measurement helper: the dense FP8 tensor-core rate of

@@ -78,10 +78,11 @@ def test_layer_seq_balance_loss(cuda_dev):
 
 @pytest.mark.parametrize("cfg_name,S", [("tiny", 64), ("v3_prefill", 4096), ("v3_prefill", 1024),
                                         ("v4_pro", 2048)])
-def test_route_fused_rows_match_three_pass(cuda_dev, cfg_name, S):
-    """The token pass fused into the router's selection writes the same rows
-    as the standalone token pass on the same logits, so both routes to the
-    loss give identical bytes (loss, f, P)."""
+def test_route_fused_partials_match_three_pass(cuda_dev, cfg_name, S):
+    """The token pass fused into the router's selection (per-8-token partial
+    sums) gives the three-pass loss on the same logits: the membership counts
+    (hence f) exactly, P and the loss up to the order of the fp32 sums; the
+    routing itself is unchanged."""
     from fp8_block_scaled_sigmoid_b200 import configs, inputs
     cfg = configs.PRESETS[cfg_name]
     if cfg.T > 4096:
@@ -90,15 +91,24 @@ def test_route_fused_rows_match_three_pass(cuda_dev, cfg_name, S):
     cent = inputs.draw_centroids(cfg, cuda_dev)
     bias = inputs.draw_bias(cfg, cuda_dev)
     logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=cuda_dev)
-    rows = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=cuda_dev)
+    part = torch.empty((cfg.T + 7) // 8, 2, cfg.E, dtype=torch.float32, device=cuda_dev)
     idx, gate = _abi.moe_route(u, cent, bias, cfg.G, cfg.M, cfg.K, logits_out=logits,
-                               aux_rows=rows)
+                               aux_part=part)
     idx2, gate2 = _abi.moe_route(u, cent, bias, cfg.G, cfg.M, cfg.K)
-    a = _abi.moe_seq_balance_loss_rows(rows, cfg.K, S, with_fp=True)
-    b = _abi.moe_seq_balance_loss(logits, cfg.K, S, with_fp=True)
+    la, fa, Pa = _abi.moe_seq_balance_loss_part(part, cfg.T, cfg.K, S, with_fp=True)
+    la2 = _abi.moe_seq_balance_loss_part(part, cfg.T, cfg.K, S)
+    lb, fb, Pb = _abi.moe_seq_balance_loss(logits, cfg.K, S, with_fp=True)
     torch.cuda.synchronize()
     assert torch.equal(idx, idx2) and torch.equal(gate, gate2)   # routing unchanged
-    for x, y in zip(a, b):
-        assert torch.equal(x, y)
-    # membership: exactly K negative entries per token
-    assert torch.all((rows < 0).sum(1) == cfg.K)
+    assert torch.equal(la, la2), "not deterministic"
+    assert torch.equal(fa, fb)
+    # every token counts K members
+    assert torch.all(part[:, 1, :].sum(1) == 8 * cfg.K)
+    assert torch.allclose(Pa, Pb, rtol=1e-5, atol=1e-9)
+    assert torch.allclose(la, lb, rtol=1e-5, atol=0)
+    # and against the oracle on the same logits
+    lo, fo, Po, margin = O.seq_balance_loss(npraw(logits).astype(np.float64), cfg.K, S, 1e-4)
+    near = (margin < 1e-6).reshape(-1, S).sum(axis=1)
+    assert np.allclose(npraw(Pa), Po, rtol=1e-4, atol=1e-7)
+    clean = near == 0
+    assert np.allclose(npraw(la)[clean], lo[clean], rtol=1e-4, atol=0)
