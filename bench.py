@@ -487,7 +487,9 @@ def run_gpu(args):
                                            ws=rws), reps)
     t_aux = timed(lambda: _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K,
                                          ws=rws, aux_part=part), reps)
-    t_red = timed(lambda: _abi.moe_seq_balance_loss_part(part, cfg.T, cfg.K, cfg.T), reps)
+    pws = torch.empty(max(_abi.moe_seq_balance_loss_part_ws(cfg.T, cfg.E, cfg.T), 16),
+                      dtype=torch.uint8, device=dev)
+    t_red = timed(lambda: _abi.moe_seq_balance_loss_part(part, cfg.T, cfg.K, cfg.T, ws=pws), reps)
     _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K, logits_out=logits, ws=rws)
     t_3p = timed(lambda: _abi.moe_seq_balance_loss(logits, cfg.K, cfg.T, ws=bl_ws), reps)
     barrier()
@@ -495,7 +497,7 @@ def run_gpu(args):
                     "route_us": round(t_plain, 2), "route_with_partials_us": round(t_aux, 2),
                     "reduction_us": round(t_red, 2), "three_pass_from_logits_us": round(t_3p, 2),
                     "seq_len": cfg.T}
-    del logits, part, rws, bl_ws
+    del logits, part, rws, bl_ws, pws
 
     # roofline of the dominant kernel (grouped GEMM 1 with the SwiGLU epilogue)
     counts = layer.perm["counts"].cpu()

@@ -63,7 +63,8 @@ _SIGS = {
     "moe_seq_balance_loss_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
     "moe_seq_balance_loss": (_i, [_p, _i, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
     "moe_fp8_mma_peak": (_i, [_i, _i, _i, _p, _p, _p]),
-    "moe_seq_balance_loss_part": (_i, [_p, _i, _i, _i, _i, _f, _p, _p, _p, _p]),
+    "moe_seq_balance_loss_part_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
+    "moe_seq_balance_loss_part": (_i, [_p, _i, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
 }
 
 EP_F32 = 0
@@ -86,7 +87,7 @@ LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant
                      "moe_tile_table": 1, "moe_segment_ids": 1,
                      "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1,
                      "moe_seq_balance_loss": 3, "moe_fp8_mma_peak": 1,
-                     "moe_seq_balance_loss_part": 1}
+                     "moe_seq_balance_loss_part": 2}
 launch_count = 0
 
 
@@ -450,18 +451,30 @@ def moe_seq_balance_loss(logits, K, seq_len, alpha=1e-4, with_fp=False, ws=None,
     return loss
 
 
-def moe_seq_balance_loss_part(part, T, K, seq_len, alpha=1e-4, with_fp=False, stream=None):
+def moe_seq_balance_loss_part_ws(T, E, seq_len) -> int:
+    n = _sz(0)
+    _check(lib().moe_seq_balance_loss_part_workspace_size(T, E, seq_len, ctypes.byref(n)),
+           "moe_seq_balance_loss_part_workspace_size")
+    return n.value
+
+
+def moe_seq_balance_loss_part(part, T, K, seq_len, alpha=1e-4, with_fp=False, ws=None,
+                              stream=None):
     """The balance loss from moe_route's aux_part fp32 [ceil(T/8)][2][E] (K =
     the routing K).  Returns loss fp32 [T/seq_len], or (loss, f, P)."""
     E = part.shape[-1]
     dev = _dev(part)
+    if ws is None:
+        ws = torch.empty(max(moe_seq_balance_loss_part_ws(T, E, seq_len), 16), dtype=torch.uint8,
+                         device=dev)
     n_seq = T // seq_len if seq_len > 0 else 0
     loss = torch.empty(max(n_seq, 1), dtype=torch.float32, device=dev)
     f = torch.empty(max(n_seq, 1), E, dtype=torch.float32, device=dev) if with_fp else None
     P = torch.empty(max(n_seq, 1), E, dtype=torch.float32, device=dev) if with_fp else None
     _count("moe_seq_balance_loss_part")
     _check(lib().moe_seq_balance_loss_part(_ptr(part), T, E, K, seq_len, float(alpha), _ptr(loss),
-                                           _ptr(f), _ptr(P), _stream(stream)),
+                                           _ptr(f), _ptr(P), _ptr(ws),
+                                           ws.numel() * ws.element_size(), _stream(stream)),
            "moe_seq_balance_loss_part")
     loss = loss[:n_seq]
     if with_fp:

@@ -227,87 +227,111 @@ extern "C" moe_status moe_seq_balance_loss(const float* logits, int T, int E, in
 namespace moe {
 namespace {
 
-// The loss from the per-8-token partials moe_route wrote (aux_part): one CTA
-// per sequence; thread (e, j) sums blocks j, j + R, ... of expert e in order,
-// the R partial sums are added in j order, then f, P and a fixed-order tree
-// over the experts give the loss.
-__global__ void __launch_bounds__(1024) aux_part_final_kernel(
-    const float* __restrict__ part, int E, int Ep, int R, int K, int seq_len, float alpha,
-    float* __restrict__ loss, float* __restrict__ f_out, float* __restrict__ p_out) {
-  __shared__ float ssum[1024];
-  __shared__ float scnt[1024];
-  __shared__ float red[1024];
-  const int e = threadIdx.x % Ep, j = threadIdx.x / Ep;
-  const int q = blockIdx.x;
-  const int nb = seq_len / 8;
+// The loss from the per-8-token partials moe_route wrote (aux_part), in two
+// deterministic levels.  Level 1: CTA (q, g) sums blocks g*G .. g*G+G-1 of
+// sequence q in block order, one thread per expert -> ws[q][g][2][E].
+// Level 2: one CTA per sequence adds its groups in order, then f, P and a
+// fixed-order tree over the experts give the loss.
+constexpr int kPartGroups = 16;
+
+__global__ void aux_part_group_kernel(const float* __restrict__ part, int E, int nb, int G,
+                                      float* __restrict__ ws) {
+  const int e = threadIdx.x;
+  if (e >= E) return;
+  const int q = blockIdx.y, g = blockIdx.x;
+  const int b0 = g * G, b1 = min(nb, b0 + G);
+  const float* base = part + static_cast<int64_t>(q) * nb * 2 * E + e;
   float acc = 0.f, cnt = 0.f;
-  if (e < E) {
-    const float* base = part + static_cast<int64_t>(q) * nb * 2 * E + e;
-    int b = j;
-    for (; b + 7 * R < nb; b += 8 * R) {  // eight loads in flight, added in block order
-      float v[8], c[8];
+  int b = b0;
+  for (; b + 8 <= b1; b += 8) {  // eight loads in flight, added in block order
+    float v[8], c[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[i] = __ldg(base + static_cast<int64_t>(b + i * R) * 2 * E);
-        c[i] = __ldg(base + static_cast<int64_t>(b + i * R) * 2 * E + E);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        acc = __fadd_rn(acc, v[i]);
-        cnt = __fadd_rn(cnt, c[i]);
-      }
+    for (int i = 0; i < 8; ++i) {
+      v[i] = __ldg(base + static_cast<int64_t>(b + i) * 2 * E);
+      c[i] = __ldg(base + static_cast<int64_t>(b + i) * 2 * E + E);
     }
-    for (; b < nb; b += R) {
-      acc = __fadd_rn(acc, __ldg(base + static_cast<int64_t>(b) * 2 * E));
-      cnt = __fadd_rn(cnt, __ldg(base + static_cast<int64_t>(b) * 2 * E + E));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      acc = __fadd_rn(acc, v[i]);
+      cnt = __fadd_rn(cnt, c[i]);
     }
   }
-  ssum[threadIdx.x] = acc;
-  scnt[threadIdx.x] = cnt;
-  __syncthreads();
+  for (; b < b1; ++b) {
+    acc = __fadd_rn(acc, __ldg(base + static_cast<int64_t>(b) * 2 * E));
+    cnt = __fadd_rn(cnt, __ldg(base + static_cast<int64_t>(b) * 2 * E + E));
+  }
+  float* dst = ws + (static_cast<int64_t>(q) * gridDim.x + g) * 2 * E;
+  dst[e] = acc;
+  dst[E + e] = cnt;
+}
+
+// blockDim = Ep (a power of two >= E, <= 1024)
+__global__ void aux_part_final_kernel(const float* __restrict__ ws, int E, int NG, int K,
+                                      int seq_len, float alpha, float* __restrict__ loss,
+                                      float* __restrict__ f_out, float* __restrict__ p_out) {
+  extern __shared__ float red[];
+  const int e = threadIdx.x;
+  const int q = blockIdx.x;
   float term = 0.f;
-  if (j == 0) {
-    if (e < E) {
-      float a2 = ssum[e], c2 = scnt[e];
-      for (int jj = 1; jj < R; ++jj) {
-        a2 = __fadd_rn(a2, ssum[jj * Ep + e]);
-        c2 = __fadd_rn(c2, scnt[jj * Ep + e]);
-      }
-      // f_i = E/(K S) * count, P_i = sum / S
-      const float f = __fdiv_rn(static_cast<float>(E) * c2,
-                                static_cast<float>(K) * static_cast<float>(seq_len));
-      const float pv = __fdiv_rn(a2, static_cast<float>(seq_len));
-      if (f_out) f_out[static_cast<int64_t>(q) * E + e] = f;
-      if (p_out) p_out[static_cast<int64_t>(q) * E + e] = pv;
-      term = __fmul_rn(f, pv);
+  if (e < E) {
+    const float* base = ws + static_cast<int64_t>(q) * NG * 2 * E + e;
+    float acc = 0.f, cnt = 0.f;
+    for (int g = 0; g < NG; ++g) {
+      acc = __fadd_rn(acc, __ldg(base + static_cast<int64_t>(g) * 2 * E));
+      cnt = __fadd_rn(cnt, __ldg(base + static_cast<int64_t>(g) * 2 * E + E));
     }
-    red[e] = term;
+    // f_i = E/(K S) * count, P_i = sum / S
+    const float f = __fdiv_rn(static_cast<float>(E) * cnt,
+                              static_cast<float>(K) * static_cast<float>(seq_len));
+    const float pv = __fdiv_rn(acc, static_cast<float>(seq_len));
+    if (f_out) f_out[static_cast<int64_t>(q) * E + e] = f;
+    if (p_out) p_out[static_cast<int64_t>(q) * E + e] = pv;
+    term = __fmul_rn(f, pv);
   }
+  red[e] = term;
   __syncthreads();
-  for (int wdt = Ep >> 1; wdt > 0; wdt >>= 1) {
-    if (threadIdx.x < wdt) red[threadIdx.x] = __fadd_rn(red[threadIdx.x], red[threadIdx.x + wdt]);
+  for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
+    if (e < w) red[e] = __fadd_rn(red[e], red[e + w]);
     __syncthreads();
   }
-  if (threadIdx.x == 0) loss[q] = __fmul_rn(alpha, red[0]);
+  if (e == 0) loss[q] = __fmul_rn(alpha, red[0]);
 }
 
 }  // namespace
 }  // namespace moe
 
+extern "C" moe_status moe_seq_balance_loss_part_workspace_size(int T, int E, int seq_len,
+                                                                size_t* bytes) {
+  using namespace moe;
+  if (!bytes || T < 0 || E <= 0 || seq_len <= 0) return MOE_ERR_INVALID_ARG;
+  *bytes = align256(static_cast<size_t>(T / seq_len) * kPartGroups * 2 * E * sizeof(float));
+  return MOE_OK;
+}
+
 extern "C" moe_status moe_seq_balance_loss_part(const float* aux_part, int T, int E, int K,
                                                 int seq_len, float alpha, float* loss,
-                                                float* f_out, float* p_out, moe_stream_t stream) {
+                                                float* f_out, float* p_out, void* ws,
+                                                size_t ws_bytes, moe_stream_t stream) {
   using namespace moe;
   if (T < 0 || E <= 0 || K <= 0 || seq_len <= 0) return MOE_ERR_INVALID_ARG;
   if (K > E || K > 32 || T % seq_len != 0 || seq_len % 8 != 0) return MOE_ERR_SHAPE;
   if (E > 1024) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
   if (!aux_part || !loss) return MOE_ERR_INVALID_ARG;
+  size_t need = 0;
+  moe_seq_balance_loss_part_workspace_size(T, E, seq_len, &need);
+  if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int n_seq = T / seq_len, nb = seq_len / 8;
+  const int G = (nb + kPartGroups - 1) / kPartGroups;
+  const int NG = (nb + G - 1) / G;  // groups actually holding blocks
+  float* w = static_cast<float*>(ws);
+  aux_part_group_kernel<<<dim3(NG, n_seq), (E + 31) / 32 * 32, 0, st>>>(aux_part, E, nb, G, w);
+  MOE_CUDA_CHECK_LAUNCH();
   int Ep = 32;
   while (Ep < E) Ep <<= 1;
-  const int R = 1024 / Ep;
-  aux_part_final_kernel<<<T / seq_len, Ep * R, 0, static_cast<cudaStream_t>(stream)>>>(
-      aux_part, E, Ep, R, K, seq_len, alpha, loss, f_out, p_out);
+  aux_part_final_kernel<<<n_seq, Ep, Ep * sizeof(float), st>>>(w, E, NG, K, seq_len, alpha, loss,
+                                                                f_out, p_out);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }

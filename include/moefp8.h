@@ -477,14 +477,16 @@ moe_status moe_seq_balance_loss(const float* logits, int T, int E, int K, int se
 
 /* moe_seq_balance_loss_part -- the same loss from the per-8-token partial
  * sums that moe_route wrote to aux_part (the token pass fused into the
- * router's selection; one more launch, no workspace).  Per sequence the
+ * router's selection; two short reductions follow).  Per sequence the
  * partials are added in a fixed order (deterministic); the result equals
  * moe_seq_balance_loss's up to the order of the fp32 sums.  f and P may be
- * NULL.  Limits: T % seq_len == 0, seq_len % 8 == 0, K <= min(E, 32),
- * E <= 1024; K must be the routing K the partials were made with. */
+ * NULL.  ws: moe_seq_balance_loss_part_workspace_size bytes.
+ * Limits: T % seq_len == 0, seq_len % 8 == 0, K <= min(E, 32), E <= 1024;
+ * K must be the routing K the partials were made with. */
+moe_status moe_seq_balance_loss_part_workspace_size(int T, int E, int seq_len, size_t* bytes);
 moe_status moe_seq_balance_loss_part(const float* aux_part, int T, int E, int K, int seq_len,
-                                     float alpha, float* loss, float* f, float* P,
-                                     moe_stream_t stream);
+                                     float alpha, float* loss, float* f, float* P, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * moe_fp8_mma_peak -- measurement helper: the dense FP8 tensor-core rate of

@@ -55,11 +55,11 @@ def test_max_m_tiles_bound():
     (lambda L: L.moe_route(None, 256, None, None, 8, 256, 2048, 8, 4, 8, None, None, None,
                            None, None, 0, None, None), 4),                    # E > 1024
     (lambda L: L.moe_seq_balance_loss_part(None, 96, 16, 4, 30, ctypes.c_float(1e-4), None,
-                                           None, None, None), 2),            # T % seq_len
+                                           None, None, None, 0, None), 2),   # T % seq_len
     (lambda L: L.moe_seq_balance_loss_part(None, 100, 16, 4, 50, ctypes.c_float(1e-4), None,
-                                           None, None, None), 2),            # seq_len % 8
+                                           None, None, None, 0, None), 2),   # seq_len % 8
     (lambda L: L.moe_seq_balance_loss_part(None, 96, 16, 4, 48, ctypes.c_float(1e-4), None,
-                                           None, None, None), 1),            # NULL partials
+                                           None, None, None, 0, None), 1),   # NULL partials
     (lambda L: L.grouped_gemm_fp8_blockscaled(None, None, 10, None, None, None, None, None,
                                               None, 4, 1, 384, 128, 0, None, None, None,
                                               None, None), 2),                # N % 256
