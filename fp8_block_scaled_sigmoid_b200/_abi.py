@@ -45,9 +45,9 @@ _SIGS = {
     "fp8_quant_1x128_scatter": (_i, [_p, _i64, _i, _i, _p, _i, _i, _p, _p, _p, _p, _p]),
     "moe_segment_ids": (_i, [_p, _i, _i, _i64, _i64, _p, _p, _p]),
     "grouped_gemm_fp8_blockscaled": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
-                                          _i, _p, _p, _p, _p, _p]),
+                                          _i, _p, _p, _p, _p, _p, _p]),
     "grouped_gemm_fp8_pow2": (_i, [_p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i,
-                                   _i, _p, _p, _p, _p, _p]),
+                                   _i, _p, _p, _p, _p, _p, _p]),
     "swiglu_quant": (_i, [_p, _i, _i, _p, _p, _p]),
     "swiglu_quant_pow2": (_i, [_p, _i, _i, _p, _p, _p]),
     "fp8_quant_1x128_f32": (_i, [_p, _i64, _i, _i, _i, _p, _p, _p]),
@@ -383,10 +383,11 @@ def moe_segment_ids(counts, E, n_rows, ids=None, dev_err=None, stream=None, lead
 # ------------------------------------------------------------------ GEMM ---
 def grouped_gemm_fp8_blockscaled(A, sa, B, sb, offsets, tile_group, tile_start, n_tiles,
                                  max_tiles, ep=EP_F32, D=None, d_scale=None, dev_err=None,
-                                 stream=None, pow2=False, d_rows=None):
+                                 stream=None, pow2=False, d_rows=None, sched=None):
     """A uint8 [rows][K], sa fp32 [rows][K/128], B uint8 [G][N][K], sb fp32
     [G][N/128][K/128].  ep=EP_F32 -> D fp32 [rows][N] (d_rows int32 [rows]
     optionally sends row j's output to D row d_rows[j]); ep=EP_SWIGLU_QUANT ->
+    (sched: one device int32 -> dynamic work scheduling; the layer passes one)
     (h uint8 [rows][N/2], h_scale fp32 [rows][N/256]).  pow2 calls
     grouped_gemm_fp8_pow2 (every scale a power of two; the tensor core
     applies them)."""
@@ -402,8 +403,8 @@ def grouped_gemm_fp8_blockscaled(A, sa, B, sb, offsets, tile_group, tile_start, 
     _count(name)
     _check(getattr(lib(), name)(_ptr(A), _ptr(sa), rows, _ptr(B), _ptr(sb), _ptr(offsets),
                                 _ptr(tile_group), _ptr(tile_start), _ptr(n_tiles), max_tiles, G,
-                                N, K, ep, _ptr(D), _ptr(d_scale), _ptr(d_rows), _ptr(dev_err),
-                                _stream(stream)),
+                                N, K, ep, _ptr(D), _ptr(d_scale), _ptr(d_rows), _ptr(sched),
+                                _ptr(dev_err), _stream(stream)),
            name)
     return D if ep == EP_F32 else (D, d_scale)
 

@@ -4,7 +4,10 @@
 
 Each .cu under csrc/ compiles to an object under _build/ (in parallel), then
 one nvcc link makes the shared library next to this file.  No --use_fast_math:
-the quantisation path relies on IEEE division and the accurate expf.
+every rounding the quantisers and the router depend on is spelled out with
+explicitly rounded intrinsics (IEEE division of the scale, the accurate expf
+in the router's sigmoid); the SwiGLU epilogue's own __expf / __fdividef are
+chosen in the source, not by a compiler flag.
 """
 from __future__ import annotations
 

@@ -62,6 +62,19 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kRingBytes = 192 * 1024;
 constexpr int kMaxGroups = 1024;
 constexpr size_t kSmemBytes = 1024 + kRingBytes + 512 + (kMaxGroups + 1) * 4 + 2048 + 64;
+// Tail m-tiles of at most kTailRows rows (an expert's last rows past a whole
+// 128-row tile, or an expert with few rows) take the swapped path below.
+// Its promotion factors sa * sb for every (K block, weight half, row) are
+// staged in shared memory: 2 x kTailRows x kTailMaxKB floats.
+constexpr int kTailRows = 32;
+constexpr int kTailMaxKB = 64;
+constexpr int kTailFactorBytes = 2 * kTailRows * kTailMaxKB * 4;
+// work queue (4 slots) and the tail path's barriers and amax exchange
+constexpr int kWQ = 4;
+constexpr int kQueueBytes = 1024;     // barriers, slots and amax; the factors start at +640
+constexpr int kTailFactorOffset = 640;
+constexpr size_t kSmemPromoteBytes = kSmemBytes + kQueueBytes + kTailFactorBytes;
+static_assert(kSmemPromoteBytes <= 232448, "shared memory per CTA");
 
 struct GemmArgs {
   const float* sa;
@@ -76,11 +89,13 @@ struct GemmArgs {
   float* d_scale;
   int32_t* dev_err;
   const int32_t* d_rows;  // fp32 epilogue: output row of A row j (NULL: row j)
+  int32_t* sched;         // work counter (zeroed before the launch), NULL: static schedule
 };
 
 struct Work {
   int e, n_idx, row0, rows;  // expert, n-tile, first row and valid rows of the m-tile
   bool ok;
+  bool swp;  // a tail tile for the swapped path (rows <= kTailRows)
 };
 
 template <int SK>
@@ -100,7 +115,7 @@ __device__ __forceinline__ void load_tile_prefix(const GemmArgs& a, int* rstart,
 // [nN*rstart[e], nN*rstart[e+1]) and the row tile varies fastest inside.
 template <int RT>
 __device__ __forceinline__ Work decode_work(int w, int nN, const int* rstart, const GemmArgs& a) {
-  Work t{0, 0, 0, 0, false};
+  Work t{0, 0, 0, 0, false, false};
   const int j = w / nN;
   int lo = 0, hi = a.groups - 1;
   while (lo < hi) {  // last group whose first tile index is <= j
@@ -121,6 +136,7 @@ __device__ __forceinline__ Work decode_work(int w, int nN, const int* rstart, co
   t.rows = min(RT, seg1 - tile0);
   t.e = e;
   t.ok = true;
+  t.swp = t.rows <= kTailRows && a.K / kBK <= kTailMaxKB;
   return t;
 }
 
@@ -313,6 +329,148 @@ __device__ __forceinline__ bool epilogue_tile(const GemmArgs& args, const Work& 
   return write_tile<EP, false>(args, t, acc, warp, lane, N, xtile, xbar, amax_x, abort_v);
 }
 
+// ------------------------------------------------------- swapped tail tiles
+// A tile of at most kTailRows rows wastes most of a 128-row MMA and of the
+// promotion.  The swapped path computes its transpose instead: the weight
+// tile's two 128-row halves are the MMA's M side and the tail's (up to 32)
+// rows its N side (tcgen05 M = 128, N = 32), so each K block costs a quarter
+// of the tensor work, and the promotion folds 16 rows x 2 halves per thread:
+// TMEM lane = weight row c (32 q + lane of warp quarter q), column = tail row
+// m.  Warpgroup g takes rows 16 g .. 16 g + 15.  The factors f = sa * sb of
+// every (K block, half, row) are staged once per tile in shared memory, with
+// the same single rounding as the 128-row path, so a row's result is the same
+// sum of the same products: acc += f * partial per K block, in K order.
+struct TailCtl {
+  float* f;          // [kTailMaxKB][2][kTailRows]
+  float* amax;       // [2 warpgroups][4 quarters][16 rows]
+  uint64_t* staged;  // all 256 epilogue threads wrote their share of f
+  uint64_t* used;    // all 256 finished the K loop of the tile (f may be rewritten)
+  uint64_t* ax;      // [2]: a warpgroup's 4 warps wrote their row amaxes
+};
+
+template <int EP>
+__device__ __forceinline__ bool epilogue_tail(const GemmArgs& args, const Work& t, uint32_t tmem,
+                                              int warp, int lane, int KB, int N, int& tit,
+                                              int& ttile, uint64_t* tfull, uint64_t* tempty,
+                                              const TailCtl& tc, volatile int* abort_v) {
+  const int g = (warp - 4) >> 2;  // rows 16 g .. 16 g + 15 of the tail
+  const int q = warp & 3;         // TMEM lane quarter: weight rows 32 q .. 32 q + 31
+  const int c = q * 32 + lane;    // this thread's weight row inside a half
+  const int tid = threadIdx.x - 128;
+  const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+  const uint32_t ph = static_cast<uint32_t>(ttile & 1);
+  // the previous tail's K loop is over on every thread before f is rewritten
+  if (ttile > 0 &&
+      !__all_sync(0xffffffffu, mbar_wait(tc.used, ph ^ 1u, abort_v, args.dev_err)))
+    return false;
+  {
+    const float* sbh = args.sb + (static_cast<int64_t>(t.e) * (N / 128) + t.n_idx * 2) * KB;
+    for (int idx = tid; idx < KB * 2 * kTailRows; idx += kEpiThreads) {
+      const int kb = idx / (2 * kTailRows), h = (idx / kTailRows) & 1, m = idx % kTailRows;
+      float v = 0.f;
+      if (m < t.rows)
+        v = __fmul_rn(__ldg(args.sa + (static_cast<int64_t>(t.row0) + m) * KB + kb),
+                      __ldg(sbh + h * KB + kb));
+      tc.f[idx] = v;
+    }
+  }
+  mbar_arrive(tc.staged);
+  if (!__all_sync(0xffffffffu, mbar_wait(tc.staged, ph, abort_v, args.dev_err))) return false;
+  float acc0[16], acc1[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc0[i] = acc1[i] = 0.f;
+  for (int kb = 0; kb < KB; ++kb, ++tit) {
+    const int p = tit & 1;
+    if (!__all_sync(0xffffffffu, mbar_wait(&tfull[p], (tit >> 1) & 1, abort_v, args.dev_err)))
+      return false;
+    tc_fence_after();
+    const uint32_t ta = tmem + lane_base + static_cast<uint32_t>(p * kBN);
+    float v0[16], v1[16];
+    tmem_ld16(ta + 16 * g, v0);                  // half 0, rows 16 g ..
+    tmem_ld16(ta + kTailRows + 16 * g, v1);      // half 1
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tempty[p]);
+    const float4* f0 = reinterpret_cast<const float4*>(tc.f + kb * 2 * kTailRows + 16 * g);
+    const float4* f1 = reinterpret_cast<const float4*>(tc.f + kb * 2 * kTailRows + kTailRows + 16 * g);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 a = f0[j], b = f1[j];
+      acc0[4 * j + 0] = __fmaf_rn(v0[4 * j + 0], a.x, acc0[4 * j + 0]);
+      acc0[4 * j + 1] = __fmaf_rn(v0[4 * j + 1], a.y, acc0[4 * j + 1]);
+      acc0[4 * j + 2] = __fmaf_rn(v0[4 * j + 2], a.z, acc0[4 * j + 2]);
+      acc0[4 * j + 3] = __fmaf_rn(v0[4 * j + 3], a.w, acc0[4 * j + 3]);
+      acc1[4 * j + 0] = __fmaf_rn(v1[4 * j + 0], b.x, acc1[4 * j + 0]);
+      acc1[4 * j + 1] = __fmaf_rn(v1[4 * j + 1], b.y, acc1[4 * j + 1]);
+      acc1[4 * j + 2] = __fmaf_rn(v1[4 * j + 2], b.z, acc1[4 * j + 2]);
+      acc1[4 * j + 3] = __fmaf_rn(v1[4 * j + 3], b.w, acc1[4 * j + 3]);
+    }
+  }
+  mbar_arrive(tc.used);
+  ++ttile;
+  const int m0 = 16 * g;
+  if (EP == MOE_EP_F32) {
+    // row m of the tail: columns n_idx*256 + c (half 0) and + 128 + c (half 1);
+    // each store instruction writes 128 contiguous bytes of one row per warp
+    float* D = static_cast<float*>(args.D);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (m0 + i >= t.rows) break;
+      int64_t row = static_cast<int64_t>(t.row0) + m0 + i;
+      if (args.d_rows != nullptr) {
+        const int dr = __ldg(args.d_rows + row);
+        if (static_cast<uint32_t>(dr) >= static_cast<uint32_t>(args.a_rows)) {
+          set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
+          continue;
+        }
+        row = dr;
+      }
+      float* out = D + row * N + t.n_idx * kBN + c;
+      out[0] = acc0[i];
+      out[128] = acc1[i];
+    }
+  } else {
+    // h = SiLU(gate) * up; the row's 1x128 amax runs over the 128 channels c
+    // held by the warpgroup's 4 warps: a butterfly over the lanes, then the
+    // 4 warp maxima through shared memory
+    float hv[16], am[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      hv[i] = silu_mul(acc0[i], acc1[i]);
+      float a = fabsf(hv[i]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      am[i] = a;
+    }
+    if (lane < 16) {
+      float mine = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i == lane) mine = am[i];
+      tc.amax[(g * 4 + q) * 16 + lane] = mine;
+    }
+    mbar_arrive(&tc.ax[g]);
+    if (!__all_sync(0xffffffffu, mbar_wait(&tc.ax[g], ph, abort_v, args.dev_err))) return false;
+    const int I = N / 2;
+    uint8_t* H = static_cast<uint8_t*>(args.D);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float a = fmaxf(fmaxf(tc.amax[(g * 4 + 0) * 16 + i], tc.amax[(g * 4 + 1) * 16 + i]),
+                            fmaxf(tc.amax[(g * 4 + 2) * 16 + i], tc.amax[(g * 4 + 3) * 16 + i]));
+      const float sq = quant_scale(a);
+      const float rq = __frcp_rn(sq);
+      if (m0 + i < t.rows) {
+        const int64_t row = static_cast<int64_t>(t.row0) + m0 + i;
+        H[row * I + t.n_idx * 128 + c] =
+            static_cast<uint8_t>(e4m3x2(div_by_scale(hv[i], sq, rq), 0.f) & 0xFFu);
+        if (q == 0 && lane == 0) args.d_scale[row * (I / 128) + t.n_idx] = sq;
+      }
+    }
+  }
+  return true;
+}
+
 // Shared-memory layout after the 1024-aligned ring.
 struct Ctl {
   uint64_t* full;
@@ -382,6 +540,19 @@ __device__ __forceinline__ void tma_producer(const CUtensorMap& tmA, const CUten
 }
 
 // =========================================================== 1-SM mainloop
+// Work items reach the three roles through a 4-slot queue in shared memory:
+// the producer thread takes the next item -- blockIdx.x + i * gridDim.x
+// (static), or from the caller's counter with an atomic add (dynamic, so a
+// CTA that drew cheap tail tiles takes more work and the grid stays on
+// neighbouring items, whose m-tiles share weight tiles in L2) -- publishes it
+// and issues its loads; the MMA thread and the epilogue warps read it and
+// free the slot when done.  An item >= total ends every role.
+struct WorkQueue {
+  uint64_t* full;   // [kWQ]
+  uint64_t* empty;  // [kWQ], 1 (MMA) + 8 (epilogue warps) arrivals
+  int* item;        // [kWQ]
+};
+
 template <int EP, int SK>
 __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -390,11 +561,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
   constexpr int kA = kBM * SK, kB = kBN * SK;    // stage bytes of A and B
   constexpr int kStage = kA + kB;
   constexpr int kStages = kRingBytes / kStage;
+  constexpr bool kTail = (SK == 128);            // the swapped tail path needs whole K blocks
   static_assert((2 * kStages + 8) * 8 + 8 <= 512, "barrier area");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const Ctl c = carve<kStages>(base);
+  // queue, tail barriers and amax after the amax exchange area, 16-aligned
+  uint8_t* qbase = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(c.amax_x + 2 * 2 * 128) + 15) & ~static_cast<uintptr_t>(15));
+  WorkQueue wq;
+  wq.full = reinterpret_cast<uint64_t*>(qbase);
+  wq.empty = wq.full + kWQ;
+  TailCtl tc;
+  tc.staged = wq.empty + kWQ;
+  tc.used = tc.staged + 1;
+  tc.ax = tc.used + 1;
+  wq.item = reinterpret_cast<int*>(tc.ax + 2);
+  tc.amax = reinterpret_cast<float*>(wq.item + kWQ);
+  tc.f = reinterpret_cast<float*>(qbase + kTailFactorOffset);  // 16-aligned, after the amax block
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = args.N, KB = args.K / kBK, nN = N / kBN;
 
@@ -407,6 +592,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
       mbar_init(&c.tfull[p], 1);
       mbar_init(&c.tempty[p], kEpiThreads / 32);
     }
+    for (int i = 0; i < kWQ; ++i) {
+      mbar_init(&wq.full[i], 1);
+      mbar_init(&wq.empty[i], 1 + kEpiThreads / 32);
+    }
+    mbar_init(tc.staged, kEpiThreads);
+    mbar_init(tc.used, kEpiThreads);
+    mbar_init(&tc.ax[0], kEpiThreads / 2);
+    mbar_init(&tc.ax[1], kEpiThreads / 2);
     mbar_init(c.done, 1);
     mbar_init(&c.xbar[0], kEpiThreads);
     mbar_init(&c.xbar[1], kEpiThreads);
@@ -430,16 +623,56 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
     if (warp == 0 && lane == 0) {
-      tma_producer<kStages, SK>(tmA, tmB, args, c, base, total, nN, KB, abort_v);
+      // ---------------------------------------------- TMA producer + queue
+      int it = 0;
+      bool live = true;
+      for (int i = 0; live; ++i) {
+        const int qs = i % kWQ;
+        if (!mbar_wait(&wq.empty[qs], ((i / kWQ) & 1) ^ 1, abort_v, args.dev_err)) break;
+        const int w = args.sched ? atomicAdd(args.sched, 1) : blockIdx.x + i * gridDim.x;
+        wq.item[qs] = w;
+        mbar_arrive(&wq.full[qs]);
+        if (w >= total) break;
+        const Work t = decode_work<128>(w, nN, c.rstart, args);
+        if (!t.ok) {
+          set_dev_err(args.dev_err, MOE_DEVERR_BAD_TABLE);
+          continue;
+        }
+        const int brow = t.e * N + t.n_idx * kBN;
+        for (int kk = 0; kk < KB * kSub; ++kk, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&c.empty[s], ((it / kStages) & 1) ^ 1, abort_v, args.dev_err)) {
+            live = false;
+            break;
+          }
+          uint8_t* sA = base + s * kStage;
+          mbar_arrive_expect_tx(&c.full[s], kStage);
+          tma_load_2d(sA, &tmA, &c.full[s], kk * SK, t.row0);
+          tma_load_2d(sA + kA, &tmB, &c.full[s], kk * SK, brow);
+        }
+      }
+      // every issued copy lands before the CTA can exit
+      const int first = it > kStages ? it - kStages : 0;
+      for (int i = first; i < it; ++i)
+        mbar_wait(&c.full[i % kStages], (i / kStages) & 1, nullptr, args.dev_err);
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------- MMA issuer
       const uint32_t idesc = instr_desc(kFmtE4M3, kFmtE4M3, kBM, kBN);
+      // swapped tail: M = the 128 weight rows of one half, N = kTailRows tail rows
+      const uint32_t idesc_t = instr_desc(kFmtE4M3, kFmtE4M3, kBM, kTailRows);
       int it = 0, tit = 0;
       bool live = true;
-      for (int w = blockIdx.x; w < total && live; w += gridDim.x) {
+      for (int i = 0; live; ++i) {
+        const int qs = i % kWQ;
+        if (!mbar_wait(&wq.full[qs], (i / kWQ) & 1, abort_v, args.dev_err)) break;
+        const int w = wq.item[qs];
+        if (w >= total) {
+          mbar_arrive(&wq.empty[qs]);
+          break;
+        }
         const Work t = decode_work<128>(w, nN, c.rstart, args);
-        if (!t.ok) continue;
-        for (int kb = 0; kb < KB && live; ++kb, ++tit) {
+        const bool swp = kTail && t.swp;
+        for (int kb = 0; t.ok && kb < KB && live; ++kb, ++tit) {
           const int p = tit & 1;
           if (!mbar_wait(&c.tempty[p], ((tit >> 1) & 1) ^ 1, abort_v, args.dev_err)) {
             live = false;
@@ -456,13 +689,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
             const uint32_t sA = smem_u32(base + s * kStage);
             const uint64_t ad = kmajor_desc<SK>(sA);
             const uint64_t bd = kmajor_desc<SK>(sA + kA);
+            if (swp) {
+              // D_half[c][m] += W_half[c] . X[m]: the weight half is the A
+              // operand (128 rows, 16 KB apart), the tail rows the B operand
+              const uint64_t wd0 = smem_desc_sw128(sA + kA);
+              const uint64_t wd1 = smem_desc_sw128(sA + kA + kBM * SK);
 #pragma unroll
-            for (int k = 0; k < SK / 32; ++k)
-              mma_f8f6f4(dt, ad + 2 * k, bd + 2 * k, idesc, (h > 0 || k > 0) ? 1u : 0u);
+              for (int k = 0; k < SK / 32; ++k) {
+                mma_f8f6f4(dt, wd0 + 2 * k, ad + 2 * k, idesc_t, k > 0 ? 1u : 0u);
+                mma_f8f6f4(dt + kTailRows, wd1 + 2 * k, ad + 2 * k, idesc_t, k > 0 ? 1u : 0u);
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < SK / 32; ++k)
+                mma_f8f6f4(dt, ad + 2 * k, bd + 2 * k, idesc, (h > 0 || k > 0) ? 1u : 0u);
+            }
             mma_commit(&c.empty[s]);
           }
           if (live) mma_commit(&c.tfull[p]);
         }
+        mbar_arrive(&wq.empty[qs]);
       }
       mma_commit(c.done);
       mbar_wait(c.done, 0, nullptr, args.dev_err);
@@ -470,13 +716,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
     __syncwarp();
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
-    int tit = 0, xtile = 0;
-    for (int w = blockIdx.x; w < total; w += gridDim.x) {
-      const Work t = decode_work<128>(w, nN, c.rstart, args);
-      if (!t.ok) continue;
-      if (!epilogue_tile<EP>(args, t, tmem, warp, lane, KB, N, tit, xtile, c.tfull,
-                                    c.tempty, c.xbar, c.amax_x, abort_v))
+    int tit = 0, xtile = 0, ttile = 0;
+    for (int i = 0;; ++i) {
+      const int qs = i % kWQ;
+      if (!__all_sync(0xffffffffu, mbar_wait(&wq.full[qs], (i / kWQ) & 1, abort_v, args.dev_err)))
         break;
+      const int w = wq.item[qs];
+      bool ok = true;
+      if (w < total) {
+        const Work t = decode_work<128>(w, nN, c.rstart, args);
+        if (t.ok) {
+          if (kTail && t.swp)
+            ok = epilogue_tail<EP>(args, t, tmem, warp, lane, KB, N, tit, ttile, c.tfull,
+                                   c.tempty, tc, abort_v);
+          else
+            ok = epilogue_tile<EP>(args, t, tmem, warp, lane, KB, N, tit, xtile, c.tfull,
+                                   c.tempty, c.xbar, c.amax_x, abort_v);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wq.empty[qs]);
+      if (w >= total || !ok) break;
     }
   }
   tc_fence_before();
@@ -945,7 +1205,7 @@ moe_status gemm_launch(bool pow2, const uint8_t* A, const float* sa, int64_t a_r
                        const int32_t* tile_group, const int32_t* tile_start,
                        const int32_t* n_tiles, int max_tiles, int groups, int N, int K,
                        moe_epilogue ep, void* D, float* d_scale, const int32_t* d_rows,
-                       int32_t* dev_err, moe_stream_t stream) {
+                       int32_t* sched, int32_t* dev_err, moe_stream_t stream) {
   using namespace moe;
   if (a_rows < 0 || groups <= 0 || N <= 0 || K <= 0 || max_tiles < 0) return MOE_ERR_INVALID_ARG;
   if (K % kBK != 0 || N % kBN != 0) return MOE_ERR_SHAPE;
@@ -984,13 +1244,14 @@ moe_status gemm_launch(bool pow2, const uint8_t* A, const float* sa, int64_t a_r
   a.d_scale = d_scale;
   a.dev_err = dev_err;
   a.d_rows = d_rows;
+  a.sched = pow2 ? nullptr : sched;
   static int configured = 0;
   if (!configured) {
     const void* fs[4] = {kernel_ptr<MOE_EP_F32>(), kernel_ptr<MOE_EP_SWIGLU_QUANT>(),
                          reinterpret_cast<const void*>(gemm_pow2_kernel<MOE_EP_F32>),
                          reinterpret_cast<const void*>(gemm_pow2_kernel<MOE_EP_SWIGLU_QUANT>)};
     for (int i = 0; i < 4; ++i) {
-      const int bytes = static_cast<int>(i < 2 ? kSmemBytes : kSmemMxBytes);
+      const int bytes = static_cast<int>(i < 2 ? kSmemPromoteBytes : kSmemMxBytes);
       if (cudaFuncSetAttribute(fs[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
           cudaSuccess)
         return MOE_ERR_CUDA;
@@ -1006,8 +1267,12 @@ moe_status gemm_launch(bool pow2, const uint8_t* A, const float* sa, int64_t a_r
                           : reinterpret_cast<const void*>(gemm_pow2_kernel<MOE_EP_SWIGLU_QUANT>);
   else
     fn = ep == MOE_EP_F32 ? kernel_ptr<MOE_EP_F32>() : kernel_ptr<MOE_EP_SWIGLU_QUANT>();
+  if (a.sched != nullptr &&
+      cudaMemsetAsync(a.sched, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   void* kargs[3] = {&tmA, &tmB, &a};
-  if (cudaLaunchKernel(fn, dim3(ctas), dim3(kThreads), kargs, pow2 ? kSmemMxBytes : kSmemBytes,
+  if (cudaLaunchKernel(fn, dim3(ctas), dim3(kThreads), kargs,
+                       pow2 ? kSmemMxBytes : kSmemPromoteBytes,
                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
@@ -1019,18 +1284,20 @@ extern "C" moe_status grouped_gemm_fp8_blockscaled(
     const uint8_t* A, const float* sa, int64_t a_rows, const uint8_t* B, const float* sb,
     const int32_t* offsets, const int32_t* tile_group, const int32_t* tile_start,
     const int32_t* n_tiles, int max_tiles, int groups, int N, int K, moe_epilogue ep, void* D,
-    float* d_scale, const int32_t* d_rows, int32_t* dev_err, moe_stream_t stream) {
+    float* d_scale, const int32_t* d_rows, int32_t* sched, int32_t* dev_err,
+    moe_stream_t stream) {
   return gemm_launch(false, A, sa, a_rows, B, sb, offsets, tile_group, tile_start, n_tiles,
-                     max_tiles, groups, N, K, ep, D, d_scale, d_rows, dev_err, stream);
+                     max_tiles, groups, N, K, ep, D, d_scale, d_rows, sched, dev_err, stream);
 }
 
 extern "C" moe_status grouped_gemm_fp8_pow2(
     const uint8_t* A, const float* sa, int64_t a_rows, const uint8_t* B, const float* sb,
     const int32_t* offsets, const int32_t* tile_group, const int32_t* tile_start,
     const int32_t* n_tiles, int max_tiles, int groups, int N, int K, moe_epilogue ep, void* D,
-    float* d_scale, const int32_t* d_rows, int32_t* dev_err, moe_stream_t stream) {
+    float* d_scale, const int32_t* d_rows, int32_t* sched, int32_t* dev_err,
+    moe_stream_t stream) {
   return gemm_launch(true, A, sa, a_rows, B, sb, offsets, tile_group, tile_start, n_tiles,
-                     max_tiles, groups, N, K, ep, D, d_scale, d_rows, dev_err, stream);
+                     max_tiles, groups, N, K, ep, D, d_scale, d_rows, sched, dev_err, stream);
 }
 
 extern "C" moe_status grouped_gemm_fp8_wgrad(const uint8_t* At, const uint8_t* sfa_atoms,

@@ -200,6 +200,7 @@ class MoELayerEP:
         self.route_ws = torch.empty(max(_abi.moe_route_workspace_size(T, d, E), 16), dtype=u8,
                                     device=dev)
         self.dev_err = torch.zeros(1, dtype=i32, device=dev)
+        self.sched = torch.zeros(1, dtype=i32, device=dev)   # the GEMMs' work counter
         # receive side: [own T tokens | received rows], then regrouped copies
         rows = T + Rcap
         self.RX = torch.empty(rows, d, dtype=u8, device=dev)
@@ -287,11 +288,12 @@ class MoELayerEP:
         a.grouped_gemm_fp8_blockscaled(self.X2[:n], self.X2s[:n], self.w1q, self.w1s,
                                        p2["offsets"], p2["tile_group"], p2["tile_start"],
                                        p2["n_tiles"], mt, a.EP_SWIGLU_QUANT, self.H2[:n],
-                                       self.H2s[:n], dev_err=self.dev_err)
+                                       self.H2s[:n], dev_err=self.dev_err, sched=self.sched)
         a.grouped_gemm_fp8_blockscaled(self.H2[:n], self.H2s[:n], self.w2q, self.w2s,
                                        p2["offsets"], p2["tile_group"], p2["tile_start"],
                                        p2["n_tiles"], mt, a.EP_F32, self.Yr[:n],
-                                       dev_err=self.dev_err, d_rows=p2["src_row"][:n])
+                                       dev_err=self.dev_err, d_rows=p2["src_row"][:n],
+                                       sched=self.sched)
 
     def return_rows(self):
         """The received rows' outputs to send back (receive order)."""

@@ -138,6 +138,8 @@ class MoELayer:
         self.Y = torch.empty(P + T, d, dtype=f32, device=dev)
         self.out = torch.empty(T, d, dtype=f32, device=dev)
         self.dev_err = torch.zeros(1, dtype=i32, device=dev)
+        # the grouped GEMMs' work counter (dynamic tile scheduling)
+        self.sched = torch.zeros(1, dtype=i32, device=dev)
         self.u_dev = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
         # second input/output pair and copy streams for forward_host_stream
         self._u_dev2 = None
@@ -170,14 +172,14 @@ class MoELayer:
         _abi.grouped_gemm_fp8_blockscaled(self.Xq, self.Xs, self.w1q, self.w1s, p["offsets"],
                                           p["tile_group"], p["tile_start"], p["n_tiles"],
                                           self.max_tiles, _abi.EP_SWIGLU_QUANT, self.H, self.Hs,
-                                          dev_err=self.dev_err, pow2=self.pow2)
+                                          dev_err=self.dev_err, pow2=self.pow2, sched=self.sched)
 
     def step_gemm2(self):
         p = self.perm
         _abi.grouped_gemm_fp8_blockscaled(self.H, self.Hs, self.w2q, self.w2s, p["offsets"],
                                           p["tile_group"], p["tile_start"], p["n_tiles"],
                                           self.max_tiles, _abi.EP_F32, self.Y,
-                                          dev_err=self.dev_err, pow2=self.pow2)
+                                          dev_err=self.dev_err, pow2=self.pow2, sched=self.sched)
 
     def step_combine(self, u, out=None):
         P = self.pairs

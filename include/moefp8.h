@@ -71,7 +71,8 @@ typedef void* moe_stream_t; /* cudaStream_t */
 /* Human-readable text for a status (static storage, never NULL). */
 const char* moe_status_string(moe_status s);
 
-/* ABI version of this header (bumped on any incompatible change). */
+/* ABI version of this header (bumped on any incompatible change); this
+ * header is version 3. */
 int moe_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -290,6 +291,15 @@ moe_status moe_segment_ids(const int32_t* counts, int n_segments, int E, int64_t
  *      channels); D is E4M3 h [a_rows][N/2] with h = SiLU(gate) * up
  *      ([ANN] SwiGLU operator notes, Swish with beta = 1) quantised 1x128 as
  *      in fp8_quant_1x128, d_scale fp32 [a_rows][N/256]; d_rows must be NULL.
+ *   sched: one int32 of device scratch, or NULL.  With it the kernel hands
+ *      out its (group, n-tile, m-tile) work items dynamically (an atomic
+ *      counter, zeroed by the call on `stream`; calls that overlap on the GPU
+ *      must not share it); NULL keeps a static round-robin order.  The results
+ *      are the same either way.  The pow2 variant ignores it.
+ *   An m-tile of at most 32 rows (an expert's tail past its whole 128-row
+ *   tiles, or an expert with few rows) is computed transposed -- the weight
+ *   tile's halves as the tensor core's M side, the rows as N = 32 -- with the
+ *   same per-128-K scaled fp32 accumulation (K <= 8192).
  * Limits: K % 128 == 0, N % 256 == 0.
  */
 moe_status grouped_gemm_fp8_blockscaled(const uint8_t* A, const float* sa, int64_t a_rows,
@@ -298,8 +308,8 @@ moe_status grouped_gemm_fp8_blockscaled(const uint8_t* A, const float* sa, int64
                                         const int32_t* tile_start, const int32_t* n_tiles,
                                         int max_tiles, int groups, int N, int K,
                                         moe_epilogue ep, void* D, float* d_scale,
-                                        const int32_t* d_rows, int32_t* dev_err,
-                                        moe_stream_t stream);
+                                        const int32_t* d_rows, int32_t* sched,
+                                        int32_t* dev_err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * grouped_gemm_fp8_pow2 -- grouped_gemm_fp8_blockscaled for operands whose
@@ -323,7 +333,8 @@ moe_status grouped_gemm_fp8_pow2(const uint8_t* A, const float* sa, int64_t a_ro
                                  const int32_t* tile_group, const int32_t* tile_start,
                                  const int32_t* n_tiles, int max_tiles, int groups, int N, int K,
                                  moe_epilogue ep, void* D, float* d_scale,
-                                 const int32_t* d_rows, int32_t* dev_err, moe_stream_t stream);
+                                 const int32_t* d_rows, int32_t* sched, int32_t* dev_err,
+                                 moe_stream_t stream);
 
 /* ===========================================================================
  * Backward of the expert FFNs.  [ANN] "Mixed Precision Framework": Fprop,
@@ -423,7 +434,12 @@ moe_status grouped_gemm_fp8_wgrad(const uint8_t* At, const uint8_t* sfa_atoms, c
 /* ---------------------------------------------------------------------------
  * swiglu_quant -- standalone SwiGLU + 1x128 quantisation of fp32 GEMM output
  * in the block-interleaved layout above; bit-identical to the fused epilogue
- * on identical input.
+ * on identical input.  [ANN] SwiGLU operator notes: h = Swish(gate) * up with
+ * Swish(x) = x * Sigmoid(x); "Fine-Grained Quantization": the input of the
+ * down projection is FP8 like every GEMM input, quantised per token per 128
+ * channels ("Online Quantization": scale from the tile's own max |h|).
+ * swiglu_quant_pow2 rounds each scale up to a power of two ([ANN]
+ * "Low-Precision Storage and Communication").
  *   gu fp32 [rows][2I];  h E4M3 [rows][I];  h_scale fp32 [rows][I/128]
  */
 moe_status swiglu_quant(const float* gu, int rows, int I, uint8_t* h, float* h_scale,

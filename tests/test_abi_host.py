@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(_abi.exported_symbols())
-    assert L.moe_abi_version() == 2
+    assert L.moe_abi_version() == 3
 
 
 def test_status_strings():
@@ -62,13 +62,13 @@ def test_max_m_tiles_bound():
                                            None, None, None, 0, None), 1),   # NULL partials
     (lambda L: L.grouped_gemm_fp8_blockscaled(None, None, 10, None, None, None, None, None,
                                               None, 4, 1, 384, 128, 0, None, None, None,
-                                              None, None), 2),                # N % 256
+                                              None, None, None), 2),          # N % 256
     (lambda L: L.grouped_gemm_fp8_blockscaled(None, None, 10, None, None, None, None, None,
                                               None, 4, 1, 256, 128, 7, None, None, None,
-                                              None, None), 1),                # bad epilogue
+                                              None, None, None), 1),          # bad epilogue
     (lambda L: L.grouped_gemm_fp8_blockscaled(None, None, 10, None, None, None, None, None,
                                               None, 4, 1, 256, 128, 1, None, None, 16, None,
-                                              None), 1),                      # row map with SwiGLU
+                                              None, None), 1),                # row map with SwiGLU
     (lambda L: L.swiglu_quant(None, 4, 100, None, None, None), 2),
     (lambda L: L.moe_seq_balance_loss(None, 100, 16, 4, 30, ctypes.c_float(1e-4), None, None,
                                       None, None, 0, None), 2),              # T % seq_len
@@ -84,7 +84,7 @@ def test_max_m_tiles_bound():
     (lambda L: L.fp8_quant_1x128_pow2(None, 200, 4, 200, None, None, None), 2),
     (lambda L: L.fp8_quant_128x128_pow2(None, 64, 4, 128, None, None, None), 2),
     (lambda L: L.grouped_gemm_fp8_pow2(None, None, 10, None, None, None, None, None, None, 4, 1,
-                                       384, 128, 0, None, None, None, None, None), 2),  # N % 256
+                                       384, 128, 0, None, None, None, None, None, None), 2),
     (lambda L: L.swiglu_quant_pow2(None, 4, 100, None, None, None), 2),
     # backward
     (lambda L: L.fp8_quant_1x128_f32(None, 200, 4, 200, 0, None, None, None), 2),

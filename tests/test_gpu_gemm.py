@@ -122,3 +122,46 @@ def test_combine(cuda_dev):
     Yn = npraw(Y)
     ref = O.combine(Yn[:P], dst, gate, Yn[P:], np32(u))
     assert np.allclose(npraw(out), ref, rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("ep", ["f32", "swiglu"])
+def test_tail_tiles_and_dynamic_schedule(cuda_dev, ep):
+    """m-tiles of at most 32 rows (an expert's rows past a whole 128-row
+    tile, or an expert with few rows) take the transposed tail path; every
+    tail size from 1 to 33 rows and a few whole tiles are checked against the
+    oracle on the same FP8 operands.  The dynamic schedule (a work counter)
+    gives the same bytes as the static one."""
+    K, N = 1024, 512
+    counts = [1, 2, 7, 16, 17, 31, 32, 33, 0, 128 + 1, 128 + 31, 128 + 32, 128 + 33, 256 + 5, 64,
+              100, 127, 128]
+    G = len(counts)
+    rows = sum(counts)
+    aq, sa, bq, sb = _quantised_operands(cuda_dev, rows, K, G, N, seed=77)
+    offsets = [int(x) for x in np.cumsum([0] + counts)]
+    max_tiles = sum(-(-c // 128) for c in counts)
+    offs, tg, ts, nt = _tables(cuda_dev, offsets, max_tiles)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_dev)
+    sched = torch.zeros(1, dtype=torch.int32, device=cuda_dev)
+    mode = _abi.EP_F32 if ep == "f32" else _abi.EP_SWIGLU_QUANT
+    out_s = _abi.grouped_gemm_fp8_blockscaled(aq, sa, bq, sb, offs, tg, ts, nt, max_tiles, mode,
+                                              dev_err=err)
+    out_d = _abi.grouped_gemm_fp8_blockscaled(aq, sa, bq, sb, offs, tg, ts, nt, max_tiles, mode,
+                                              dev_err=err, sched=sched)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    gu = O.grouped_gemm(npraw(aq), npraw(sa), npraw(bq), npraw(sb), offsets)
+    if ep == "f32":
+        assert torch.equal(out_s, out_d)
+        assert_within_rms(npraw(out_s), gu, what="tail/whole tiles")
+        # every row is within the bound on its own: the tails are not hidden
+        # behind the whole tiles' magnitude
+        g = npraw(out_s)
+        for r in range(rows):
+            assert_within_rms(g[r], gu[r], what=f"row {r}")
+    else:
+        (h_s, hs_s), (h_d, hs_d) = out_s, out_d
+        assert torch.equal(h_s, h_d) and torch.equal(hs_s, hs_d)
+        hq, hs = O.swiglu_quant(gu, N // 2)
+        d = e4m3_step_distance(npraw(h_s), hq)
+        assert d.max() <= 1 and (d > 0).mean() < 2e-2
+        assert np.allclose(npraw(hs_s), hs, rtol=1e-4, atol=0)
