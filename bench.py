@@ -460,44 +460,50 @@ def run_gpu(args):
     out_host = out_hosts[0]
 
     # the sequence-wise balance loss (eqs. 17-20) of this batch, one sequence
-    # of T tokens: the router's selection pass writes its per-8-token partial
-    # sums (aux_part), one short reduction finishes it.  Its cost is the route
-    # with the partials minus the route without them, plus the reduction; the
-    # three-pass form from kept logits is timed beside it.
+    # of T tokens: the router's selection pass computes it (integer sums per
+    # sequence, the last block finishes the loss).  Its cost is the route
+    # with the loss minus the route without it; the three-pass form from
+    # kept logits is timed beside it.
     logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
-    part = torch.empty((cfg.T + 7) // 8, 2, cfg.E, dtype=torch.float32, device=dev)
+    bstate = _abi.BalanceLossState(cfg.T, cfg.E, cfg.T, 1e-4, with_fp=True, device=dev)
     rws = torch.empty(max(_abi.moe_route_workspace_size(cfg.T, cfg.d, cfg.E), 16),
                       dtype=torch.uint8, device=dev)
     bl_ws = torch.empty(max(_abi.moe_seq_balance_loss_ws(cfg.T, cfg.E, cfg.T), 16),
                         dtype=torch.uint8, device=dev)
 
     def timed(fn, n):
+        # n calls recorded into one CUDA graph, so the device time is measured
+        # and not the host's per-call overhead (these kernels run for a few us)
         for _ in range(3):
             fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(n):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
         a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a_.record(st)
-        for _ in range(n):
-            fn()
+        g.replay()
         b_.record(st)
         b_.synchronize()
+        del g
         return a_.elapsed_time(b_) * 1e3 / n
 
     reps = max(args.steps, 10)
     t_plain = timed(lambda: _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K,
                                            ws=rws), reps)
     t_aux = timed(lambda: _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K,
-                                         ws=rws, aux_part=part), reps)
-    pws = torch.empty(max(_abi.moe_seq_balance_loss_part_ws(cfg.T, cfg.E, cfg.T), 16),
-                      dtype=torch.uint8, device=dev)
-    t_red = timed(lambda: _abi.moe_seq_balance_loss_part(part, cfg.T, cfg.K, cfg.T, ws=pws), reps)
+                                         ws=rws, aux=bstate), reps)
     _abi.moe_route(u, layer.centroids, layer.bias, cfg.G, cfg.M, cfg.K, logits_out=logits, ws=rws)
     t_3p = timed(lambda: _abi.moe_seq_balance_loss(logits, cfg.K, cfg.T, ws=bl_ws), reps)
     barrier()
-    balance_loss = {"extra_us": round(t_aux - t_plain + t_red, 2),
-                    "route_us": round(t_plain, 2), "route_with_partials_us": round(t_aux, 2),
-                    "reduction_us": round(t_red, 2), "three_pass_from_logits_us": round(t_3p, 2),
-                    "seq_len": cfg.T}
-    del logits, part, rws, bl_ws, pws
+    balance_loss = {"extra_us": round(t_aux - t_plain, 2),
+                    "route_us": round(t_plain, 2), "route_with_loss_us": round(t_aux, 2),
+                    "three_pass_from_logits_us": round(t_3p, 2), "seq_len": cfg.T,
+                    "how": "device time per call, 10+ calls replayed from one CUDA graph"}
+    del logits, bstate, rws, bl_ws
 
     # roofline of the dominant kernel (grouped GEMM 1 with the SwiGLU epilogue)
     counts = layer.perm["counts"].cpu()

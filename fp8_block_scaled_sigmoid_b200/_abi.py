@@ -63,12 +63,36 @@ _SIGS = {
     "moe_seq_balance_loss_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
     "moe_seq_balance_loss": (_i, [_p, _i, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
     "moe_fp8_mma_peak": (_i, [_i, _i, _i, _p, _p, _p]),
-    "moe_seq_balance_loss_part_workspace_size": (_i, [_i, _i, _i, _c.POINTER(_sz)]),
-    "moe_seq_balance_loss_part": (_i, [_p, _i, _i, _i, _i, _f, _p, _p, _p, _p, _sz, _p]),
 }
 
 EP_F32 = 0
 EP_SWIGLU_QUANT = 1
+
+
+class _BalanceLoss(ctypes.Structure):
+    """moe_balance_loss (include/moefp8.h)."""
+    _fields_ = [("seq_len", _i), ("alpha", _f), ("acc", _p), ("cnt", _p), ("done", _p),
+                ("loss", _p), ("f", _p), ("P", _p)]
+
+
+class BalanceLossState:
+    """Device buffers of the balance loss that moe_route computes in its
+    selection pass, for T tokens in sequences of seq_len: the zeroed sums and
+    counters (each call leaves them zero) and the outputs loss [T/seq_len],
+    f and P [T/seq_len][E] (with_fp)."""
+
+    def __init__(self, T, E, seq_len, alpha=1e-4, with_fp=False, device=None):
+        n_seq = T // seq_len if seq_len > 0 else 0
+        n = max(n_seq, 1)
+        self.T, self.E, self.seq_len, self.alpha, self.n_seq = T, E, seq_len, alpha, n_seq
+        self.acc = torch.zeros(n, E, dtype=torch.int64, device=device)
+        self.cnt = torch.zeros(n, E, dtype=torch.int32, device=device)
+        self.done = torch.zeros(n, dtype=torch.int32, device=device)
+        self.loss = torch.zeros(n, dtype=torch.float32, device=device)
+        self.f = torch.zeros(n, E, dtype=torch.float32, device=device) if with_fp else None
+        self.P = torch.zeros(n, E, dtype=torch.float32, device=device) if with_fp else None
+        self.c = _BalanceLoss(int(seq_len), float(alpha), _ptr(self.acc), _ptr(self.cnt),
+                              _ptr(self.done), _ptr(self.loss), _ptr(self.f), _ptr(self.P))
 DEVERR = {0: "none", 1: "bounded wait timed out", 2: "inconsistent segment table",
           3: "expert index out of range", 4: "a scale is not a power of two"}
 
@@ -86,8 +110,7 @@ LAUNCHES_PER_CALL = {"fp8_quant_1x128": 1, "fp8_quant_128x128": 1, "swiglu_quant
                      "moe_permute_index": 2, "fp8_quant_1x128_scatter": 1,
                      "moe_tile_table": 1, "moe_segment_ids": 1,
                      "grouped_gemm_fp8_blockscaled": 1, "moe_combine": 1, "moe_bias_update": 1,
-                     "moe_seq_balance_loss": 3, "moe_fp8_mma_peak": 1,
-                     "moe_seq_balance_loss_part": 2}
+                     "moe_seq_balance_loss": 3, "moe_fp8_mma_peak": 1}
 launch_count = 0
 
 
@@ -198,7 +221,8 @@ def moe_route_workspace_size(T, d, E) -> int:
 
 
 def moe_route(u, centroids, bias, G, M, K, topk_idx=None, topk_gate=None, logits_out=None,
-              ws=None, dev_err=None, stream=None, aux_part=None):
+              ws=None, dev_err=None, stream=None, aux=None):
+    """aux: a BalanceLossState for the same T, or None."""
     T, d = u.shape
     E = centroids.shape[0]
     dev = _dev(u)
@@ -209,7 +233,8 @@ def moe_route(u, centroids, bias, G, M, K, topk_idx=None, topk_gate=None, logits
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     _count("moe_route")
     _check(lib().moe_route(_ptr(u), u.stride(0), _ptr(centroids), _ptr(bias), T, d, E, G, M, K,
-                           _ptr(topk_idx), _ptr(topk_gate), _ptr(logits_out), _ptr(aux_part),
+                           _ptr(topk_idx), _ptr(topk_gate), _ptr(logits_out),
+                           ctypes.addressof(aux.c) if aux is not None else None,
                            _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_err),
                            _stream(stream)),
            "moe_route")
@@ -452,35 +477,6 @@ def moe_seq_balance_loss(logits, K, seq_len, alpha=1e-4, with_fp=False, ws=None,
     return loss
 
 
-def moe_seq_balance_loss_part_ws(T, E, seq_len) -> int:
-    n = _sz(0)
-    _check(lib().moe_seq_balance_loss_part_workspace_size(T, E, seq_len, ctypes.byref(n)),
-           "moe_seq_balance_loss_part_workspace_size")
-    return n.value
-
-
-def moe_seq_balance_loss_part(part, T, K, seq_len, alpha=1e-4, with_fp=False, ws=None,
-                              stream=None):
-    """The balance loss from moe_route's aux_part fp32 [ceil(T/8)][2][E] (K =
-    the routing K).  Returns loss fp32 [T/seq_len], or (loss, f, P)."""
-    E = part.shape[-1]
-    dev = _dev(part)
-    if ws is None:
-        ws = torch.empty(max(moe_seq_balance_loss_part_ws(T, E, seq_len), 16), dtype=torch.uint8,
-                         device=dev)
-    n_seq = T // seq_len if seq_len > 0 else 0
-    loss = torch.empty(max(n_seq, 1), dtype=torch.float32, device=dev)
-    f = torch.empty(max(n_seq, 1), E, dtype=torch.float32, device=dev) if with_fp else None
-    P = torch.empty(max(n_seq, 1), E, dtype=torch.float32, device=dev) if with_fp else None
-    _count("moe_seq_balance_loss_part")
-    _check(lib().moe_seq_balance_loss_part(_ptr(part), T, E, K, seq_len, float(alpha), _ptr(loss),
-                                           _ptr(f), _ptr(P), _ptr(ws),
-                                           ws.numel() * ws.element_size(), _stream(stream)),
-           "moe_seq_balance_loss_part")
-    loss = loss[:n_seq]
-    if with_fp:
-        return loss, f[:n_seq], P[:n_seq]
-    return loss
 
 
 def moe_bias_update(counts, T, K, gamma, bias, stream=None):

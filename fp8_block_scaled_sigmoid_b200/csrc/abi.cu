@@ -18,7 +18,7 @@ extern "C" const char* moe_status_string(moe_status s) {
   return "unknown status";
 }
 
-extern "C" int moe_abi_version(void) { return 3; }
+extern "C" int moe_abi_version(void) { return 4; }
 
 namespace {
 

@@ -6,10 +6,11 @@
 // the TopK taken over the raw affinities of all E routed experts (ties to
 // the lower index).
 //
-// The token pass spreads a row's experts over the lanes exactly as the
-// router's selection kernel does (same experts per lane, same orders), so the
-// per-token values the selection computes when the loss is fused into it
-// (moe_route's aux_part, finished by moe_seq_balance_loss_part) are the same.
+// This is the unfused form, from logits kept by moe_route (logits_out); the
+// fused form runs inside moe_route's selection pass (moe_balance_loss).  The
+// token pass spreads a row's experts over the lanes exactly as the selection
+// kernel does (same experts per lane, same orders), so the per-token values
+// are the same in both.
 //
 // Three deterministic passes, no atomics:
 //  1. token  -- one warp per token: s, its row sum (fixed butterfly), the
@@ -227,111 +228,5 @@ extern "C" moe_status moe_seq_balance_loss(const float* logits, int T, int E, in
 namespace moe {
 namespace {
 
-// The loss from the per-8-token partials moe_route wrote (aux_part), in two
-// deterministic levels.  Level 1: CTA (q, g) sums blocks g*G .. g*G+G-1 of
-// sequence q in block order, one thread per expert -> ws[q][g][2][E].
-// Level 2: one CTA per sequence adds its groups in order, then f, P and a
-// fixed-order tree over the experts give the loss.
-constexpr int kPartGroups = 16;
-
-__global__ void aux_part_group_kernel(const float* __restrict__ part, int E, int nb, int G,
-                                      float* __restrict__ ws) {
-  const int e = threadIdx.x;
-  if (e >= E) return;
-  const int q = blockIdx.y, g = blockIdx.x;
-  const int b0 = g * G, b1 = min(nb, b0 + G);
-  const float* base = part + static_cast<int64_t>(q) * nb * 2 * E + e;
-  float acc = 0.f, cnt = 0.f;
-  int b = b0;
-  for (; b + 8 <= b1; b += 8) {  // eight loads in flight, added in block order
-    float v[8], c[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] = __ldg(base + static_cast<int64_t>(b + i) * 2 * E);
-      c[i] = __ldg(base + static_cast<int64_t>(b + i) * 2 * E + E);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      acc = __fadd_rn(acc, v[i]);
-      cnt = __fadd_rn(cnt, c[i]);
-    }
-  }
-  for (; b < b1; ++b) {
-    acc = __fadd_rn(acc, __ldg(base + static_cast<int64_t>(b) * 2 * E));
-    cnt = __fadd_rn(cnt, __ldg(base + static_cast<int64_t>(b) * 2 * E + E));
-  }
-  float* dst = ws + (static_cast<int64_t>(q) * gridDim.x + g) * 2 * E;
-  dst[e] = acc;
-  dst[E + e] = cnt;
-}
-
-// blockDim = Ep (a power of two >= E, <= 1024)
-__global__ void aux_part_final_kernel(const float* __restrict__ ws, int E, int NG, int K,
-                                      int seq_len, float alpha, float* __restrict__ loss,
-                                      float* __restrict__ f_out, float* __restrict__ p_out) {
-  extern __shared__ float red[];
-  const int e = threadIdx.x;
-  const int q = blockIdx.x;
-  float term = 0.f;
-  if (e < E) {
-    const float* base = ws + static_cast<int64_t>(q) * NG * 2 * E + e;
-    float acc = 0.f, cnt = 0.f;
-    for (int g = 0; g < NG; ++g) {
-      acc = __fadd_rn(acc, __ldg(base + static_cast<int64_t>(g) * 2 * E));
-      cnt = __fadd_rn(cnt, __ldg(base + static_cast<int64_t>(g) * 2 * E + E));
-    }
-    // f_i = E/(K S) * count, P_i = sum / S
-    const float f = __fdiv_rn(static_cast<float>(E) * cnt,
-                              static_cast<float>(K) * static_cast<float>(seq_len));
-    const float pv = __fdiv_rn(acc, static_cast<float>(seq_len));
-    if (f_out) f_out[static_cast<int64_t>(q) * E + e] = f;
-    if (p_out) p_out[static_cast<int64_t>(q) * E + e] = pv;
-    term = __fmul_rn(f, pv);
-  }
-  red[e] = term;
-  __syncthreads();
-  for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
-    if (e < w) red[e] = __fadd_rn(red[e], red[e + w]);
-    __syncthreads();
-  }
-  if (e == 0) loss[q] = __fmul_rn(alpha, red[0]);
-}
-
 }  // namespace
 }  // namespace moe
-
-extern "C" moe_status moe_seq_balance_loss_part_workspace_size(int T, int E, int seq_len,
-                                                                size_t* bytes) {
-  using namespace moe;
-  if (!bytes || T < 0 || E <= 0 || seq_len <= 0) return MOE_ERR_INVALID_ARG;
-  *bytes = align256(static_cast<size_t>(T / seq_len) * kPartGroups * 2 * E * sizeof(float));
-  return MOE_OK;
-}
-
-extern "C" moe_status moe_seq_balance_loss_part(const float* aux_part, int T, int E, int K,
-                                                int seq_len, float alpha, float* loss,
-                                                float* f_out, float* p_out, void* ws,
-                                                size_t ws_bytes, moe_stream_t stream) {
-  using namespace moe;
-  if (T < 0 || E <= 0 || K <= 0 || seq_len <= 0) return MOE_ERR_INVALID_ARG;
-  if (K > E || K > 32 || T % seq_len != 0 || seq_len % 8 != 0) return MOE_ERR_SHAPE;
-  if (E > 1024) return MOE_ERR_UNSUPPORTED;
-  if (T == 0) return MOE_OK;
-  if (!aux_part || !loss) return MOE_ERR_INVALID_ARG;
-  size_t need = 0;
-  moe_seq_balance_loss_part_workspace_size(T, E, seq_len, &need);
-  if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int n_seq = T / seq_len, nb = seq_len / 8;
-  const int G = (nb + kPartGroups - 1) / kPartGroups;
-  const int NG = (nb + G - 1) / G;  // groups actually holding blocks
-  float* w = static_cast<float*>(ws);
-  aux_part_group_kernel<<<dim3(NG, n_seq), (E + 31) / 32 * 32, 0, st>>>(aux_part, E, nb, G, w);
-  MOE_CUDA_CHECK_LAUNCH();
-  int Ep = 32;
-  while (Ep < E) Ep <<= 1;
-  aux_part_final_kernel<<<n_seq, Ep, Ep * sizeof(float), st>>>(w, E, NG, K, seq_len, alpha, loss,
-                                                                f_out, p_out);
-  MOE_CUDA_CHECK_LAUNCH();
-  return MOE_OK;
-}

@@ -156,6 +156,21 @@ struct Cand {
   float s;  // raw score
 };
 
+// Order-preserving unsigned key of a float score (+0 for both zeros): a > b
+// as floats iff key(a) > key(b).
+__device__ __forceinline__ uint32_t score_key(float v) {
+  const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The lane holding the warp's largest key; among equal keys the lowest lane
+// (lanes own ascending experts, so the lowest expert).  One warp max
+// (redux.sync) and one ballot.
+__device__ __forceinline__ int warp_argmax_lane(uint32_t key) {
+  const uint32_t m = __reduce_max_sync(0xffffffffu, key);
+  return __ffs(__ballot_sync(0xffffffffu, key == m)) - 1;
+}
+
 __device__ __forceinline__ bool better(float v1, int i1, float v2, int i2) {
   return v1 > v2 || (v1 == v2 && i1 < i2);
 }
@@ -193,6 +208,9 @@ __device__ __forceinline__ void aux_token_row(const float (&s)[P], int E, int K,
     if (e0 + i < E) sum = __fadd_rn(sum, s[i]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
+  // raw top-K: each lane keeps its best remaining expert (bi); a round takes
+  // the warp's best (score descending, then lower expert) and only its owner
+  // looks for its next best
   uint32_t taken = 0;
   int bi = -1;
   float bv = 0.f;
@@ -203,19 +221,9 @@ __device__ __forceinline__ void aux_token_row(const float (&s)[P], int E, int K,
       bv = s[i];
     }
   for (int k = 0; k < K; ++k) {
-    uint32_t key = bi < 0 ? 0u : __float_as_uint(bv);  // s > 0 orders like its bits
-    int ex = bi < 0 ? INT_MAX : e0 + bi;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const uint32_t ok = __shfl_xor_sync(0xffffffffu, key, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, ex, off);
-      if (ok > key || (ok == key && oe < ex)) {
-        key = ok;
-        ex = oe;
-      }
-    }
-    if (ex / P == lane) {
-      taken |= 1u << (ex - e0);
+    const int owner = warp_argmax_lane(bi < 0 ? 0u : score_key(bv));  // s > 0
+    if (lane == owner) {
+      taken |= 1u << bi;
       bi = -1;
       bv = 0.f;
 #pragma unroll
@@ -364,44 +372,28 @@ __device__ __forceinline__ void select_token(
   for (int i = 0; i < P; ++i)
     if (e0 + i < E && !((allowed >> ((e0 + i) / gs)) & 1u)) beta[i] = -INFINITY;
 
-  // each lane keeps its best remaining candidate (local index bi); a round
-  // takes the warp's best (biased score descending, then lower expert) with
-  // one 5-step argmax on (order-preserving key, expert), and only the lane
-  // that owned it looks for its next best
+  // each lane keeps its best remaining candidate (local index bi, biased
+  // score bv, raw score bs); a round takes the warp's best (biased score
+  // descending, then lower expert): one warp max over the order-preserving
+  // keys and a ballot; only the lane that owned it looks for its next best
   uint32_t taken = 0;
   int bi = -1;
-  float bv = -INFINITY;
+  float bv = -INFINITY, bs = 0.f;
 #pragma unroll
   for (int i = 0; i < P; ++i)
     if (e0 + i < E && (bi < 0 || beta[i] > bv)) {
       bi = i;
       bv = beta[i];
+      bs = sc[i];
     }
   float ssum = 0.f, my_s = 0.f;
   int my_idx = 0;
   for (int k = 0; k < K; ++k) {
-    // order-preserving unsigned key of the score (+0 for both zeros)
-    const float v = bv == 0.f ? 0.f : bv;
-    const uint32_t u = __float_as_uint(v);
-    uint32_t key = bi < 0 ? 0u : ((u & 0x80000000u) ? ~u : (u | 0x80000000u));
-    int ex = bi < 0 ? INT_MAX : e0 + bi;
-    float s_mine = 0.f;
-#pragma unroll
-    for (int i = 0; i < P; ++i)
-      if (i == bi) s_mine = sc[i];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const uint32_t ok = __shfl_xor_sync(0xffffffffu, key, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, ex, off);
-      if (ok > key || (ok == key && oe < ex)) {
-        key = ok;
-        ex = oe;
-      }
-    }
-    const int owner = ex / P;
-    const float s_win = __shfl_sync(0xffffffffu, s_mine, owner);
+    const int owner = warp_argmax_lane(bi < 0 ? 0u : score_key(bv));
+    const int ex = owner * P + __shfl_sync(0xffffffffu, bi, owner);
+    const float s_win = __shfl_sync(0xffffffffu, bs, owner);
     if (lane == owner) {
-      taken |= 1u << (ex - e0);
+      taken |= 1u << bi;
       bi = -1;
       bv = -INFINITY;
 #pragma unroll
@@ -409,6 +401,7 @@ __device__ __forceinline__ void select_token(
         if (e0 + i < E && !((taken >> i) & 1u) && (bi < 0 || beta[i] > bv)) {
           bi = i;
           bv = beta[i];
+          bs = sc[i];
         }
     }
     ssum = __fadd_rn(ssum, s_win);
@@ -423,22 +416,29 @@ __device__ __forceinline__ void select_token(
   }
 }
 
-// Selection, and with aux_part the balance loss's per-block partials: each
-// warp writes its token's s' and raw top-K membership to shared memory, then
-// the CTA sums its 8 tokens in token order per expert -> aux_part[blk][0][e]
-// (sum of s') and aux_part[blk][1][e] (members, an exact small integer).
+// Selection, and with the balance loss (has_aux) its sums: each warp writes
+// its token's s' and raw top-K membership to shared memory; each thread then
+// adds one expert's 8 values (s' in fixed point, 2^32 units) and adds them to
+// the sequence's sums with integer atomics, so the totals do not depend on
+// the order of the CTAs.  The CTA that finds itself last of its sequence
+// (a counter taken after a fence) forms f, P and the loss from the totals,
+// which it reads and zeroes in one exchange, and resets the counter.
+constexpr float kAuxFix = 4294967296.0f;  // 2^32
+
 template <int P>
 __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
     const float* __restrict__ part, int splits, int T, int E, int G, int M, int K,
     const float* __restrict__ bias, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
-    float* __restrict__ logits_out, float* __restrict__ aux_part) {
+    float* __restrict__ logits_out, moe_balance_loss aux, int has_aux) {
   extern __shared__ float aux_sm[];  // [8][E] s', then [8][E] membership bytes
+  __shared__ float warp_term[kSelThreads / 32];
+  __shared__ int is_last;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int t = blockIdx.x * (kSelThreads / 32) + w;
   float sc[P];
   if (t < T)
     select_token<P>(part, splits, t, T, E, G, M, K, bias, idx_out, gate_out, logits_out, lane, sc);
-  if (aux_part == nullptr) return;  // the same for the whole grid
+  if (!has_aux) return;  // the same for the whole grid
   float* sp = aux_sm + w * E;
   uint8_t* sm8 = reinterpret_cast<uint8_t*>(aux_sm + (kSelThreads / 32) * E) + w * E;
   if (t < T) {
@@ -450,29 +450,65 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
     }
   }
   __syncthreads();
+  const int S = aux.seq_len;
+  const int q = blockIdx.x * (kSelThreads / 32) / S;  // 8 | S: the CTA's tokens share q
   const uint8_t* mem = reinterpret_cast<const uint8_t*>(aux_sm + (kSelThreads / 32) * E);
-  float* dst = aux_part + static_cast<int64_t>(blockIdx.x) * 2 * E;
+  unsigned long long* acc = reinterpret_cast<unsigned long long*>(aux.acc) + static_cast<int64_t>(q) * E;
+  int32_t* cnt = aux.cnt + static_cast<int64_t>(q) * E;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float acc = 0.f;
-    int cnt = 0;
+    unsigned long long a = 0;
+    int c = 0;
 #pragma unroll
     for (int j = 0; j < kSelThreads / 32; ++j) {
-      acc = __fadd_rn(acc, aux_sm[j * E + e]);
-      cnt += mem[j * E + e];
+      a += static_cast<unsigned long long>(__float2ll_rn(__fmul_rn(aux_sm[j * E + e], kAuxFix)));
+      c += mem[j * E + e];
     }
-    dst[e] = acc;
-    dst[E + e] = static_cast<float>(cnt);
+    if (a) atomicAdd(acc + e, a);
+    if (c) atomicAdd(cnt + e, c);
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    is_last = atomicAdd(aux.done + q, 1) == S / (kSelThreads / 32) - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  // f_i = E/(K S) * count, P_i = sum / S; term over this thread's experts in
+  // ascending order, then the warps' butterflies and the warp sums in order
+  float term = 0.f;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const unsigned long long a = atomicExch(acc + e, 0ull);
+    const int c = atomicExch(cnt + e, 0);
+    const float f = __fdiv_rn(static_cast<float>(E) * static_cast<float>(c),
+                              static_cast<float>(K) * static_cast<float>(S));
+    const float pv = static_cast<float>(static_cast<double>(a) / (4294967296.0 * S));
+    if (aux.f) aux.f[static_cast<int64_t>(q) * E + e] = f;
+    if (aux.P) aux.P[static_cast<int64_t>(q) * E + e] = pv;
+    term = __fadd_rn(term, __fmul_rn(f, pv));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) term = __fadd_rn(term, __shfl_xor_sync(0xffffffffu, term, off));
+  if (lane == 0) warp_term[w] = term;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSelThreads / 32; ++i) tot = __fadd_rn(tot, warp_term[i]);
+    aux.loss[q] = __fmul_rn(aux.alpha, tot);
+    aux.done[q] = 0;
   }
 }
 
 template <int P>
 void launch_select(int blocks, cudaStream_t st, const float* part, int splits, int T, int E,
                    int G, int M, int K, const float* bias, int32_t* idx, float* gate,
-                   float* logits, float* aux) {
+                   float* logits, const moe_balance_loss* aux) {
   // 8 tokens x E x (4 + 1) bytes <= 40 KB for E <= 1024
   const size_t sm = aux ? static_cast<size_t>(kSelThreads / 32) * E * 5 : 0;
+  moe_balance_loss a{};
+  if (aux) a = *aux;
   route_select_kernel<P><<<blocks, kSelThreads, sm, st>>>(part, splits, T, E, G, M, K, bias, idx,
-                                                           gate, logits, aux);
+                                                           gate, logits, a, aux ? 1 : 0);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -492,16 +528,23 @@ extern "C" moe_status moe_route_workspace_size(int T, int d, int E, size_t* byte
 extern "C" moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* centroids,
                                 const float* bias, int T, int d, int E, int G, int M, int K,
                                 int32_t* topk_idx, float* topk_gate, float* logits_out,
-                                float* aux_part, void* ws, size_t ws_bytes, int32_t* dev_err,
-                                moe_stream_t stream) {
+                                const moe_balance_loss* aux, void* ws, size_t ws_bytes,
+                                int32_t* dev_err, moe_stream_t stream) {
   using namespace moe;
   if (T < 0 || d <= 0 || E <= 0 || G <= 0 || M <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
   if (d % 128 != 0 || E % 16 != 0 || E % G != 0 || M > G || K > E || ldu < d) return MOE_ERR_SHAPE;
   if (E > 1024 || G > 32 || K > 32) return MOE_ERR_UNSUPPORTED;
   if (M < G && (K % M != 0 || M * (E / G) < K)) return MOE_ERR_SHAPE;
+  if (aux) {
+    if (aux->seq_len <= 0) return MOE_ERR_INVALID_ARG;
+    if (aux->seq_len % 8 != 0 || T % aux->seq_len != 0 || aux->seq_len > (1 << 30))
+      return MOE_ERR_SHAPE;
+  }
   if (T == 0) return MOE_OK;
   if (!u || !centroids || !bias || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
+  if (aux && (!aux->acc || !aux->cnt || !aux->done || !aux->loss)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(u) || !aligned16(centroids) || ldu % 8 != 0) return MOE_ERR_ALIGN;
+  if (aux && (reinterpret_cast<uintptr_t>(aux->acc) & 7u) != 0) return MOE_ERR_ALIGN;
   size_t need = 0;
   moe_route_workspace_size(T, d, E, &need);
   if (ws_bytes < need || (!ws && need)) return MOE_ERR_WORKSPACE;
@@ -530,13 +573,13 @@ extern "C" moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* 
 
   const int blocks = (T + kSelThreads / 32 - 1) / (kSelThreads / 32);
   const int P = (E + 31) / 32;
-  if (P <= 1) launch_select<1>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
-  else if (P <= 2) launch_select<2>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
-  else if (P <= 4) launch_select<4>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
-  else if (P <= 8) launch_select<8>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
-  else if (P <= 12) launch_select<12>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
-  else if (P <= 16) launch_select<16>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
-  else launch_select<32>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux_part);
+  if (P <= 1) launch_select<1>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux);
+  else if (P <= 2) launch_select<2>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux);
+  else if (P <= 4) launch_select<4>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux);
+  else if (P <= 8) launch_select<8>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux);
+  else if (P <= 12) launch_select<12>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux);
+  else if (P <= 16) launch_select<16>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux);
+  else launch_select<32>(blocks, st, part, r.splits, T, E, G, M, K, bias, topk_idx, topk_gate, logits_out, aux);
   MOE_CUDA_CHECK_LAUNCH();
   return MOE_OK;
 }

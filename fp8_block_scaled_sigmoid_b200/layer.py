@@ -104,7 +104,8 @@ class MoELayer:
 
     def __init__(self, cfg: MoEConfig, centroids: torch.Tensor, bias: torch.Tensor,
                  w1q, w1s, w2q, w2s, T: int | None = None, process_group=None,
-                 keep_logits: bool = False, pow2: bool = False, balance_loss: bool = False):
+                 keep_logits: bool = False, pow2: bool = False, balance_loss: bool = False,
+                 seq_len: int | None = None, alpha: float = 1e-4):
         self.cfg = cfg
         self.pow2 = pow2
         self.T = cfg.T if T is None else T
@@ -119,12 +120,13 @@ class MoELayer:
         dev = self.dev
         i32, f32, u8 = torch.int32, torch.float32, torch.uint8
         self.idx = torch.empty(T, K, dtype=i32, device=dev)
-        # router logits of the last step (keep_logits), and the balance loss's
-        # per-8-token partial sums written by the router's selection pass
-        # (balance_loss)
+        # router logits of the last step (keep_logits), and the sequence-wise
+        # balance loss the router's selection pass computes (balance_loss:
+        # sequences of seq_len tokens, default one sequence of T)
         self.logits = torch.empty(T, E, dtype=f32, device=dev) if keep_logits else None
-        self.aux_part = (torch.empty((T + 7) // 8, 2, E, dtype=f32, device=dev)
-                         if balance_loss else None)
+        self.balance = (_abi.BalanceLossState(T, E, T if seq_len is None else seq_len, alpha,
+                                              with_fp=True, device=dev)
+                        if balance_loss else None)
         self.gate = torch.empty(T, K, dtype=f32, device=dev)
         self.route_ws = torch.empty(max(_abi.moe_route_workspace_size(T, d, E), 16), dtype=u8, device=dev)
         self.Xq = torch.empty(P + T, d, dtype=u8, device=dev)
@@ -153,7 +155,7 @@ class MoELayer:
         c = self.cfg
         _abi.moe_route(u, self.centroids, self.bias, c.G, c.M, c.K, self.idx, self.gate,
                        logits_out=self.logits, ws=self.route_ws, dev_err=self.dev_err,
-                       aux_part=self.aux_part)
+                       aux=self.balance)
 
     def step_permute(self):
         """Counts, offsets, row maps and the tile table (no row moves yet)."""
@@ -302,17 +304,22 @@ class MoELayer:
         out_host.copy_(self.out, non_blocking=True)
         return out_host
 
-    def seq_balance_loss(self, seq_len: int, alpha: float = 1e-4, with_fp: bool = False):
+    def seq_balance_loss(self, seq_len: int | None = None, alpha: float | None = None,
+                         with_fp: bool = False):
         """The complementary sequence-wise balance loss (eqs. 17-20) of the
         last step's routing, per sequence of seq_len tokens.  With
-        balance_loss=True the router's selection pass already wrote the
-        per-8-token partial sums and one short reduction finishes the loss;
-        with keep_logits=True the loss is computed from the kept logits."""
-        if self.aux_part is not None:
-            return _abi.moe_seq_balance_loss_part(self.aux_part, self.T, self.cfg.K, seq_len,
-                                                  alpha, with_fp)
+        balance_loss=True the router's selection pass has already computed it
+        (for the seq_len and alpha the layer was built with); with
+        keep_logits=True it is computed from the kept logits."""
+        b = self.balance
+        if b is not None:
+            assert seq_len in (None, b.seq_len) and alpha in (None, b.alpha), \
+                "the fused loss uses the layer's seq_len and alpha"
+            loss = b.loss[:b.n_seq]
+            return (loss, b.f[:b.n_seq], b.P[:b.n_seq]) if with_fp else loss
         assert self.logits is not None, "build the layer with balance_loss or keep_logits"
-        return _abi.moe_seq_balance_loss(self.logits, self.cfg.K, seq_len, alpha, with_fp)
+        return _abi.moe_seq_balance_loss(self.logits, self.cfg.K, self.T if seq_len is None
+                                         else seq_len, 1e-4 if alpha is None else alpha, with_fp)
 
     def capture(self, u: torch.Tensor, update_bias: bool = True):
         """Record one forward step on the device input ``u`` (bf16 [T][d];

@@ -72,7 +72,7 @@ typedef void* moe_stream_t; /* cudaStream_t */
 const char* moe_status_string(moe_status s);
 
 /* ABI version of this header (bumped on any incompatible change); this
- * header is version 3. */
+ * header is version 4. */
 int moe_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -118,6 +118,37 @@ moe_status fp8_quant_128x128_pow2(const uint16_t* w, int64_t ldw, int rows, int 
                                   uint8_t* q, float* scale, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_balance_loss -- state and outputs of the complementary sequence-wise
+ * balance loss ([ANN] "Complementary Sequence-Wise Auxiliary Loss", eqs.
+ * (17)-(20)) when moe_route computes it in its selection pass.  For each
+ * sequence q of seq_len consecutive tokens:
+ *   L_q = alpha * sum_i f_i P_i,  f_i = E/(K S) * #{t : i in TopK_K(s_t)},
+ *   P_i = (1/S) sum_t s'_{i,t},   s'_{i,t} = s_{i,t} / sum_j s_{j,t},
+ * the TopK over the raw affinities of all E experts (no bias, no group
+ * limit, ties to the lower index, K the routing K).  Each block of 8 tokens
+ * adds its sums with integer atomics -- s' in fixed point with 32 fraction
+ * bits, so the sum does not depend on the order of the additions and the
+ * result is deterministic -- and the last block of a sequence forms f, P and
+ * the loss (a fixed-order tree over the experts) and zeroes the sequence's
+ * state again.  The caller owns every buffer:
+ *   acc   int64 [T/seq_len][E], cnt int32 [T/seq_len][E], done int32
+ *         [T/seq_len]: all zero before the first call (cudaMemset); every
+ *         call leaves them zero.  One state serves one call at a time.
+ *   loss  fp32 [T/seq_len];  f, P fp32 [T/seq_len][E] or NULL.
+ * Limits: seq_len % 8 == 0, T % seq_len == 0, seq_len <= 2^30.
+ */
+typedef struct moe_balance_loss {
+  int seq_len;
+  float alpha;
+  int64_t* acc;
+  int32_t* cnt;
+  int32_t* done;
+  float* loss;
+  float* f;
+  float* P;
+} moe_balance_loss;
+
+/* ---------------------------------------------------------------------------
  * moe_route -- sigmoid router with bias-based, group-limited top-K selection.
  * [ANN] eqs. (13)-(16): s_{i,t} = Sigmoid(u_t . e_i); the top-K is taken over
  * s_{i,t} + b_i, the gate g_{i,t} = s_{i,t} / sum of the chosen s; "Node-
@@ -129,14 +160,8 @@ moe_status fp8_quant_128x128_pow2(const uint16_t* w, int64_t ldw, int rows, int 
  *   u          bf16 [T][ldu];  centroids bf16 [E][d];  bias fp32 [E]
  *   topk_idx   int32 [T][K];   topk_gate fp32 [T][K]
  *   logits_out fp32 [T][E] or NULL (the logits the selection used)
- *   aux_part   fp32 [ceil(T/8)][2][E] or NULL: the complementary sequence-wise
- *              balance loss's partial sums ([ANN] eqs. (17)-(20)), computed from
- *              the same affinities in the same pass.  For each block b of 8
- *              tokens (8b .. 8b+7): [b][0][i] = the sum over its tokens of
- *              s'_{i,t} = s_{i,t} / sum_j s_{j,t}, [b][1][i] = how many of them
- *              have expert i in their raw top-K (over all E experts, no bias,
- *              no group limit, ties to the lower index, K the routing K).
- *              moe_seq_balance_loss_part turns them into the loss.
+ *   aux        NULL, or the balance loss to compute from the same affinities
+ *              in the same pass (see moe_balance_loss)
  *   ws         scratch of moe_route_workspace_size() bytes (may be NULL if 0)
  * Limits: d % 128 == 0, E % 16 == 0, 16 <= E <= 1024, E % G == 0,
  * 1 <= M <= G <= 32, K <= E, K % M == 0 when M < G, K <= 32.
@@ -145,8 +170,8 @@ moe_status moe_route_workspace_size(int T, int d, int E, size_t* bytes);
 moe_status moe_route(const uint16_t* u, int64_t ldu, const uint16_t* centroids,
                      const float* bias, int T, int d, int E, int G, int M, int K,
                      int32_t* topk_idx, float* topk_gate, float* logits_out,
-                     float* aux_part, void* ws, size_t ws_bytes, int32_t* dev_err,
-                     moe_stream_t stream);
+                     const moe_balance_loss* aux, void* ws, size_t ws_bytes,
+                     int32_t* dev_err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * moe_permute -- local permutation of (token, expert) pairs by expert, the
@@ -490,19 +515,6 @@ moe_status moe_seq_balance_loss_workspace_size(int T, int E, int seq_len, size_t
 moe_status moe_seq_balance_loss(const float* logits, int T, int E, int K, int seq_len,
                                 float alpha, float* loss, float* f, float* P, void* ws,
                                 size_t ws_bytes, moe_stream_t stream);
-
-/* moe_seq_balance_loss_part -- the same loss from the per-8-token partial
- * sums that moe_route wrote to aux_part (the token pass fused into the
- * router's selection; two short reductions follow).  Per sequence the
- * partials are added in a fixed order (deterministic); the result equals
- * moe_seq_balance_loss's up to the order of the fp32 sums.  f and P may be
- * NULL.  ws: moe_seq_balance_loss_part_workspace_size bytes.
- * Limits: T % seq_len == 0, seq_len % 8 == 0, K <= min(E, 32), E <= 1024;
- * K must be the routing K the partials were made with. */
-moe_status moe_seq_balance_loss_part_workspace_size(int T, int E, int seq_len, size_t* bytes);
-moe_status moe_seq_balance_loss_part(const float* aux_part, int T, int E, int K, int seq_len,
-                                     float alpha, float* loss, float* f, float* P, void* ws,
-                                     size_t ws_bytes, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * moe_fp8_mma_peak -- measurement helper: the dense FP8 tensor-core rate of

@@ -12,6 +12,17 @@ from fp8_block_scaled_sigmoid_b200 import _abi
 HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "moefp8.h")
 
 
+_BL = []
+
+
+def _bl(seq_len):
+    """Address of a moe_balance_loss with the given seq_len and NULL buffers
+    (kept alive for the test session)."""
+    b = _abi._BalanceLoss(seq_len, 1e-4, None, None, None, None, None, None)
+    _BL.append(b)
+    return ctypes.addressof(b)
+
+
 def _declared():
     src = open(HEADER).read()
     return sorted(set(re.findall(r"^(?:moe_status|int|const char\*)\s+(\w+)\(", src, re.M)))
@@ -24,7 +35,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(_abi.exported_symbols())
-    assert L.moe_abi_version() == 3
+    assert L.moe_abi_version() == 4
 
 
 def test_status_strings():
@@ -54,12 +65,12 @@ def test_max_m_tiles_bound():
                            None, None, 0, None, None), 2),                    # K % M
     (lambda L: L.moe_route(None, 256, None, None, 8, 256, 2048, 8, 4, 8, None, None, None,
                            None, None, 0, None, None), 4),                    # E > 1024
-    (lambda L: L.moe_seq_balance_loss_part(None, 96, 16, 4, 30, ctypes.c_float(1e-4), None,
-                                           None, None, None, 0, None), 2),   # T % seq_len
-    (lambda L: L.moe_seq_balance_loss_part(None, 100, 16, 4, 50, ctypes.c_float(1e-4), None,
-                                           None, None, None, 0, None), 2),   # seq_len % 8
-    (lambda L: L.moe_seq_balance_loss_part(None, 96, 16, 4, 48, ctypes.c_float(1e-4), None,
-                                           None, None, None, 0, None), 1),   # NULL partials
+    (lambda L: L.moe_route(None, 256, None, None, 96, 256, 16, 4, 2, 4, None, None, None,
+                           _bl(30), None, 0, None, None), 2),                # T % seq_len
+    (lambda L: L.moe_route(None, 256, None, None, 100, 256, 16, 4, 2, 4, None, None, None,
+                           _bl(50), None, 0, None, None), 2),                # seq_len % 8
+    (lambda L: L.moe_route(None, 256, None, None, 96, 256, 16, 4, 2, 4, None, None, None,
+                           _bl(0), None, 0, None, None), 1),                 # seq_len 0
     (lambda L: L.grouped_gemm_fp8_blockscaled(None, None, 10, None, None, None, None, None,
                                               None, 4, 1, 384, 128, 0, None, None, None,
                                               None, None, None), 2),          # N % 256

@@ -1,4 +1,6 @@
-"""GPU parity of moe_seq_balance_loss against the oracle.
+"""GPU parity of the sequence-wise balance loss against the oracle: the
+three-pass form from logits (moe_seq_balance_loss) and the form fused into
+moe_route's selection pass (moe_balance_loss).
 
 "DeepSeek_V3_Report：Annotation", "Complementary Sequence-Wise Auxiliary
 Loss", eqs. (17)-(20).  The oracle runs on the GPU's own fp32 logits:
@@ -66,23 +68,27 @@ def test_layer_seq_balance_loss(cuda_dev):
     cfg = configs.TINY
     w1q, w1s, w2q, w2s = make_fp8_weights(cfg, cuda_dev)
     layer = MoELayer(cfg, inputs.draw_centroids(cfg, cuda_dev), inputs.draw_bias(cfg, cuda_dev),
-                     w1q, w1s, w2q, w2s, keep_logits=True, balance_loss=True)
+                     w1q, w1s, w2q, w2s, keep_logits=True, balance_loss=True,
+                     seq_len=cfg.T // 2)
     layer.forward(inputs.draw_u(cfg, cuda_dev))
-    loss = layer.seq_balance_loss(cfg.T // 2)
+    loss = layer.seq_balance_loss().clone()
+    loss3 = _abi.moe_seq_balance_loss(layer.logits, cfg.K, cfg.T // 2)
     torch.cuda.synchronize()
     lo, _, _, margin = O.seq_balance_loss(npraw(layer.logits).astype(np.float64), cfg.K,
                                           cfg.T // 2, 1e-4)
     clean = (margin < 1e-6).reshape(2, -1).sum(axis=1) == 0
     assert np.allclose(npraw(loss)[clean], lo[clean], rtol=1e-4, atol=0)
+    assert torch.allclose(loss, loss3, rtol=1e-5, atol=0)
 
 
-@pytest.mark.parametrize("cfg_name,S", [("tiny", 64), ("v3_prefill", 4096), ("v3_prefill", 1024),
-                                        ("v4_pro", 2048)])
-def test_route_fused_partials_match_three_pass(cuda_dev, cfg_name, S):
-    """The token pass fused into the router's selection (per-8-token partial
-    sums) gives the three-pass loss on the same logits: the membership counts
-    (hence f) exactly, P and the loss up to the order of the fp32 sums; the
-    routing itself is unchanged."""
+@pytest.mark.parametrize("cfg_name,S", [("tiny", 64), ("tiny", 8), ("v3_prefill", 4096),
+                                        ("v3_prefill", 1024), ("v4_pro", 2048)])
+def test_route_fused_loss_matches_three_pass(cuda_dev, cfg_name, S):
+    """The loss fused into the router's selection (integer sums, the last
+    block of each sequence finishes it) gives the three-pass loss on the same
+    logits: the membership counts (hence f) exactly, P and the loss up to the
+    rounding of the sums; the routing itself is unchanged; two calls give
+    the same bits and leave the state zeroed."""
     from fp8_block_scaled_sigmoid_b200 import configs, inputs
     cfg = configs.PRESETS[cfg_name]
     if cfg.T > 4096:
@@ -91,21 +97,26 @@ def test_route_fused_partials_match_three_pass(cuda_dev, cfg_name, S):
     cent = inputs.draw_centroids(cfg, cuda_dev)
     bias = inputs.draw_bias(cfg, cuda_dev)
     logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=cuda_dev)
-    part = torch.empty((cfg.T + 7) // 8, 2, cfg.E, dtype=torch.float32, device=cuda_dev)
-    idx, gate = _abi.moe_route(u, cent, bias, cfg.G, cfg.M, cfg.K, logits_out=logits,
-                               aux_part=part)
-    idx2, gate2 = _abi.moe_route(u, cent, bias, cfg.G, cfg.M, cfg.K)
-    la, fa, Pa = _abi.moe_seq_balance_loss_part(part, cfg.T, cfg.K, S, with_fp=True)
-    la2 = _abi.moe_seq_balance_loss_part(part, cfg.T, cfg.K, S)
+    st = _abi.BalanceLossState(cfg.T, cfg.E, S, 1e-4, with_fp=True, device=cuda_dev)
+    idx, gate = _abi.moe_route(u, cent, bias, cfg.G, cfg.M, cfg.K, logits_out=logits, aux=st)
+    la, fa, Pa = st.loss.clone(), st.f.clone(), st.P.clone()
+    idx2, gate2 = _abi.moe_route(u, cent, bias, cfg.G, cfg.M, cfg.K, aux=st)
+    idx3, gate3 = _abi.moe_route(u, cent, bias, cfg.G, cfg.M, cfg.K)
     lb, fb, Pb = _abi.moe_seq_balance_loss(logits, cfg.K, S, with_fp=True)
     torch.cuda.synchronize()
-    assert torch.equal(idx, idx2) and torch.equal(gate, gate2)   # routing unchanged
-    assert torch.equal(la, la2), "not deterministic"
+    assert torch.equal(idx, idx3) and torch.equal(gate, gate3)   # routing unchanged
+    assert torch.equal(idx2, idx3) and torch.equal(gate2, gate3)
+    assert torch.equal(la, st.loss) and torch.equal(fa, st.f) and torch.equal(Pa, st.P), \
+        "not deterministic"
+    assert not st.acc.any() and not st.cnt.any() and not st.done.any(), "state not zeroed"
     assert torch.equal(fa, fb)
     # every token counts K members
-    assert torch.all(part[:, 1, :].sum(1) == 8 * cfg.K)
-    assert torch.allclose(Pa, Pb, rtol=1e-5, atol=1e-9)
-    assert torch.allclose(la, lb, rtol=1e-5, atol=0)
+    assert torch.all(torch.round(fa * cfg.K * S / cfg.E).sum(1) == cfg.K * S)
+    # the three-pass P is an fp32 sum over 32-token chunks and then over the
+    # chunks: up to (32 + S/32) roundings of 2^-24 relative
+    tol = (32 + S / 32) * 2.0 ** -24
+    assert torch.allclose(Pa, Pb, rtol=tol, atol=1e-9)
+    assert torch.allclose(la, lb, rtol=tol, atol=0)
     # and against the oracle on the same logits
     lo, fo, Po, margin = O.seq_balance_loss(npraw(logits).astype(np.float64), cfg.K, S, 1e-4)
     near = (margin < 1e-6).reshape(-1, S).sum(axis=1)
