@@ -92,6 +92,17 @@ struct GemmArgs {
   int32_t* sched;         // work counter (zeroed before the launch), NULL: static schedule
 };
 
+// Tensor maps of A with boxes of 32, 64, 96 and 128 rows: an m-tile loads
+// only the 32-row groups that hold its rows (the MMA still reads 128 rows;
+// the rest of the stage holds older bytes, whose results land in rows that
+// are never written out).
+struct ATmaps {
+  CUtensorMap box[4];
+};
+
+// index of the smallest A box holding `rows` rows
+__device__ __forceinline__ int a_box(int rows) { return min(3, max(0, (rows - 1) >> 5)); }
+
 struct Work {
   int e, n_idx, row0, rows;  // expert, n-tile, first row and valid rows of the m-tile
   bool ok;
@@ -505,7 +516,7 @@ __device__ __forceinline__ Ctl carve(uint8_t* base, int ctl_off = kRingBytes) {
 // A rows and the weight tile into the stage ring; waits for its own copies
 // before returning.
 template <int STAGES, int SK>
-__device__ __forceinline__ void tma_producer(const CUtensorMap& tmA, const CUtensorMap& tmB,
+__device__ __forceinline__ void tma_producer(const ATmaps& tmA, const CUtensorMap& tmB,
                                              const GemmArgs& args, const Ctl& c, uint8_t* base,
                                              int total, int nN, int KB, volatile int* abort_v) {
   constexpr int kSub = kBK / SK;
@@ -520,6 +531,8 @@ __device__ __forceinline__ void tma_producer(const CUtensorMap& tmA, const CUten
       continue;
     }
     const int brow = t.e * N + t.n_idx * kBN;
+    const int ab = a_box(t.rows);
+    const uint32_t bytes = static_cast<uint32_t>((ab + 1) * 32 * SK + kBN * SK);
     for (int kk = 0; kk < KB * kSub; ++kk, ++it) {
       const int s = it % STAGES;
       const uint32_t ph = (it / STAGES) & 1;
@@ -528,8 +541,8 @@ __device__ __forceinline__ void tma_producer(const CUtensorMap& tmA, const CUten
         break;
       }
       uint8_t* sA = base + s * kStage;
-      mbar_arrive_expect_tx(&c.full[s], kStage);
-      tma_load_2d(sA, &tmA, &c.full[s], kk * SK, t.row0);
+      mbar_arrive_expect_tx(&c.full[s], bytes);
+      tma_load_2d(sA, &tmA.box[ab], &c.full[s], kk * SK, t.row0);
       tma_load_2d(sA + kA, &tmB, &c.full[s], kk * SK, brow);
     }
   }
@@ -555,7 +568,7 @@ struct WorkQueue {
 
 template <int EP, int SK>
 __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
-    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const __grid_constant__ ATmaps tmA, const __grid_constant__ CUtensorMap tmB,
     const GemmArgs args) {
   constexpr int kSub = kBK / SK;                 // stages per K block
   constexpr int kA = kBM * SK, kB = kBN * SK;    // stage bytes of A and B
@@ -605,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
     mbar_init(&c.xbar[1], kEpiThreads);
     *c.abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tmA);
+    for (int b = 0; b < 4; ++b) prefetch_tmap(&tmA.box[b]);
     prefetch_tmap(&tmB);
   }
   if (warp == 2) load_tile_prefix(args, c.rstart, lane);
@@ -639,6 +652,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
           continue;
         }
         const int brow = t.e * N + t.n_idx * kBN;
+        const int ab = a_box(t.rows);
+        const uint32_t bytes = static_cast<uint32_t>((ab + 1) * 32 * SK + kB);
         for (int kk = 0; kk < KB * kSub; ++kk, ++it) {
           const int s = it % kStages;
           if (!mbar_wait(&c.empty[s], ((it / kStages) & 1) ^ 1, abort_v, args.dev_err)) {
@@ -646,8 +661,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm1sm_kernel(
             break;
           }
           uint8_t* sA = base + s * kStage;
-          mbar_arrive_expect_tx(&c.full[s], kStage);
-          tma_load_2d(sA, &tmA, &c.full[s], kk * SK, t.row0);
+          mbar_arrive_expect_tx(&c.full[s], bytes);
+          tma_load_2d(sA, &tmA.box[ab], &c.full[s], kk * SK, t.row0);
           tma_load_2d(sA + kA, &tmB, &c.full[s], kk * SK, brow);
         }
       }
@@ -894,7 +909,7 @@ __device__ __forceinline__ bool epilogue_mx_tile(const GemmArgs& args, const Wor
 // Stages are whole 128-wide K blocks.
 template <int EP>
 __global__ void __launch_bounds__(kThreads, 1) gemm_pow2_kernel(
-    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const __grid_constant__ ATmaps tmA, const __grid_constant__ CUtensorMap tmB,
     const GemmArgs args) {
   constexpr int kA = kBM * kBK, kB = kBN * kBK;
   constexpr int kStage = kA + kB;
@@ -921,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pow2_kernel(
     mbar_init(&c.xbar[1], kEpiThreads);
     *c.abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tmA);
+    for (int b = 0; b < 4; ++b) prefetch_tmap(&tmA.box[b]);
     prefetch_tmap(&tmB);
   }
   if (warp == 2) load_tile_prefix(args, c.rstart, lane);
@@ -1223,9 +1238,13 @@ moe_status gemm_launch(bool pow2, const uint8_t* A, const float* sa, int64_t a_r
   const int SK = pow2 ? kBK : MOE_GEMM_SK;
   // A: 128-row boxes; B: the 256 weight rows of a tile; boxes are SK bytes
   // wide with an SK-byte swizzle
-  CUtensorMap tmA, tmB;
-  if (!moe_make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, a_rows, K, SK, kBM, SK) ||
-      !moe_make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K,
+  ATmaps tmA;
+  CUtensorMap tmB;
+  for (int b = 0; b < 4; ++b)
+    if (!moe_make_tmap_2d(&tmA.box[b], A, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, a_rows, K, SK,
+                          32 * (b + 1), SK))
+      return MOE_ERR_CUDA;
+  if (!moe_make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, K,
                         static_cast<uint64_t>(groups) * N, K, SK, kBN, SK))
     return MOE_ERR_CUDA;
   GemmArgs a;
