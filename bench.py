@@ -89,6 +89,7 @@ class ClockSampler:
         self.stop_flag = False
         self.win = None
         self.max_mhz = None
+        self.handle = None
 
     def _nvml_handle(self):
         import pynvml
@@ -116,6 +117,23 @@ class ClockSampler:
                 pass
             time.sleep(0.002)
 
+    def sample_until(self, done) -> None:
+        """Poll from the calling thread until done() is true (the GPU work of
+        the timed region has drained): the region's samples do not depend on
+        the polling thread being scheduled while the host enqueues."""
+        if self.nvml is None or self.handle is None:
+            return
+        pynvml, h = self.nvml, self.handle
+        while not done():
+            try:
+                self.samples.append((time.perf_counter(),
+                                     pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                     pynvml.nvmlDeviceGetCurrentClocksEventReasons(h),
+                                     pynvml.nvmlDeviceGetPowerUsage(h)))
+            except Exception:  # noqa: BLE001
+                return
+            time.sleep(0.001)
+
     def window(self, t0: float, t1: float):
         """Keep only samples taken between t0 and t1 (time.perf_counter)."""
         self.win = (t0, t1)
@@ -125,6 +143,7 @@ class ClockSampler:
         try:
             pynvml, h = self._nvml_handle()
             self.nvml = pynvml
+            self.handle = h
             self.thread = threading.Thread(target=self._poll, args=(pynvml, h), daemon=True)
             self.thread.start()
             return
@@ -403,6 +422,8 @@ def run_gpu(args):
         e[6].record(st)
         layer.step_bias_update()
         e[7].record(st)
+    if sampler:
+        sampler.sample_until(ev[-1][-1].query)
     barrier()
     t_hi = time.perf_counter()
     launches = _abi.launch_count - lc0
@@ -429,6 +450,8 @@ def run_gpu(args):
             gev[i][0].record(st)
             graph.replay()
             gev[i][1].record(st)
+        if sampler:
+            sampler.sample_until(gev[-1][1].query)
         barrier()
         t_hi = time.perf_counter()
         layer.check()
@@ -725,6 +748,7 @@ def run_gemm(args):
         e0.record()
         _abi.grouped_gemm_fp8_blockscaled(aq, sa, bq, sb, offs, tg, ts, nt, mt, D=D, pow2=args.pow2)
         e1.record()
+        sampler.sample_until(e1.query)
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
     clocks = sampler.stop()
@@ -793,6 +817,8 @@ def run_ep(args, cfg, cfg_rank, dev, pg, world, rank, local):
         e0.record(st)
         layer.forward(u)
         e1.record(st)
+        if sampler:
+            sampler.sample_until(e1.query)
         e1.synchronize()   # the next step's dispatch plan reads its split sizes on the host
         total += e0.elapsed_time(e1)
     barrier()
@@ -872,6 +898,7 @@ def run_backward(args):
         lc0 = _abi.launch_count
         layer.backward(dout, mark=mark)
         launches += _abi.launch_count - lc0
+        sampler.sample_until(ev[-1].query)
         torch.cuda.synchronize()
         for j, n in enumerate(names):
             per[n] += ev[j].elapsed_time(ev[j + 1])
