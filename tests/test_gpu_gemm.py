@@ -128,12 +128,14 @@ def test_combine(cuda_dev):
 def test_tail_tiles_and_dynamic_schedule(cuda_dev, ep):
     """m-tiles of at most 32 rows (an expert's rows past a whole 128-row
     tile, or an expert with few rows) take the transposed tail path; every
-    tail size from 1 to 33 rows and a few whole tiles are checked against the
-    oracle on the same FP8 operands.  The dynamic schedule (a work counter)
+    tail size from 1 to 33 rows, partial tiles of every A box size and a few
+    whole tiles are checked against the oracle on the same FP8 operands.  The dynamic schedule (a work counter)
     gives the same bytes as the static one."""
     K, N = 1024, 512
+    # also every A box size (a partial m-tile loads 32, 64, 96 or 128 rows):
+    # 63/64/65, 96/97 and their repeats past a whole tile
     counts = [1, 2, 7, 16, 17, 31, 32, 33, 0, 128 + 1, 128 + 31, 128 + 32, 128 + 33, 256 + 5, 64,
-              100, 127, 128]
+              100, 127, 128, 63, 65, 96, 97, 128 + 64, 128 + 65, 128 + 96, 128 + 97]
     G = len(counts)
     rows = sum(counts)
     aq, sa, bq, sb = _quantised_operands(cuda_dev, rows, K, G, N, seed=77)

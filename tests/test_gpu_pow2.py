@@ -63,6 +63,7 @@ def _tables(dev, offsets, max_tiles):
     (128, 256, [1], 0),
     (384, 512, [0, 1, 130, 300, 17], 0),
     (640, 256, [129, 0, 255], 3),
+    (512, 256, [31, 32, 33, 64, 65, 96, 97, 160, 225], 0),   # every A box size
     (1024, 768, [5, 0, 0, 256, 129], 10),
     (7168, 512, [200, 60], 0),
 ])
