@@ -399,6 +399,10 @@ def run_gpu(args):
     # K CUDA-graph replays of the step are timed as the headline instead)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
           for _ in range(args.steps)]
+    # the bias the timed steps start from: their routing is replayed after the
+    # timed region to count each step's active experts (the bias update moves
+    # the routing from step to step)
+    bias_t0 = layer.bias.clone()
     if not use_graph:
         start_sampler()
     barrier()
@@ -429,6 +433,20 @@ def run_gpu(args):
     launches = _abi.launch_count - lc0
     layer.check()
     step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
+    gemm1_ms = [ev[i][4].elapsed_time(ev[i][5]) for i in range(args.steps)]
+    gemm2_ms = [ev[i][5].elapsed_time(ev[i][6]) for i in range(args.steps)]
+    # untimed replay of the timed steps' routing (same bias sequence, same
+    # inputs, deterministic): the experts each step's GEMMs streamed
+    bias_t1 = layer.bias.clone()
+    layer.bias.copy_(bias_t0)
+    step_counts = []
+    for i in range(args.steps):
+        layer.step_route(u)
+        layer.step_permute()
+        step_counts.append(layer.perm["counts"].clone())
+        layer.step_bias_update()
+    layer.bias.copy_(bias_t1)
+    step_counts = [c.cpu() for c in step_counts]
     per_kernel = {n: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)) / args.steps
                   for j, n in enumerate(names)}
     eager_ms = max_over_ranks(sum(step_ms), dev, pg)
@@ -528,9 +546,11 @@ def run_gpu(args):
                     "how": "device time per call, 10+ calls replayed from one CUDA graph"}
     del logits, bstate, rws, bl_ws
 
-    # roofline of the dominant kernel (grouped GEMM 1 with the SwiGLU epilogue)
-    counts = layer.perm["counts"].cpu()
-    active = int((counts > 0).sum()) + cfg.n_shared
+    # roofline of the dominant kernel (grouped GEMM 1 with the SwiGLU epilogue):
+    # algorithmic bytes of each timed step (its own active experts) over the
+    # GEMM's total time in those steps
+    counts = step_counts[-1]
+    active = sum(int((c > 0).sum()) + cfg.n_shared for c in step_counts) / len(step_counts)
     rows = cfg.pairs + cfg.T
     w1_bytes = active * 2 * cfg.I * cfg.d * (1 + 4.0 / (128 * 128))
     a_bytes = rows * cfg.d * (1 + 4.0 / 128)
@@ -540,8 +560,8 @@ def run_gpu(args):
     g2_bytes = w2_bytes + rows * cfg.I * (1 + 4.0 / 128) + rows * cfg.d * 4
     g1_flops = 2.0 * rows * cfg.d * 2 * cfg.I
     g2_flops = 2.0 * rows * cfg.I * cfg.d
-    t1 = per_kernel["gemm1"] / 1e3
-    t2 = per_kernel["gemm2"] / 1e3
+    t1 = sum(gemm1_ms) / len(gemm1_ms) / 1e3
+    t2 = sum(gemm2_ms) / len(gemm2_ms) / 1e3
     peaks, peak_src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     fp8 = measure_fp8_peak(dev, args.pow2)
@@ -614,7 +634,10 @@ def run_gpu(args):
         "memory_kernels": memory_kernels,
         "seq_balance_loss": balance_loss,
         "loads": {"max": int(counts.max()), "mean": float(counts.float().mean()),
-                  "active_experts": active - cfg.n_shared},
+                  "active_experts": round(active - cfg.n_shared, 1),
+                  "how": "routing of the timed steps, replayed untimed from their starting "
+                         "bias; max and mean of the last step, active experts averaged over "
+                         "the steps"},
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
