@@ -433,8 +433,9 @@ def run_gpu(args):
     launches = _abi.launch_count - lc0
     layer.check()
     step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
-    gemm1_ms = [ev[i][4].elapsed_time(ev[i][5]) for i in range(args.steps)]
-    gemm2_ms = [ev[i][5].elapsed_time(ev[i][6]) for i in range(args.steps)]
+    j1, j2 = names.index("gemm1"), names.index("gemm2")
+    gemm1_ms = [ev[i][j1].elapsed_time(ev[i][j1 + 1]) for i in range(args.steps)]
+    gemm2_ms = [ev[i][j2].elapsed_time(ev[i][j2 + 1]) for i in range(args.steps)]
     # untimed replay of the timed steps' routing (same bias sequence, same
     # inputs, deterministic): the experts each step's GEMMs streamed
     bias_t1 = layer.bias.clone()
