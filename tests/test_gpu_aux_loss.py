@@ -123,3 +123,26 @@ def test_route_fused_loss_matches_three_pass(cuda_dev, cfg_name, S):
     assert np.allclose(npraw(Pa), Po, rtol=1e-4, atol=1e-7)
     clean = near == 0
     assert np.allclose(npraw(la)[clean], lo[clean], rtol=1e-4, atol=0)
+
+
+def test_fused_loss_in_a_cuda_graph(cuda_dev):
+    """The fused loss's state zeroes itself, so a step captured in a CUDA
+    graph gives the eager step's loss on every replay (same bits), and the
+    state is zero after each."""
+    from fp8_block_scaled_sigmoid_b200 import MoELayer, configs, inputs, make_fp8_weights
+    cfg = configs.TINY
+    w1q, w1s, w2q, w2s = make_fp8_weights(cfg, cuda_dev)
+    layer = MoELayer(cfg, inputs.draw_centroids(cfg, cuda_dev), inputs.draw_bias(cfg, cuda_dev),
+                     w1q, w1s, w2q, w2s, balance_loss=True, seq_len=cfg.T // 4)
+    u = inputs.draw_u(cfg, cuda_dev)
+    layer.forward(u, update_bias=False)
+    eager = layer.seq_balance_loss().clone()
+    graph, _ = layer.capture(u, update_bias=False)
+    b = layer.balance
+    for _ in range(2):
+        b.loss.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(b.loss[:b.n_seq], eager)
+        assert not b.acc.any() and not b.cnt.any() and not b.done.any()
+    del graph
