@@ -18,7 +18,10 @@
 //     on the device from the segment offsets and the tile table's per-expert
 //     tile prefix, so the ragged expert segments need no host
 //     synchronisation; the m-tiles of one expert that share a weight tile run
-//     next to each other for L2 reuse.
+//     next to each other for L2 reuse.  With a caller work counter the items
+//     are handed out dynamically; an m-tile of at most 32 rows is computed
+//     transposed (the weight tile's halves as M, its rows as N), and a
+//     partial m-tile loads only the 32-row groups of A that hold its rows.
 //
 // The shared-memory ring is staged in K slices of SK bytes (128, or 64 with
 // the 64-byte swizzle): a stage is released as soon as the MMAs of its slice

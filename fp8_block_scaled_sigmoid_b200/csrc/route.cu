@@ -11,7 +11,10 @@
 //  2. route_select_kernel -- one warp per token, experts spread over lanes,
 //     everything in registers and warp shuffles: sigmoid, biased scores,
 //     group scores (sum of each group's top K/M), top-M groups, top-K experts
-//     within them (ties to the lower index), gates from the raw scores.
+//     within them (ties to the lower index), gates from the raw scores.  With
+//     a moe_balance_loss state it also computes the complementary
+//     sequence-wise balance loss ("Complementary Sequence-Wise Auxiliary
+//     Loss", eqs. (17)-(20)) from the same affinities.
 #include <algorithm>
 #include <climits>
 
