@@ -4,10 +4,11 @@
                     [--impl reference] [--no-cpu-baseline] [--graph] [--pow2] [--ep]
                     [--gemm | --backward]
 
-One step = one forward pass of the whole layer (route, 1x128 quantisation,
-permutation, grouped GEMM 1 with fused SwiGLU + requantisation, grouped
-GEMM 2, combine, bias update) over one batch of T tokens, with the FP8
-weights already resident (they are quantised once, before timing).  With N
+One step = one forward pass of the whole layer (route, the permutation's
+index tables, the 1x128 quantisation with the dispatch's row scatter fused in,
+grouped GEMM 1 with fused SwiGLU + requantisation, grouped GEMM 2, combine,
+bias update) over one batch of T tokens, with the FP8 weights already
+resident (they are quantised once, before timing).  With N
 GPUs (torchrun, one process per GPU) every rank runs its own batch of T
 tokens over the full expert set and the per-expert load counts are summed
 with an NCCL all-reduce before the bias update (weak scaling).
@@ -16,7 +17,12 @@ Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; between steps a 512 MB buffer is overwritten to
 flush the 126 MB L2 (outside the events).  The reported time is the max over
 ranks of the summed step times.  Clocks are polled through NVML every 2 ms
-during the timed region.
+during the timed region.  The dominant GEMM's roofline counts each timed
+step's own active experts (their routing is replayed untimed afterwards).
+The end-to-end figure (e2e) runs the same steps through
+MoELayer.forward_host_stream from pinned host buffers, the copies inside the
+timed region.  The sequence-wise balance loss, fused into the router's
+selection, is timed on its own (graph-replayed calls).
 
 ``--impl reference`` times the CPU oracle instead (rank 0 only) on a bounded
 sample of the same workload and prints the same JSON line with
