@@ -600,13 +600,22 @@ def run_gpu(args):
     Tn, dn = cfg.T, cfg.d
     q_bytes = Tn * dn * 2 + (cfg.pairs + Tn) * dn * (1 + 4.0 / 128)
     c_bytes = Tn * ((cfg.K + 1) * 4 * dn + 2 * dn + 4 * dn)
+    r_bytes = Tn * dn * 2 + cfg.E * dn * 2 + Tn * cfg.K * 8
     tq, tc = per_kernel["quant"] / 1e3, per_kernel["combine"] / 1e3
+    tr = per_kernel["route"] / 1e3
     memory_kernels = {
         "quant_scatter": {"bytes": int(q_bytes), "gbs": round(q_bytes / tq / 1e9, 1),
                           "frac": round(q_bytes / tq / 1e9 / hbm, 4)},
         "combine": {"bytes": int(c_bytes), "gbs": round(c_bytes / tc / 1e9, 1),
                     "frac": round(c_bytes / tc / 1e9 / hbm, 4)},
         "permute_index_us": round(per_kernel["permute"] * 1e3, 1),
+        # the router: u and the centroids read once, the indices and gates
+        # written; its logits GEMM is a bf16 tensor-core product (2·T·E·d)
+        "route": {"bytes": int(r_bytes), "gbs": round(r_bytes / tr / 1e9, 1),
+                  "frac": round(r_bytes / tr / 1e9 / hbm, 4),
+                  "bf16_tflops": round(2.0 * Tn * cfg.E * dn / tr / 1e12, 1),
+                  "note": "logits GEMM (bf16 tensor cores, split over K) + one warp per token "
+                          "selection; bound by the selection's instruction issue, not HBM"},
         "peak": hbm, "unit": "GB/s"}
     gemm = {"gemm1_tflops": round(g1_flops / t1 / 1e12, 1),
             "gemm2_tflops": round(g2_flops / t2 / 1e12, 1),
